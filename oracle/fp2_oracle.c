@@ -1,0 +1,290 @@
+/*
+ * fp2_oracle.c -- plain CPU oracle of block-sparse prefill attention with a
+ * block-mean score estimator, a max-relative threshold and a mean correction
+ * (the method described in "FlashPrefill V2: Block-Sparse Prefill Attention for
+ * Long-Context LLM Serving", lode.cx write-up, section "How It Works"; the
+ * aimodeling.com write-up, section "From Prototype to Production").
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check and the CPU
+ * baseline leg of the benchmark may load this file.  It shares no code, header
+ * or constant with the CUDA library; the two meet only through the seeded
+ * inputs.  All arithmetic is IEEE double (no fast-math), one plain loop per
+ * definition below, no blocking or fusion beyond what the definition states.
+ * OpenMP only splits independent (q-block, head) rows across host cores.
+ *
+ * Definitions (the pages give them in words only; where they are silent the
+ * plainest reading is taken and named):
+ *   D0 blocks   Request b of length L_b is cut into blocks of Bs rows starting
+ *               at its first token ("fixed-size blocks", 345tool.com page,
+ *               section "Why block-sparse attention for prefill?"; stuffinsider
+ *               page, "Technical Details").  n_j = rows of block j.  Token r sees
+ *               tokens c <= r of the same request (causal prefill).
+ *   D1 estimate xbar_j = (1/n_j) sum_{r in j} x_r for x in {q, k, v}
+ *               (reading of "computes a small sample of attention scores" /
+ *               "estimating scores at the block level": block means), and
+ *               s[h,i,j] = tau * qbar[h,i] . kbar[g(h),j] for j <= i, g(h) = h / G.
+ *   D2 keep     m = max_{j<=i} s[h,i,j]; head h keeps j iff s - m >= ln(alpha)
+ *               ("finds the maximum, and attends only to tokens that exceed a
+ *               threshold relative to that max"; read in the probability domain,
+ *               exp(s - m) >= alpha).  A KV group keeps the union over its
+ *               heads plus the diagonal block i.  alpha <= 0 keeps every j <= i.
+ *   D3 attend   For row r (head h) of q-block i with kept set K and pruned set
+ *               P = {j < i not kept}:
+ *               o = [sum_{c in K, c<=r} e^{l_c} v_c + sum_{j in P} n_j e^{lbar_j} vbar_j]
+ *                 / [sum_{c in K, c<=r} e^{l_c}     + sum_{j in P} n_j e^{lbar_j}],
+ *               l_c = tau q_r . k_c, lbar_j = tau q_r . kbar_j (reading of the
+ *               "mean correction term that calibrates for the bias introduced by
+ *               pruning": every pruned block replaced by n_j copies of its mean
+ *               key and mean value).  LSE = ln(denominator).
+ *   D4 e4m3     inputs are codes times a per-(tensor, head) scale; the oracle
+ *               dequantises them exactly in double.
+ *
+ * Build with -DORC_MUTANT=n to plant one deliberate mistake (see the MUT()
+ * sites); the oracle self-tests check that every such mistake is caught.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#ifndef ORC_MUTANT
+#define ORC_MUTANT 0
+#endif
+#define MUT(n) (ORC_MUTANT == (n))
+
+/* D0: number of blocks of a request of length L. */
+static int64_t nblocks(int64_t L, int64_t Bs) { return (L + Bs - 1) / Bs; }
+
+/* D0: first global block id of every request (cb[B] = total blocks). */
+static void block_offsets(const int32_t* cu, int B, int Bs, int64_t* cb) {
+    cb[0] = 0;
+    for (int b = 0; b < B; ++b) cb[b + 1] = cb[b] + nblocks(cu[b + 1] - cu[b], Bs);
+}
+
+/* Total blocks of a batch. */
+int64_t orc_total_blocks(const int32_t* cu, int B, int Bs) {
+    int64_t t = 0;
+    for (int b = 0; b < B; ++b) t += nblocks(cu[b + 1] - cu[b], Bs);
+    return t;
+}
+
+/* D1: block means of a dequantised input x[T, H, d] (value * scale[h]).
+ * out: [total_blocks, H, d]. */
+void orc_block_means(const float* x, const double* scale, const int32_t* cu, int B, int H, int d,
+                     int Bs, double* out) {
+    int64_t* cb = (int64_t*)malloc(sizeof(int64_t) * (B + 1));
+    block_offsets(cu, B, Bs, cb);
+    for (int b = 0; b < B; ++b) {
+        int64_t L = cu[b + 1] - cu[b];
+        int64_t nb = nblocks(L, Bs);
+#pragma omp parallel for schedule(static)
+        for (int64_t j = 0; j < nb; ++j) {
+            int64_t n = L - j * Bs < Bs ? L - j * Bs : Bs;
+            double denom = MUT(5) ? (double)Bs : (double)n;
+            for (int h = 0; h < H; ++h) {
+                for (int c = 0; c < d; ++c) {
+                    double s = 0.0;
+                    for (int64_t r = 0; r < n; ++r) {
+                        int64_t row = cu[b] + j * Bs + r;
+                        s += (double)x[(row * H + h) * (int64_t)d + c] * scale[h];
+                    }
+                    out[((cb[b] + j) * H + h) * (int64_t)d + c] = s / denom;
+                }
+            }
+        }
+    }
+    free(cb);
+}
+
+/* D1 score of one (head, q-block, k-block) pair. */
+static double block_score(const double* qbar, const double* kbar, int64_t qb, int64_t kb, int h,
+                          int g, int Hq, int Hkv, int d, double tau) {
+    double dot = 0.0;
+    for (int c = 0; c < d; ++c)
+        dot += qbar[(qb * Hq + h) * (int64_t)d + c] * kbar[(kb * Hkv + g) * (int64_t)d + c];
+    return MUT(7) ? dot : tau * dot;
+}
+
+/* D1 + D2: kept-block lists.
+ *   kept_cnt [total_blocks, Hkv], kept_idx [total_blocks, Hkv, nb_max] (ascending);
+ *   s_out    [total_blocks, Hq, nb_max] raw scores s (NULL to skip), entries j > i untouched;
+ *   m_out    [total_blocks, Hq] row maxima (NULL to skip).
+ * Returns 0, or -1 when a request has more than nb_max blocks. */
+int orc_estimate(const double* qbar, const double* kbar, const int32_t* cu, int B, int Hq, int Hkv,
+                 int d, int Bs, double tau, double alpha, int nb_max, int32_t* kept_cnt,
+                 int32_t* kept_idx, double* s_out, double* m_out) {
+    int G = Hq / Hkv;
+    double ln_alpha = alpha > 0 ? log(alpha) : -INFINITY;
+    int64_t* cb = (int64_t*)malloc(sizeof(int64_t) * (B + 1));
+    block_offsets(cu, B, Bs, cb);
+    for (int b = 0; b < B; ++b)
+        if (nblocks(cu[b + 1] - cu[b], Bs) > nb_max) { free(cb); return -1; }
+    for (int b = 0; b < B; ++b) {
+        int64_t nb = nblocks(cu[b + 1] - cu[b], Bs);
+#pragma omp parallel for schedule(dynamic, 1)
+        for (int64_t i = 0; i < nb; ++i) {
+            int64_t qb = cb[b] + i;
+            double* s = (double*)malloc(sizeof(double) * (i + 1));
+            unsigned char* keep = (unsigned char*)malloc(i + 1);
+            for (int g = 0; g < Hkv; ++g) {
+                memset(keep, 0, i + 1);
+                for (int hh = 0; hh < G; ++hh) {
+                    int h = g * G + hh;
+                    int gk = MUT(3) ? h % Hkv : g;  /* mutant: wrong head -> group map */
+                    double m = -INFINITY;
+                    for (int64_t j = 0; j <= i; ++j) {
+                        s[j] = block_score(qbar, kbar, qb, cb[b] + j, h, gk, Hq, Hkv, d, tau);
+                        if (s[j] > m) m = s[j];
+                    }
+                    for (int64_t j = 0; j <= i; ++j) {
+                        int k;
+                        if (alpha <= 0) k = 1;
+                        else if (MUT(2)) k = s[j] >= alpha * m;          /* mutant: linear fraction */
+                        else if (MUT(4)) k = s[j] - m > ln_alpha;       /* mutant: strict */
+                        else k = s[j] - m >= ln_alpha;
+                        if (k) keep[j] = 1;
+                        if (s_out) s_out[(qb * Hq + h) * (int64_t)nb_max + j] = s[j];
+                    }
+                    if (m_out) m_out[qb * Hq + h] = m;
+                }
+                if (!MUT(8)) keep[i] = 1;
+                int32_t cnt = 0;
+                int32_t* idx = kept_idx + (qb * Hkv + g) * (int64_t)nb_max;
+                for (int64_t j = 0; j <= i; ++j)
+                    if (keep[j]) idx[cnt++] = (int32_t)j;
+                kept_cnt[qb * Hkv + g] = cnt;
+            }
+            free(s);
+            free(keep);
+        }
+    }
+    free(cb);
+    return 0;
+}
+
+/* Checks one kept list: strictly ascending entries in [0, i] ending with i. */
+static int list_ok(const int32_t* idx, int32_t cnt, int64_t i) {
+    if (cnt < 1 || cnt > i + 1) return 0;
+    for (int32_t t = 0; t < cnt; ++t) {
+        if (idx[t] < 0 || idx[t] > i) return 0;
+        if (t > 0 && idx[t] <= idx[t - 1]) return 0;
+    }
+    return idx[cnt - 1] == i;
+}
+
+/* D3: attention over the kept blocks plus (correction != 0) the mean-corrected
+ * pruned blocks.
+ *   q [T, Hq, d], k/v [T, Hkv, d] stored values; qs/ks/vs per-head scales;
+ *   kbar/vbar [total_blocks, Hkv, d] block means (needed when correction != 0);
+ *   sel: global q-block ids to compute (NULL = all), nsel entries;
+ *   o [T, Hq, d], lse [T, Hq], wsum [T, Hq] (sum of normalised weights; NULL ok).
+ * Returns 0, -1 on an invalid kept list, -2 on a bad q-block id. */
+int orc_attend(const float* q, const float* k, const float* v, const double* qs, const double* ks,
+               const double* vs, const int32_t* cu, int B, int Hq, int Hkv, int d, int Bs,
+               double tau, const int32_t* kept_cnt, const int32_t* kept_idx, int nb_max,
+               int correction, const double* kbar, const double* vbar, const int64_t* sel,
+               int64_t nsel, double* o, double* lse, double* wsum) {
+    int G = Hq / Hkv;
+    int64_t* cb = (int64_t*)malloc(sizeof(int64_t) * (B + 1));
+    block_offsets(cu, B, Bs, cb);
+    int64_t total = cb[B];
+    int64_t nwork = sel ? nsel : total;
+    /* request of every block */
+    int32_t* req = (int32_t*)malloc(sizeof(int32_t) * (total > 0 ? total : 1));
+    for (int b = 0; b < B; ++b)
+        for (int64_t t = cb[b]; t < cb[b + 1]; ++t) req[t] = b;
+    int status = 0;
+    for (int64_t w = 0; w < nwork; ++w) {
+        int64_t qb = sel ? sel[w] : w;
+        if (qb < 0 || qb >= total) { status = -2; break; }
+        int b = req[qb];
+        int64_t i = qb - cb[b];
+        for (int g = 0; g < Hkv; ++g)
+            if (!list_ok(kept_idx + (qb * Hkv + g) * (int64_t)nb_max, kept_cnt[qb * Hkv + g], i))
+                status = -1;
+    }
+    if (status != 0) { free(cb); free(req); return status; }
+
+#pragma omp parallel for schedule(dynamic, 1) collapse(2)
+    for (int64_t w = 0; w < nwork; ++w) {
+        for (int h = 0; h < Hq; ++h) {
+            int64_t qb = sel ? sel[w] : w;
+            int b = req[qb];
+            int64_t i = qb - cb[b];
+            int64_t L = cu[b + 1] - cu[b];
+            int g = MUT(3) ? h % Hkv : h / G;
+            const int32_t* idx = kept_idx + (qb * Hkv + g) * (int64_t)nb_max;
+            int32_t cnt = kept_cnt[qb * Hkv + g];
+            /* pruned set P = {j < i not kept} */
+            unsigned char* kept = (unsigned char*)calloc(i + 1, 1);
+            for (int32_t t = 0; t < cnt; ++t) kept[idx[t]] = 1;
+            int64_t nmax = (int64_t)cnt * Bs + i + 1;
+            double* lg = (double*)malloc(sizeof(double) * nmax);     /* logits */
+            const double** vrow = (const double**)malloc(sizeof(double*) * nmax);
+            double* vbuf = (double*)malloc(sizeof(double) * (size_t)cnt * Bs * d);
+            double* qd = (double*)malloc(sizeof(double) * d);
+            double* acc = (double*)malloc(sizeof(double) * d);
+            int64_t nrows = (L - i * Bs) < Bs ? (L - i * Bs) : Bs;
+            for (int64_t rr = 0; rr < nrows; ++rr) {
+                int64_t p = i * Bs + rr;                 /* request-local position */
+                int64_t grow = cu[b] + p;
+                for (int c = 0; c < d; ++c) qd[c] = (double)q[(grow * Hq + h) * (int64_t)d + c] * qs[h];
+                int64_t n = 0;
+                int64_t nv = 0;
+                for (int32_t t = 0; t < cnt; ++t) {
+                    int64_t j = idx[t];
+                    for (int64_t cc = 0; cc < Bs; ++cc) {
+                        int64_t kp = j * Bs + cc;
+                        int visible = MUT(6) ? (kp < p) : (kp <= p);
+                        if (kp >= L || !visible) continue;
+                        int64_t krow = cu[b] + kp;
+                        double dot = 0.0;
+                        for (int c = 0; c < d; ++c)
+                            dot += qd[c] * ((double)k[(krow * Hkv + g) * (int64_t)d + c] * ks[g]);
+                        lg[n] = tau * dot;
+                        double* vr = vbuf + nv * d;
+                        double vsc = MUT(10) ? 1.0 : vs[g];
+                        for (int c = 0; c < d; ++c) vr[c] = (double)v[(krow * Hkv + g) * (int64_t)d + c] * vsc;
+                        vrow[n] = vr;
+                        ++n;
+                        ++nv;
+                    }
+                }
+                if (correction) {
+                    for (int64_t j = 0; j < i; ++j) {
+                        if (kept[j]) continue;
+                        int64_t kb = cb[b] + j;
+                        int64_t nj = (L - j * Bs) < Bs ? (L - j * Bs) : Bs;
+                        double dot = 0.0;
+                        for (int c = 0; c < d; ++c) dot += qd[c] * kbar[(kb * Hkv + g) * (int64_t)d + c];
+                        lg[n] = tau * dot + (MUT(1) ? 0.0 : log((double)nj));
+                        vrow[n] = (MUT(9) ? kbar : vbar) + (kb * Hkv + g) * (int64_t)d;
+                        ++n;
+                    }
+                }
+                double m = -INFINITY;
+                for (int64_t t = 0; t < n; ++t) if (lg[t] > m) m = lg[t];
+                double den = 0.0;
+                for (int c = 0; c < d; ++c) acc[c] = 0.0;
+                for (int64_t t = 0; t < n; ++t) {
+                    double e = exp(lg[t] - m);
+                    den += e;
+                    for (int c = 0; c < d; ++c) acc[c] += e * vrow[t][c];
+                }
+                for (int c = 0; c < d; ++c) o[(grow * Hq + h) * (int64_t)d + c] = acc[c] / den;
+                lse[grow * Hq + h] = MUT(11) ? log(den) : m + log(den);
+                if (wsum) {
+                    double ws = 0.0;
+                    for (int64_t t = 0; t < n; ++t) ws += exp(lg[t] - m) / den;
+                    wsum[grow * Hq + h] = ws;
+                }
+            }
+            free(kept); free(lg); free(vrow); free(vbuf); free(qd); free(acc);
+        }
+    }
+    free(cb);
+    free(req);
+    return 0;
+}
+
+int orc_mutant_id(void) { return ORC_MUTANT; }

@@ -1,0 +1,306 @@
+"""Pins of the CPU oracle against facts fixed outside the oracle itself.
+
+Each ``pin_*`` takes an ``oracle.oracle.Oracle`` and raises ``AssertionError``
+on a mismatch.  ``test_oracle_pins.py`` runs them on the real oracle;
+``test_oracle_mutants.py`` runs them on builds with one planted mistake and
+requires that every mistake trips at least one pin.
+
+What pins what (definitions D0-D4 in the oracle header):
+  dense_sdpa        D3 core, D0 causality, LSE: alpha <= 0 equals
+                    torch's scaled_dot_product_attention (fp64, GQA expanded)
+  means_numpy       D1 block means (partial tail block) against numpy.mean
+  bilinearity       D1 score = mean of the brute-force token logit block
+  threshold_golden  D2 on hand-derived cases (tests/golden/threshold_cases.json)
+  diagonal_kept     D2 forced diagonal
+  nesting           D2 monotone in alpha
+  weights_sum       D3 normalised weights (with correction) sum to one
+  exact_correction  D3 correction is exact when K/V rows are constant per block
+  gqa_packing       D2/D3 head -> group map: packed heads = each head alone
+  ragged            D0 ragged batch = each request alone
+  e4m3_scales       D4 dequantisation: codes x power-of-two scale = scaled values
+"""
+from __future__ import annotations
+
+import json
+import math
+import os
+
+import numpy as np
+import torch
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+TAU = 1.0 / math.sqrt(128.0)
+
+
+def _rand_inputs(seqlens, hq, hkv, d=128, seed=0, scale=1.0):
+    rng = np.random.default_rng(seed)
+    T = int(sum(seqlens))
+    q = (rng.standard_normal((T, hq, d)) * scale).astype(np.float32)
+    k = (rng.standard_normal((T, hkv, d)) * scale).astype(np.float32)
+    v = rng.standard_normal((T, hkv, d)).astype(np.float32)
+    cu = np.concatenate([[0], np.cumsum(seqlens)]).astype(np.int32)
+    return q, k, v, cu
+
+
+def _sdpa(q, k, v, cu, hq, hkv):
+    """Dense causal attention per request with torch (fp64), GQA expanded."""
+    g = hq // hkv
+    outs, lses = [], []
+    for b in range(len(cu) - 1):
+        s, e = int(cu[b]), int(cu[b + 1])
+        qt = torch.from_numpy(q[s:e]).double().permute(1, 0, 2)
+        kt = torch.from_numpy(k[s:e]).double().repeat_interleave(g, dim=1).permute(1, 0, 2)
+        vt = torch.from_numpy(v[s:e]).double().repeat_interleave(g, dim=1).permute(1, 0, 2)
+        o = torch.nn.functional.scaled_dot_product_attention(qt[None], kt[None], vt[None], is_causal=True,
+                                                             scale=TAU)[0]
+        logits = (qt @ kt.transpose(1, 2)) * TAU
+        mask = torch.ones(e - s, e - s, dtype=torch.bool).tril()
+        lse = torch.logsumexp(logits.masked_fill(~mask, -math.inf), dim=-1)
+        outs.append(o.permute(1, 0, 2).numpy())
+        lses.append(lse.permute(1, 0).numpy())
+    return np.concatenate(outs), np.concatenate(lses)
+
+
+def _means(orc, q, k, v, cu, bs=128):
+    return orc.block_means(q, cu, bs), orc.block_means(k, cu, bs), orc.block_means(v, cu, bs)
+
+
+def pin_dense_sdpa(orc):
+    lens = [1, 127, 129, 200, 383, 512]
+    hq, hkv = 4, 2
+    q, k, v, cu = _rand_inputs(lens, hq, hkv, seed=11)
+    qb, kb, vb = _means(orc, q, k, v, cu)
+    est = orc.estimate(qb, kb, cu, 128, alpha=0.0, tau=TAU)
+    ref_o, ref_lse = _sdpa(q, k, v, cu, hq, hkv)
+    for corr in (False, True):
+        r = orc.attend(q, k, v, cu, 128, TAU, est["kept_cnt"], est["kept_idx"], correction=corr,
+                       kbar=kb, vbar=vb)
+        assert np.abs(r["o"] - ref_o).max() < 1e-12, "alpha<=0 output differs from dense SDPA"
+        assert np.abs(r["lse"] - ref_lse).max() < 1e-12, "LSE differs from torch.logsumexp"
+
+
+def pin_means_numpy(orc):
+    lens = [1, 200, 383]
+    q, k, v, cu = _rand_inputs(lens, 2, 1, seed=12)
+    kb = orc.block_means(k, cu, 128)
+    t = 0
+    for b, L in enumerate(lens):
+        for j in range((L + 127) // 128):
+            rows = k[cu[b] + j * 128: cu[b] + min(L, (j + 1) * 128)].astype(np.float64)
+            assert np.abs(kb[t] - rows.mean(axis=0)).max() < 1e-14, "block mean differs from numpy.mean"
+            t += 1
+    assert t == kb.shape[0]
+    # scales multiply the stored values
+    sc = np.array([0.25, 3.0])
+    qb = orc.block_means(q, cu, 128, scale=sc)
+    qb1 = orc.block_means(q, cu, 128)
+    assert np.abs(qb - qb1 * sc[None, :, None]).max() < 1e-13
+
+
+def pin_bilinearity(orc):
+    lens = [383, 256]
+    hq, hkv = 4, 2
+    q, k, v, cu = _rand_inputs(lens, hq, hkv, seed=13)
+    qb, kb, vb = _means(orc, q, k, v, cu)
+    est = orc.estimate(qb, kb, cu, 128, alpha=0.1, tau=TAU, want_scores=True)
+    s = est["s"]
+    t0 = 0
+    for b, L in enumerate(lens):
+        nb = (L + 127) // 128
+        qq = torch.from_numpy(q[cu[b]:cu[b + 1]]).double()
+        kk = torch.from_numpy(k[cu[b]:cu[b + 1]]).double()
+        for h in range(hq):
+            g = h // (hq // hkv)
+            logits = (qq[:, h, :] @ kk[:, g, :].T * TAU).numpy()
+            for i in range(nb):
+                for j in range(i + 1):
+                    blk = logits[i * 128:min(L, (i + 1) * 128), j * 128:min(L, (j + 1) * 128)]
+                    assert abs(s[t0 + i, h, j] - blk.mean()) < 1e-12, "score is not the mean block logit"
+        t0 += nb
+
+
+def _golden_case(c):
+    L, hq, hkv = c["L"], c["Hq"], c["Hkv"]
+    d = 128
+    q = np.zeros((L, hq, d), np.float32)
+    for h, ax in enumerate(c["qaxis"]):
+        q[:, h, ax] = 8.0
+    k = np.zeros((L, hkv, d), np.float32)
+    for ax, coefs in c["coef"].items():
+        for j, cval in enumerate(coefs):
+            k[j * 128:min(L, (j + 1) * 128), :, int(ax)] = cval
+    v = np.zeros((L, hkv, d), np.float32)
+    cu = np.array([0, L], np.int32)
+    return q, k, v, cu
+
+
+def pin_threshold_golden(orc):
+    with open(os.path.join(GOLDEN, "threshold_cases.json")) as f:
+        cases = json.load(f)["cases"]
+    for c in cases:
+        q, k, v, cu = _golden_case(c)
+        qb, kb, _ = _means(orc, q, k, v, cu)
+        est = orc.estimate(qb, kb, cu, 128, alpha=c["alpha"], tau=TAU, want_scores=True)
+        nb = len(c["kept"])
+        for i in range(nb):
+            for g in range(c["Hkv"]):
+                got = list(est["kept_idx"][i, g, :est["kept_cnt"][i, g]])
+                assert got == c["kept"][i][g], f"{c['name']}: q-block {i} kept {got}, expected {c['kept'][i][g]}"
+        if "s_last_row" in c:
+            assert np.abs(est["s"][nb - 1, 0, :nb] - np.array(c["s_last_row"])).max() < 1e-7
+
+
+def _structured(seqlens, hq=4, hkv=2, seed=21, lam=7.5):
+    from workloads import make_workload
+    return make_workload(seqlens, hq, hkv, alpha=0.1, seed=seed, n_retrieval=2, lam=lam)
+
+
+def pin_diagonal_kept(orc):
+    wl = _structured([1000, 640])
+    q, k, v = wl.float_inputs()
+    cu = wl.cu_seqlens
+    qb, kb, _ = _means(orc, q, k, v, cu)
+    for a in (0.5, 1.0):
+        est = orc.estimate(qb, kb, cu, 128, alpha=a, tau=TAU)
+        t = 0
+        for L in wl.seqlens:
+            for i in range((L + 127) // 128):
+                for g in range(wl.num_kv_heads):
+                    c = est["kept_cnt"][t, g]
+                    assert c >= 1 and est["kept_idx"][t, g, c - 1] == i, "diagonal block not kept"
+                t += 1
+
+
+def pin_nesting(orc):
+    wl = _structured([2048])
+    q, k, v = wl.float_inputs()
+    cu = wl.cu_seqlens
+    qb, kb, _ = _means(orc, q, k, v, cu)
+    prev = None
+    for a in (0.02, 0.05, 0.1, 0.2, 0.5):
+        est = orc.estimate(qb, kb, cu, 128, alpha=a, tau=TAU)
+        sets = [[set(est["kept_idx"][i, g, :est["kept_cnt"][i, g]]) for g in range(2)] for i in range(16)]
+        if prev is not None:
+            for i in range(16):
+                for g in range(2):
+                    assert sets[i][g] <= prev[i][g], "kept set grew when alpha grew"
+        prev = sets
+
+
+def pin_weights_sum(orc):
+    wl = _structured([1024])
+    q, k, v = wl.float_inputs()
+    cu = wl.cu_seqlens
+    qb, kb, vb = _means(orc, q, k, v, cu)
+    est = orc.estimate(qb, kb, cu, 128, alpha=0.3, tau=TAU)
+    assert (est["kept_cnt"][1:] < np.arange(2, 9)[:, None]).any(), "case prunes nothing"
+    r = orc.attend(q, k, v, cu, 128, TAU, est["kept_cnt"], est["kept_idx"], correction=True, kbar=kb,
+                   vbar=vb, want_wsum=True)
+    assert np.abs(r["wsum"] - 1.0).max() < 1e-12, "softmax weights do not sum to one"
+
+
+def pin_exact_correction(orc):
+    """K and V rows constant inside every block: replacing a pruned block by n_j
+    copies of its mean key/value is then exact, so the corrected sparse output
+    equals dense attention for any alpha."""
+    lens = [1024, 700]
+    hq, hkv = 4, 2
+    rng = np.random.default_rng(31)
+    T = sum(lens)
+    # a shared query direction spreads the block scores so that alpha prunes
+    q = (rng.standard_normal((T, hq, 128)) + rng.standard_normal((1, hq, 128))).astype(np.float32)
+    k = np.zeros((T, hkv, 128), np.float32)
+    v = np.zeros((T, hkv, 128), np.float32)
+    cu = np.array([0, lens[0], T], np.int32)
+    for b, L in enumerate(lens):
+        for j in range((L + 127) // 128):
+            s, e = cu[b] + j * 128, cu[b] + min(L, (j + 1) * 128)
+            k[s:e] = (rng.standard_normal((hkv, 128)) * 1.5).astype(np.float32)
+            v[s:e] = rng.standard_normal((hkv, 128)).astype(np.float32)
+    qb, kb, vb = _means(orc, q, k, v, cu)
+    ref_o, ref_lse = _sdpa(q, k, v, cu, hq, hkv)
+    for a in (0.3, 0.9):
+        est = orc.estimate(qb, kb, cu, 128, alpha=a, tau=TAU)
+        full = np.array([min(i, 7) + 1 for i in range(8)] + [i + 1 for i in range(6)])
+        assert (est["kept_cnt"].min(axis=1) < full).any(), "case prunes nothing"
+        r = orc.attend(q, k, v, cu, 128, TAU, est["kept_cnt"], est["kept_idx"], correction=True, kbar=kb, vbar=vb)
+        assert np.abs(r["o"] - ref_o).max() < 1e-11, "mean correction is not exact on block-constant K/V"
+        assert np.abs(r["lse"] - ref_lse).max() < 1e-11
+        r0 = orc.attend(q, k, v, cu, 128, TAU, est["kept_cnt"], est["kept_idx"], correction=False)
+        assert np.abs(r0["o"] - ref_o).max() > 1e-3, "pruning had no effect"
+
+
+def pin_gqa_packing(orc):
+    wl = _structured([900], hq=4, hkv=2, seed=41)
+    q, k, v = wl.float_inputs()
+    cu = wl.cu_seqlens
+    qb, kb, vb = _means(orc, q, k, v, cu)
+    est = orc.estimate(qb, kb, cu, 128, alpha=0.2, tau=TAU)
+    packed = orc.attend(q, k, v, cu, 128, TAU, est["kept_cnt"], est["kept_idx"], correction=True, kbar=kb, vbar=vb)
+    for h in range(4):
+        g = h // 2
+        one = orc.attend(q[:, h:h + 1], k[:, g:g + 1], v[:, g:g + 1], cu, 128, TAU,
+                         est["kept_cnt"][:, g:g + 1], est["kept_idx"][:, g:g + 1], correction=True,
+                         kbar=kb[:, g:g + 1], vbar=vb[:, g:g + 1])
+        assert np.abs(one["o"][:, 0] - packed["o"][:, h]).max() == 0.0, "packed head differs from head alone"
+    # the group list is the union of the per-head lists
+    for h in range(4):
+        g = h // 2
+        alone = orc.estimate(qb[:, h:h + 1], kb[:, g:g + 1], cu, 128, alpha=0.2, tau=TAU)
+        for i in range(qb.shape[0]):
+            sh = set(alone["kept_idx"][i, 0, :alone["kept_cnt"][i, 0]])
+            sg = set(est["kept_idx"][i, g, :est["kept_cnt"][i, g]])
+            assert sh <= sg, "group list misses a head's block"
+
+
+def pin_ragged(orc):
+    lens = [300, 1, 520]
+    wl = _structured(lens, seed=51)
+    q, k, v = wl.float_inputs()
+    cu = wl.cu_seqlens
+    qb, kb, vb = _means(orc, q, k, v, cu)
+    est = orc.estimate(qb, kb, cu, 128, alpha=0.2, tau=TAU)
+    full = orc.attend(q, k, v, cu, 128, TAU, est["kept_cnt"], est["kept_idx"], correction=True, kbar=kb, vbar=vb)
+    t0 = 0
+    for b, L in enumerate(lens):
+        s, e = int(cu[b]), int(cu[b + 1])
+        cu1 = np.array([0, L], np.int32)
+        qb1, kb1, vb1 = _means(orc, q[s:e], k[s:e], v[s:e], cu1)
+        e1 = orc.estimate(qb1, kb1, cu1, 128, alpha=0.2, tau=TAU, nb_max=est["nb_max"])
+        nb = (L + 127) // 128
+        assert (e1["kept_cnt"] == est["kept_cnt"][t0:t0 + nb]).all()
+        r1 = orc.attend(q[s:e], k[s:e], v[s:e], cu1, 128, TAU, e1["kept_cnt"], e1["kept_idx"], correction=True,
+                        kbar=kb1, vbar=vb1)
+        assert np.abs(r1["o"] - full["o"][s:e]).max() == 0.0, "request in a batch differs from request alone"
+        t0 += nb
+
+
+def pin_e4m3_scales(orc):
+    lens = [500]
+    hq, hkv = 4, 2
+    rng = np.random.default_rng(61)
+    codes = [torch.from_numpy(rng.standard_normal((500, h, 128)).astype(np.float32) * 40).to(torch.float8_e4m3fn).float().numpy()
+             for h in (hq, hkv, hkv)]
+    q8, k8, v8 = codes
+    cu = np.array([0, 500], np.int32)
+    qs = np.array([2.0 ** -6, 2.0 ** -5, 2.0 ** -7, 2.0 ** -6])
+    ks = np.array([2.0 ** -5, 2.0 ** -6])
+    vs = np.array([2.0 ** -4, 2.0 ** -3])
+    qsc, ksc, vsc = (q8 * qs[None, :, None]).astype(np.float32), (k8 * ks[None, :, None]).astype(np.float32), \
+        (v8 * vs[None, :, None]).astype(np.float32)
+    qb = orc.block_means(q8, cu, 128, qs)
+    kb = orc.block_means(k8, cu, 128, ks)
+    vb = orc.block_means(v8, cu, 128, vs)
+    est = orc.estimate(qb, kb, cu, 128, alpha=0.3, tau=TAU)
+    a = orc.attend(q8, k8, v8, cu, 128, TAU, est["kept_cnt"], est["kept_idx"], correction=True, kbar=kb, vbar=vb,
+                   q_scale=qs, k_scale=ks, v_scale=vs)
+    qb2, kb2, vb2 = _means(orc, qsc, ksc, vsc, cu)
+    est2 = orc.estimate(qb2, kb2, cu, 128, alpha=0.3, tau=TAU)
+    assert (est2["kept_cnt"] == est["kept_cnt"]).all()
+    b = orc.attend(qsc, ksc, vsc, cu, 128, TAU, est2["kept_cnt"], est2["kept_idx"], correction=True,
+                   kbar=kb2, vbar=vb2)
+    assert np.abs(a["o"] - b["o"]).max() < 1e-12, "e4m3 dequantisation differs from scaled values"
+
+
+ALL_PINS = [pin_dense_sdpa, pin_means_numpy, pin_bilinearity, pin_threshold_golden, pin_diagonal_kept,
+            pin_nesting, pin_weights_sum, pin_exact_correction, pin_gqa_packing, pin_ragged, pin_e4m3_scales]

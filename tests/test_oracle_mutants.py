@@ -1,0 +1,33 @@
+"""Every mistake planted in the oracle (built with -DORC_MUTANT=n) must trip at
+least one pin, so the pins would notice such a mistake in the oracle itself."""
+import pytest
+
+from oracle.oracle import Oracle
+import oracle_pins
+
+MUTANTS = {
+    1: "correction weight n_j dropped",
+    2: "threshold as a linear fraction of the max",
+    3: "query head mapped to KV group h % Hkv",
+    4: "strict comparison at the threshold",
+    5: "block mean divided by the block size, not the row count",
+    6: "causal mask excludes the diagonal token",
+    7: "score without the softmax scale",
+    8: "diagonal block not forced",
+    9: "mean key used as the correction value",
+    10: "value scale ignored",
+    11: "LSE without the row max",
+}
+
+
+@pytest.mark.parametrize("mutant", sorted(MUTANTS), ids=[MUTANTS[m] for m in sorted(MUTANTS)])
+def test_mutant_is_caught(mutant):
+    orc = Oracle(mutant)
+    assert orc.lib.orc_mutant_id() == mutant
+    tripped = []
+    for pin in oracle_pins.ALL_PINS:
+        try:
+            pin(orc)
+        except (AssertionError, ValueError):
+            tripped.append(pin.__name__)
+    assert tripped, f"planted mistake '{MUTANTS[mutant]}' passes every pin"

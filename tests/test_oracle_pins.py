@@ -1,0 +1,15 @@
+"""The CPU oracle against its pins (no GPU)."""
+import pytest
+
+from oracle.oracle import Oracle
+import oracle_pins
+
+
+@pytest.fixture(scope="module")
+def orc():
+    return Oracle()
+
+
+@pytest.mark.parametrize("pin", oracle_pins.ALL_PINS, ids=[p.__name__ for p in oracle_pins.ALL_PINS])
+def test_pin(orc, pin):
+    pin(orc)
