@@ -1,0 +1,186 @@
+"""B200 (sm_100a) block-sparse prefill attention: Python binding of libfp2.
+
+Every function here marshals torch tensors into the C ABI of include/fp2.h;
+all work runs in the CUDA kernels of libfp2.so.  There is no CPU path: a
+missing library raises.
+
+    params = Params(num_q_heads=32, num_kv_heads=8, alpha=0.05)
+    meta = BlockMeta.empty(params, batch, total_tokens, max_seqlen, device)
+    ws = Workspace(params, batch, total_tokens, max_seqlen, device)
+    estimate(params, q, k, v, cu_seqlens, max_seqlen, meta, ws)
+    sparse_prefill(params, q, k, v, cu_seqlens, max_seqlen, meta, out, ws, lse=lse)
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+from typing import Optional
+
+import torch
+
+from . import _lib
+from ._lib import FP2_BF16, FP2_E4M3, STATUS
+
+__all__ = ["Params", "BlockMeta", "Workspace", "FP2Error", "max_blocks", "workspace_bytes",
+           "estimate", "sparse_prefill", "prefill_paged", "get_error", "status_string", "version",
+           "FP2_BF16", "FP2_E4M3"]
+
+BLOCK = 128
+HEAD_DIM = 128
+
+
+class FP2Error(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {STATUS.get(code, code)} ({status_string(code)})")
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _check(code: int, where: str):
+    if code != 0:
+        raise FP2Error(code, where)
+
+
+@dataclasses.dataclass
+class Params:
+    """Mirror of ``fp2_params``.  Scales are device tensors (e4m3 only)."""
+
+    num_q_heads: int
+    num_kv_heads: int
+    alpha: float = 0.05
+    sm_scale: float = 0.0
+    correction: bool = True
+    dtype: int = FP2_BF16
+    q_scale: Optional[torch.Tensor] = None
+    k_scale: Optional[torch.Tensor] = None
+    v_scale: Optional[torch.Tensor] = None
+    head_dim: int = HEAD_DIM
+    block_size: int = BLOCK
+
+    def c(self) -> _lib.fp2_params:
+        return _lib.fp2_params(self.num_q_heads, self.num_kv_heads, self.head_dim, self.block_size,
+                               float(self.alpha), float(self.sm_scale), 1 if self.correction else 0,
+                               int(self.dtype), _ptr(self.q_scale), _ptr(self.k_scale),
+                               _ptr(self.v_scale))
+
+
+def max_blocks(batch: int, total_tokens: int, block_size: int = BLOCK) -> int:
+    return int(_lib.load().fp2_max_blocks(batch, total_tokens, block_size))
+
+
+def workspace_bytes(params: Params, batch: int, total_tokens: int, max_seqlen: int) -> int:
+    p = params.c()
+    return int(_lib.load().fp2_workspace_bytes(ctypes.byref(p), batch, total_tokens, max_seqlen))
+
+
+class Workspace:
+    """Caller-owned scratch memory of the library (a uint8 device tensor)."""
+
+    def __init__(self, params: Params, batch: int, total_tokens: int, max_seqlen: int,
+                 device="cuda", stream=None):
+        n = workspace_bytes(params, batch, total_tokens, max_seqlen)
+        if n == 0:
+            raise FP2Error(1, "fp2_workspace_bytes")
+        self.buf = torch.empty(n + 256, dtype=torch.uint8, device=device)
+        off = (-self.buf.data_ptr()) % 256
+        self.tensor = self.buf[off:off + n]
+        self.nbytes = n
+        _check(_lib.load().fp2_workspace_init(_ptr(self.tensor), n, _stream(stream)), "fp2_workspace_init")
+
+    @property
+    def ptr(self):
+        return _ptr(self.tensor)
+
+
+@dataclasses.dataclass
+class BlockMeta:
+    """Mirror of ``fp2_blockmeta``, holding the device tensors."""
+
+    kept_cnt: torch.Tensor
+    kept_idx: torch.Tensor
+    k_mean: torch.Tensor
+    v_mean: Optional[torch.Tensor]
+    score_dbg: Optional[torch.Tensor]
+    nb_max: int
+    max_blocks: int
+
+    @staticmethod
+    def empty(params: Params, batch: int, total_tokens: int, max_seqlen: int, device="cuda",
+              scores: bool = False, nb_max: Optional[int] = None) -> "BlockMeta":
+        mb = max(1, max_blocks(batch, total_tokens))
+        nbm = nb_max or max(1, (max_seqlen + BLOCK - 1) // BLOCK)
+        hkv = params.num_kv_heads
+        return BlockMeta(
+            kept_cnt=torch.zeros((mb, hkv), dtype=torch.int32, device=device),
+            kept_idx=torch.full((mb, hkv, nbm), -1, dtype=torch.int32, device=device),
+            k_mean=torch.zeros((mb, hkv, HEAD_DIM), dtype=torch.float32, device=device),
+            v_mean=torch.zeros((mb, hkv, HEAD_DIM), dtype=torch.float32, device=device),
+            score_dbg=(torch.full((mb, params.num_q_heads, nbm), float("nan"), dtype=torch.float32,
+                                  device=device) if scores else None),
+            nb_max=nbm, max_blocks=mb)
+
+    def c(self) -> _lib.fp2_blockmeta:
+        return _lib.fp2_blockmeta(_ptr(self.kept_cnt), _ptr(self.kept_idx), _ptr(self.k_mean),
+                                  _ptr(self.v_mean), _ptr(self.score_dbg), self.nb_max, self.max_blocks)
+
+
+def _bt_args(block_table: Optional[torch.Tensor], num_pages: int):
+    if block_table is None:
+        return None, 0, 0
+    return _ptr(block_table), int(block_table.shape[1]), int(num_pages)
+
+
+def estimate(params: Params, q, k, v, cu_seqlens, max_seqlen: int, meta: BlockMeta, ws: Workspace,
+             block_table: Optional[torch.Tensor] = None, num_pages: int = 0, stream=None) -> None:
+    """``fp2_estimate``: kept-block lists and block means into ``meta``."""
+    p, m = params.c(), meta.c()
+    bt, mbps, npg = _bt_args(block_table, num_pages)
+    _check(_lib.load().fp2_estimate(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens),
+                                    int(cu_seqlens.numel()) - 1, int(q.shape[0]), int(max_seqlen), bt,
+                                    mbps, npg, ctypes.byref(m), ws.ptr, ws.nbytes, _stream(stream)),
+           "fp2_estimate")
+
+
+def sparse_prefill(params: Params, q, k, v, cu_seqlens, max_seqlen: int, meta: BlockMeta, out,
+                   ws: Workspace, lse=None, stream=None) -> None:
+    """``fp2_sparse_prefill``: attention over the kept blocks (+ mean correction)."""
+    p, m = params.c(), meta.c()
+    _check(_lib.load().fp2_sparse_prefill(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens),
+                                          int(cu_seqlens.numel()) - 1, int(q.shape[0]), int(max_seqlen),
+                                          ctypes.byref(m), _ptr(out), _ptr(lse), ws.ptr, ws.nbytes,
+                                          _stream(stream)),
+           "fp2_sparse_prefill")
+
+
+def prefill_paged(params: Params, q, k_pool, v_pool, cu_seqlens, max_seqlen: int, block_table,
+                  num_pages: int, meta: BlockMeta, out, ws: Workspace, lse=None, stream=None) -> None:
+    """``fp2_prefill_paged``: estimator + attention on a paged KV cache."""
+    p, m = params.c(), meta.c()
+    _check(_lib.load().fp2_prefill_paged(ctypes.byref(p), _ptr(q), _ptr(k_pool), _ptr(v_pool),
+                                         _ptr(cu_seqlens), int(cu_seqlens.numel()) - 1, int(q.shape[0]),
+                                         int(max_seqlen), _ptr(block_table), int(block_table.shape[1]),
+                                         int(num_pages), ctypes.byref(m), _ptr(out), _ptr(lse), ws.ptr,
+                                         ws.nbytes, _stream(stream)),
+           "fp2_prefill_paged")
+
+
+def get_error(ws: Workspace, stream=None) -> int:
+    """``fp2_get_error``: device-side status since the last read (synchronises)."""
+    return int(_lib.load().fp2_get_error(ws.ptr, _stream(stream)))
+
+
+def status_string(code: int) -> str:
+    return _lib.load().fp2_status_string(int(code)).decode()
+
+
+def version() -> int:
+    return int(_lib.load().fp2_version())

@@ -1,0 +1,407 @@
+// api.cu -- the C ABI (include/fp2.h): argument checks, workspace layout,
+// TMA descriptors and kernel launches.  No allocation, no global state besides
+// the cached driver entry point of cuTensorMapEncodeTiled.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "common.cuh"
+#include "kernels.h"
+
+using namespace fp2;
+
+namespace {
+
+constexpr size_t kMaxSmem = 232448;  // 227 KB opt-in per CTA on sm_100
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// 3-D map over [rows, heads, 128] (token-major) with 128-byte-swizzled boxes of
+// 128 rows x one head x 128 bytes.
+bool make_map(CUtensorMap* m, const void* base, bool e4m3, int64_t heads, int64_t rows) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    const cuuint64_t esz = e4m3 ? 1 : 2;
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kHeadDim), static_cast<cuuint64_t>(heads),
+                                static_cast<cuuint64_t>(rows > 0 ? rows : 1)};
+    const cuuint64_t strides[2] = {kHeadDim * esz, kHeadDim * esz * static_cast<cuuint64_t>(heads)};
+    const cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / esz), 1, 128};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, e4m3 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+               const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int32_t esize(const fp2_params* p) { return p->dtype == FP2_E4M3 ? 1 : 2; }
+
+fp2_status check_params(const fp2_params* p) {
+    if (!p) return FP2_ERR_INVALID_ARG;
+    if (p->num_q_heads < 1 || p->num_kv_heads < 1 || p->num_q_heads % p->num_kv_heads != 0)
+        return FP2_ERR_INVALID_ARG;
+    if (p->dtype != FP2_BF16 && p->dtype != FP2_E4M3) return FP2_ERR_INVALID_ARG;
+    if (p->correction != 0 && p->correction != 1) return FP2_ERR_INVALID_ARG;
+    if (std::isnan(p->alpha) || p->alpha > 1.f) return FP2_ERR_INVALID_ARG;
+    if (!std::isfinite(p->sm_scale) || p->sm_scale < 0.f) return FP2_ERR_INVALID_ARG;
+    if (p->head_dim <= 0 || p->block_size <= 0) return FP2_ERR_INVALID_ARG;
+    if (p->head_dim != kHeadDim || p->block_size != kBlock) return FP2_ERR_UNSUPPORTED;
+    if (p->dtype == FP2_E4M3 && (!p->q_scale || !p->k_scale || !p->v_scale))
+        return FP2_ERR_INVALID_ARG;
+    return FP2_OK;
+}
+
+float tau_of(const fp2_params* p) {
+    return p->sm_scale > 0.f ? p->sm_scale : 1.f / std::sqrt(static_cast<float>(p->head_dim));
+}
+
+struct Problem {
+    int32_t batch;
+    int64_t total_tokens;
+    int32_t max_seqlen;
+    int64_t max_blocks;   // host bound of sum_b nb_b
+    int32_t nb_need;      // ceil(max_seqlen / block)
+    WsLayout ws;
+};
+
+fp2_status check_problem(const fp2_params* p, const void* q, const void* k, const void* v,
+                         const int32_t* cu, int32_t batch, int64_t total_tokens,
+                         int32_t max_seqlen, void* workspace, size_t ws_bytes, Problem* out) {
+    fp2_status st = check_params(p);
+    if (st != FP2_OK) return st;
+    if (batch < 0 || total_tokens < 0 || max_seqlen < 0) return FP2_ERR_INVALID_ARG;
+    if (total_tokens > (int64_t(1) << 31) - 1) return FP2_ERR_UNSUPPORTED;
+    if (batch > 0 && !cu) return FP2_ERR_INVALID_ARG;
+    if (total_tokens > 0 && (!q || !k || !v)) return FP2_ERR_INVALID_ARG;
+    if ((q && !aligned(q, 16)) || (k && !aligned(k, 16)) || (v && !aligned(v, 16)))
+        return FP2_ERR_INVALID_ARG;
+    out->batch = batch;
+    out->total_tokens = total_tokens;
+    out->max_seqlen = max_seqlen;
+    out->max_blocks = fp2_max_blocks(batch, total_tokens, kBlock);
+    out->nb_need = (max_seqlen + kBlock - 1) / kBlock;
+    out->ws = ws_layout(batch, out->max_blocks, p->num_q_heads, p->num_kv_heads, esize(p));
+    if (!workspace || !aligned(workspace, 256) || ws_bytes < out->ws.total) return FP2_ERR_WORKSPACE;
+    return FP2_OK;
+}
+
+fp2_status check_meta(const fp2_blockmeta* m, const fp2_params* p, const Problem& pr, bool need_v) {
+    if (!m || !m->kept_cnt || !m->kept_idx || !m->k_mean) return FP2_ERR_INVALID_ARG;
+    if (need_v && p->correction && !m->v_mean) return FP2_ERR_INVALID_ARG;
+    if (m->nb_max < pr.nb_need || m->nb_max < 1) return FP2_ERR_INVALID_ARG;
+    if (m->max_blocks < 0) return FP2_ERR_INVALID_ARG;
+    if (!aligned(m->k_mean, 16) || (m->v_mean && !aligned(m->v_mean, 16))) return FP2_ERR_INVALID_ARG;
+    return FP2_OK;
+}
+
+template <class T>
+T* at(void* ws, size_t off) {
+    return reinterpret_cast<T*>(static_cast<char*>(ws) + off);
+}
+
+fp2_status launched(cudaError_t e) { return e == cudaSuccess ? FP2_OK : FP2_ERR_CUDA; }
+
+// Score-kernel tiling: q-blocks per tile so that the score rows fit in shared memory.
+bool score_tiling(int32_t G, int32_t nb_need, int32_t* qt, int32_t* rp, int32_t* ncap, size_t* smem) {
+    const int32_t cap = ((nb_need + kScoreKC - 1) / kScoreKC) * kScoreKC;
+    int32_t q = G >= 32 ? 1 : 32 / G;
+    while (true) {
+        const int32_t r = ((q * G + 3) / 4) * 4;
+        const size_t bytes = sizeof(float) * (size_t(kHeadDim) * r + size_t(kHeadDim) * (kScoreKC + 4) +
+                                              size_t(r) * cap + r);
+        if (r <= 64 && bytes <= kMaxSmem) {
+            *qt = q;
+            *rp = r;
+            *ncap = cap > 0 ? cap : kScoreKC;
+            *smem = bytes;
+            return true;
+        }
+        if (q == 1) return false;
+        q /= 2;
+    }
+}
+
+fp2_status run_setup(const Problem& pr, void* ws, const int32_t* cu, int32_t qt, bool paged,
+                     int32_t mbps, int64_t meta_blocks, cudaStream_t s) {
+    SetupArgs sa;
+    sa.cu = cu;
+    sa.batch = pr.batch;
+    sa.total_tokens = pr.total_tokens;
+    sa.max_seqlen = pr.max_seqlen;
+    sa.qt = qt;
+    sa.paged = paged ? 1 : 0;
+    sa.max_blocks_per_seq = mbps;
+    sa.max_blocks = meta_blocks < pr.max_blocks ? meta_blocks : pr.max_blocks;
+    sa.hdr = at<WsHeader>(ws, 0);
+    sa.cu_blocks = at<int32_t>(ws, pr.ws.cu_blocks);
+    sa.cu_tiles = at<int32_t>(ws, pr.ws.cu_tiles);
+    sa.blk_req = at<int32_t>(ws, pr.ws.blk_req);
+    setup_kernel<<<1, 256, 0, s>>>(sa);
+    return launched(cudaGetLastError());
+}
+
+fp2_status run_estimate(const fp2_params* p, const void* q, const void* k, const void* v,
+                        const int32_t* cu, const Problem& pr, const int32_t* block_table,
+                        int32_t mbps, int32_t num_pages, fp2_blockmeta* meta, void* ws,
+                        cudaStream_t s) {
+    const int32_t G = p->num_q_heads / p->num_kv_heads;
+    int32_t qt, rp, ncap;
+    size_t score_smem;
+    if (!score_tiling(G, pr.nb_need, &qt, &rp, &ncap, &score_smem)) return FP2_ERR_UNSUPPORTED;
+    fp2_status st = run_setup(pr, ws, cu, qt, block_table != nullptr, mbps, meta->max_blocks, s);
+    if (st != FP2_OK || pr.batch == 0 || pr.max_blocks == 0) return st;
+
+    const bool e4m3 = p->dtype == FP2_E4M3;
+    WsHeader* hdr = at<WsHeader>(ws, 0);
+    PoolArgs pa;
+    memset(&pa, 0, sizeof(pa));
+    pa.x[0] = q;
+    pa.x[1] = k;
+    pa.x[2] = v;
+    pa.out[0] = at<float>(ws, pr.ws.qbar);
+    pa.out[1] = meta->k_mean;
+    pa.out[2] = meta->v_mean;
+    pa.scale[0] = e4m3 ? p->q_scale : nullptr;
+    pa.scale[1] = e4m3 ? p->k_scale : nullptr;
+    pa.scale[2] = e4m3 ? p->v_scale : nullptr;
+    pa.heads[0] = p->num_q_heads;
+    pa.heads[1] = p->num_kv_heads;
+    pa.heads[2] = p->num_kv_heads;
+    const int32_t per_cta = 128 * (e4m3 ? 16 : 8);
+    for (int x = 0; x < 3; ++x) pa.slabs[x] = (pa.heads[x] * kHeadDim + per_cta - 1) / per_cta;
+    pa.paged[0] = 0;
+    pa.paged[1] = pa.paged[2] = block_table ? 1 : 0;
+    pa.ntensors = meta->v_mean ? 3 : 2;
+    pa.cu = cu;
+    pa.cu_blocks = at<int32_t>(ws, pr.ws.cu_blocks);
+    pa.blk_req = at<int32_t>(ws, pr.ws.blk_req);
+    pa.block_table = block_table;
+    pa.max_blocks_per_seq = mbps;
+    pa.num_pages = num_pages;
+    pa.hdr = hdr;
+    const int32_t ys = pa.slabs[0] + pa.slabs[1] + (pa.ntensors == 3 ? pa.slabs[2] : 0);
+    dim3 pgrid(static_cast<unsigned>(pr.max_blocks), static_cast<unsigned>(ys));
+    if (e4m3)
+        pool_kernel<true><<<pgrid, kPoolThreads, 0, s>>>(pa);
+    else
+        pool_kernel<false><<<pgrid, kPoolThreads, 0, s>>>(pa);
+    if ((st = launched(cudaGetLastError())) != FP2_OK) return st;
+
+    ScoreArgs sa;
+    sa.qbar = at<float>(ws, pr.ws.qbar);
+    sa.kbar = meta->k_mean;
+    sa.cu_blocks = at<int32_t>(ws, pr.ws.cu_blocks);
+    sa.cu_tiles = at<int32_t>(ws, pr.ws.cu_tiles);
+    sa.batch = pr.batch;
+    sa.hq = p->num_q_heads;
+    sa.hkv = p->num_kv_heads;
+    sa.G = G;
+    sa.qt = qt;
+    sa.rp = rp;
+    sa.ncap = ncap;
+    sa.nb_max = meta->nb_max;
+    sa.tau = tau_of(p);
+    sa.keep_all = p->alpha <= 0.f ? 1 : 0;
+    sa.ln_alpha = p->alpha > 0.f ? std::log(p->alpha) : 0.f;
+    sa.kept_cnt = meta->kept_cnt;
+    sa.kept_idx = meta->kept_idx;
+    sa.score_dbg = meta->score_dbg;
+    sa.hdr = hdr;
+    if (cudaFuncSetAttribute(score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(score_smem)) != cudaSuccess)
+        return FP2_ERR_CUDA;
+    const int64_t tiles = (pr.max_blocks + qt - 1) / qt + pr.batch;
+    score_kernel<<<dim3(static_cast<unsigned>(tiles), static_cast<unsigned>(p->num_kv_heads)),
+                   rp * 8, score_smem, s>>>(sa);
+    return launched(cudaGetLastError());
+}
+
+fp2_status run_attention(const fp2_params* p, const void* q, const void* k, const void* v,
+                         const int32_t* cu, const Problem& pr, const int32_t* block_table,
+                         int32_t mbps, int32_t num_pages, const fp2_blockmeta* meta, void* out,
+                         float* lse, void* ws, cudaStream_t s, bool need_setup) {
+    const bool e4m3 = p->dtype == FP2_E4M3;
+    if (attn_smem_bytes(e4m3, pr.nb_need) > kMaxSmem) return FP2_ERR_UNSUPPORTED;
+    fp2_status st = FP2_OK;
+    if (need_setup) {
+        st = run_setup(pr, ws, cu, 1, block_table != nullptr, mbps, meta->max_blocks, s);
+        if (st != FP2_OK) return st;
+    }
+    if (pr.batch == 0 || pr.max_blocks == 0) return FP2_OK;
+    WsHeader* hdr = at<WsHeader>(ws, 0);
+    void* kb_lp = at<void>(ws, pr.ws.kbar_lp);
+    void* vb_lp = at<void>(ws, pr.ws.vbar_lp);
+    if (p->correction) {
+        MeanLpArgs ma;
+        ma.k_mean = meta->k_mean;
+        ma.v_mean = meta->v_mean;
+        ma.k_lp = kb_lp;
+        ma.v_lp = vb_lp;
+        ma.k_scale = p->k_scale;
+        ma.v_scale = p->v_scale;
+        ma.hkv = p->num_kv_heads;
+        ma.e4m3 = e4m3 ? 1 : 0;
+        ma.max_blocks = pr.max_blocks;
+        ma.hdr = hdr;
+        meanlp_kernel<<<592, 256, 0, s>>>(ma);
+        if ((st = launched(cudaGetLastError())) != FP2_OK) return st;
+    }
+    const int64_t kv_rows = block_table ? int64_t(num_pages) * kBlock : pr.total_tokens;
+    CUtensorMap tq, tk, tv, tkb, tvb;
+    if (!make_map(&tq, q, e4m3, p->num_q_heads, pr.total_tokens) ||
+        !make_map(&tk, k, e4m3, p->num_kv_heads, kv_rows) ||
+        !make_map(&tv, v, e4m3, p->num_kv_heads, kv_rows) ||
+        !make_map(&tkb, kb_lp, e4m3, p->num_kv_heads, pr.max_blocks) ||
+        !make_map(&tvb, vb_lp, e4m3, p->num_kv_heads, pr.max_blocks))
+        return FP2_ERR_CUDA;
+    AttnArgs a;
+    a.cu = cu;
+    a.cu_blocks = at<int32_t>(ws, pr.ws.cu_blocks);
+    a.blk_req = at<int32_t>(ws, pr.ws.blk_req);
+    a.block_table = block_table;
+    a.max_blocks_per_seq = mbps;
+    a.num_pages = num_pages;
+    a.kept_cnt = meta->kept_cnt;
+    a.kept_idx = meta->kept_idx;
+    a.nb_max = meta->nb_max;
+    a.nb_cap = pr.nb_need > 0 ? pr.nb_need : 1;
+    a.hq = p->num_q_heads;
+    a.hkv = p->num_kv_heads;
+    a.G = p->num_q_heads / p->num_kv_heads;
+    a.pairs = (a.G + 1) / 2;
+    a.correction = p->correction;
+    a.scale_log2 = tau_of(p) * 1.4426950408889634f;
+    a.q_scale = p->q_scale;
+    a.k_scale = p->k_scale;
+    a.v_scale = p->v_scale;
+    a.out = out;
+    a.lse = lse;
+    a.hdr = hdr;
+    return launched(launch_attention(e4m3, a, tq, tk, tv, tkb, tvb, pr.max_blocks, s));
+}
+
+}  // namespace
+
+extern "C" {
+
+int64_t fp2_max_blocks(int32_t batch, int64_t total_tokens, int32_t block_size) {
+    if (batch < 0 || total_tokens < 0 || block_size <= 0) return 0;
+    return total_tokens / block_size + batch;
+}
+
+size_t fp2_workspace_bytes(const fp2_params* params, int32_t batch, int64_t total_tokens,
+                           int32_t max_seqlen) {
+    if (check_params(params) != FP2_OK || batch < 0 || total_tokens < 0 || max_seqlen < 0) return 0;
+    return ws_layout(batch, fp2_max_blocks(batch, total_tokens, kBlock), params->num_q_heads,
+                     params->num_kv_heads, esize(params))
+        .total;
+}
+
+fp2_status fp2_workspace_init(void* workspace, size_t ws_bytes, void* stream) {
+    if (!workspace || !aligned(workspace, 256) || ws_bytes < sizeof(WsHeader)) return FP2_ERR_WORKSPACE;
+    return launched(cudaMemsetAsync(workspace, 0, sizeof(WsHeader), static_cast<cudaStream_t>(stream)));
+}
+
+fp2_status fp2_estimate(const fp2_params* params, const void* q, const void* k, const void* v,
+                        const int32_t* cu_seqlens, int32_t batch, int64_t total_tokens,
+                        int32_t max_seqlen, const int32_t* block_table, int32_t max_blocks_per_seq,
+                        int32_t num_pages, fp2_blockmeta* meta, void* workspace, size_t ws_bytes,
+                        void* stream) {
+    Problem pr;
+    fp2_status st = check_problem(params, q, k, v, cu_seqlens, batch, total_tokens, max_seqlen,
+                                  workspace, ws_bytes, &pr);
+    if (st != FP2_OK) return st;
+    if ((st = check_meta(meta, params, pr, false)) != FP2_OK) return st;
+    if (block_table && (max_blocks_per_seq < 1 || num_pages < 1)) return FP2_ERR_INVALID_ARG;
+    return run_estimate(params, q, k, v, cu_seqlens, pr, block_table, max_blocks_per_seq, num_pages,
+                        meta, workspace, static_cast<cudaStream_t>(stream));
+}
+
+fp2_status fp2_sparse_prefill(const fp2_params* params, const void* q, const void* k, const void* v,
+                              const int32_t* cu_seqlens, int32_t batch, int64_t total_tokens,
+                              int32_t max_seqlen, const fp2_blockmeta* meta, void* out, float* lse,
+                              void* workspace, size_t ws_bytes, void* stream) {
+    Problem pr;
+    fp2_status st = check_problem(params, q, k, v, cu_seqlens, batch, total_tokens, max_seqlen,
+                                  workspace, ws_bytes, &pr);
+    if (st != FP2_OK) return st;
+    if ((st = check_meta(meta, params, pr, true)) != FP2_OK) return st;
+    if (total_tokens > 0 && (!out || !aligned(out, 16))) return FP2_ERR_INVALID_ARG;
+    if (lse && !aligned(lse, 4)) return FP2_ERR_INVALID_ARG;
+    return run_attention(params, q, k, v, cu_seqlens, pr, nullptr, 0, 0, meta, out, lse, workspace,
+                         static_cast<cudaStream_t>(stream), true);
+}
+
+fp2_status fp2_prefill_paged(const fp2_params* params, const void* q, const void* k_pool,
+                             const void* v_pool, const int32_t* cu_seqlens, int32_t batch,
+                             int64_t total_tokens, int32_t max_seqlen, const int32_t* block_table,
+                             int32_t max_blocks_per_seq, int32_t num_pages, fp2_blockmeta* meta,
+                             void* out, float* lse, void* workspace, size_t ws_bytes, void* stream) {
+    Problem pr;
+    fp2_status st = check_problem(params, q, k_pool, v_pool, cu_seqlens, batch, total_tokens,
+                                  max_seqlen, workspace, ws_bytes, &pr);
+    if (st != FP2_OK) return st;
+    if ((st = check_meta(meta, params, pr, true)) != FP2_OK) return st;
+    if (batch > 0 && (!block_table || max_blocks_per_seq < 1 || num_pages < 1)) return FP2_ERR_INVALID_ARG;
+    if (total_tokens > 0 && (!out || !aligned(out, 16))) return FP2_ERR_INVALID_ARG;
+    if (lse && !aligned(lse, 4)) return FP2_ERR_INVALID_ARG;
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if ((st = run_estimate(params, q, k_pool, v_pool, cu_seqlens, pr, block_table, max_blocks_per_seq,
+                           num_pages, meta, workspace, s)) != FP2_OK)
+        return st;
+    return run_attention(params, q, k_pool, v_pool, cu_seqlens, pr, block_table, max_blocks_per_seq,
+                         num_pages, meta, out, lse, workspace, s, false);
+}
+
+fp2_status fp2_get_error(void* workspace, void* stream) {
+    if (!workspace || !aligned(workspace, 256)) return FP2_ERR_WORKSPACE;
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int32_t h[2] = {0, 0};
+    if (cudaMemcpyAsync(h, workspace, sizeof(h), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
+        return FP2_ERR_CUDA;
+    if (h[0] != 0) {
+        if (cudaMemsetAsync(workspace, 0, 2 * sizeof(int32_t), s) != cudaSuccess ||
+            cudaStreamSynchronize(s) != cudaSuccess)
+            return FP2_ERR_CUDA;
+    }
+    return static_cast<fp2_status>(h[0]);
+}
+
+const char* fp2_status_string(fp2_status status) {
+    switch (status) {
+        case FP2_OK: return "ok";
+        case FP2_ERR_INVALID_ARG: return "invalid argument";
+        case FP2_ERR_UNSUPPORTED: return "unsupported configuration";
+        case FP2_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+        case FP2_ERR_CUDA: return "CUDA call or kernel launch failed";
+        case FP2_ERR_TIMEOUT: return "device pipeline wait timed out";
+        case FP2_ERR_BAD_INDEX: return "bad cu_seqlens or page index";
+    }
+    return "unknown status";
+}
+
+int32_t fp2_version(void) { return 100; }
+
+}  // extern "C"

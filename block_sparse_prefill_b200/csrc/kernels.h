@@ -1,0 +1,111 @@
+// kernels.h -- argument blocks and declarations of the device kernels.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+
+#include "common.cuh"
+
+namespace fp2 {
+
+constexpr int kPoolThreads = 512;  // 4 row groups x 128 column lanes
+constexpr int kScoreKC = 64;       // key blocks per shared-memory chunk in score_kernel
+
+struct SetupArgs {
+    const int32_t* cu;
+    int32_t batch;
+    int64_t total_tokens;
+    int32_t max_seqlen;
+    int32_t qt;  // q-blocks per estimator tile
+    int32_t paged;
+    int32_t max_blocks_per_seq;
+    int64_t max_blocks;
+    WsHeader* hdr;
+    int32_t* cu_blocks;
+    int32_t* cu_tiles;
+    int32_t* blk_req;
+};
+
+struct PoolArgs {
+    const void* x[3];        // q, k, v (k/v may be page pools)
+    float* out[3];           // qbar, k_mean, v_mean
+    const float* scale[3];   // per-head dequantisation scales (NULL = 1)
+    int32_t heads[3];
+    int32_t slabs[3];        // CTAs per block along the columns of each tensor
+    int32_t paged[3];
+    int32_t ntensors;        // 2 (q, k) or 3 (q, k, v)
+    const int32_t* cu;
+    const int32_t* cu_blocks;
+    const int32_t* blk_req;
+    const int32_t* block_table;
+    int32_t max_blocks_per_seq;
+    int32_t num_pages;
+    WsHeader* hdr;
+};
+
+struct ScoreArgs {
+    const float* qbar;   // [max_blocks, Hq, d]
+    const float* kbar;   // [max_blocks, Hkv, d]
+    const int32_t* cu_blocks;
+    const int32_t* cu_tiles;
+    int32_t batch;
+    int32_t hq, hkv, G;
+    int32_t qt, rp, ncap, nb_max;
+    float tau, ln_alpha;
+    int32_t keep_all;
+    int32_t* kept_cnt;
+    int32_t* kept_idx;
+    float* score_dbg;
+    WsHeader* hdr;
+};
+
+struct MeanLpArgs {
+    const float* k_mean;
+    const float* v_mean;
+    void* k_lp;
+    void* v_lp;
+    const float* k_scale;
+    const float* v_scale;
+    int32_t hkv;
+    int32_t e4m3;
+    int64_t max_blocks;   // rows of k_lp / v_lp; rows past the last block are zeroed
+    WsHeader* hdr;
+};
+
+struct AttnArgs {
+    const int32_t* cu;
+    const int32_t* cu_blocks;
+    const int32_t* blk_req;
+    const int32_t* block_table;  // NULL = contiguous K/V
+    int32_t max_blocks_per_seq;
+    int32_t num_pages;
+    const int32_t* kept_cnt;
+    const int32_t* kept_idx;
+    int32_t nb_max;              // row stride of kept_idx
+    int32_t nb_cap;              // >= key blocks of the longest request (shared-memory lists)
+    int32_t hq, hkv, G, pairs;   // pairs = ceil(G / 2) CTAs per (q-block, KV head)
+    int32_t correction;
+    float scale_log2;            // tau * log2(e)
+    const float* q_scale;        // e4m3 only
+    const float* k_scale;
+    const float* v_scale;
+    void* out;                   // bf16 [T, Hq, d]
+    float* lse;                  // [T, Hq] or NULL
+    WsHeader* hdr;
+};
+
+__global__ void setup_kernel(SetupArgs a);
+template <bool kE4M3>
+__global__ void pool_kernel(PoolArgs a);
+__global__ void score_kernel(ScoreArgs a);
+__global__ void meanlp_kernel(MeanLpArgs a);
+
+// Shared-memory bytes of the attention kernel for a kept-list capacity.
+size_t attn_smem_bytes(bool e4m3, int32_t nb_cap);
+// Launches the attention kernel (one CTA per (q-block, KV head, query-head pair)).
+cudaError_t launch_attention(bool e4m3, const AttnArgs& a, const CUtensorMap& tq,
+                             const CUtensorMap& tk, const CUtensorMap& tv,
+                             const CUtensorMap& tkb, const CUtensorMap& tvb, int64_t max_blocks,
+                             cudaStream_t stream);
+
+}  // namespace fp2

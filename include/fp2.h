@@ -1,0 +1,173 @@
+/*
+ * fp2.h -- C ABI of the B200 (sm_100a) block-sparse prefill attention library.
+ *
+ * The method (write-ups of "FlashPrefill V2: Block-Sparse Prefill Attention for
+ * Long-Context LLM Serving"):
+ *   - lode.cx, "How It Works": a block-level sample of attention scores, its
+ *     maximum, and a threshold relative to that maximum pick the attended
+ *     blocks; a mean correction term compensates the pruned mass;
+ *   - aipulsen.com: scores are estimated at the block level;
+ *   - aimodeling.com, "From Prototype to Production": max-based dynamic
+ *     thresholding, the mean correction term, FP8, paged KV cache and
+ *     continuous batching;
+ *   - stuffinsider.com, "Technical Details": queries and keys are cut into
+ *     blocks; prefill only.
+ * The write-ups fix these steps only in words.  The exact readings used here:
+ *   blocks   block_size rows from the first token of each request; causal
+ *            (token r sees keys c <= r of its own request);
+ *   estimate qbar/kbar/vbar = per-block means of the (dequantised) rows;
+ *            s[h,i,j] = sm_scale * qbar[h,i] . kbar[h/G, j] for j <= i;
+ *   keep     m = max_j s; head h keeps j iff s - m >= ln(alpha); a KV head keeps
+ *            the union over its G query heads plus the diagonal block;
+ *            alpha <= 0 keeps every causal block;
+ *   attend   softmax attention over kept blocks; with correction, each pruned
+ *            block j < i adds n_j * exp(sm_scale q.kbar_j) * vbar_j to the
+ *            numerator and n_j * exp(sm_scale q.kbar_j) to the denominator.
+ *
+ * Layouts (all row-major, token-major "THD"):
+ *   q        [total_tokens, Hq, head_dim]          bf16 or e4m3
+ *   k, v     [total_tokens, Hkv, head_dim]         contiguous mode
+ *   k_pool   [num_pages * block_size, Hkv, head_dim] paged mode; page p holds
+ *            rows p*block_size .. p*block_size + block_size - 1
+ *   out      [total_tokens, Hq, head_dim]          bf16
+ *   lse      [total_tokens, Hq]                    fp32 natural-log sum-exp
+ *   cu_seqlens [batch + 1] int32, cu_seqlens[0] = 0, non-decreasing,
+ *            cu_seqlens[batch] = total_tokens; request b is rows
+ *            cu_seqlens[b] .. cu_seqlens[b+1]-1 of q (and of k/v when contiguous)
+ *   block_table [batch, max_blocks_per_seq] int32: page of logical block j of
+ *            request b (paged mode).
+ *   Blocks of all requests are numbered globally in request order:
+ *   block id of (b, j) = sum_{b' < b} ceil(L_b' / block_size) + j.
+ *
+ * Ownership: every pointer passed to a compute call is a DEVICE pointer owned
+ * by the caller, except the fp2_params / fp2_blockmeta structs themselves,
+ * which are read on the host during the call.  The library allocates no memory
+ * and keeps no global state; scratch memory is the caller's workspace.
+ *
+ * Errors: argument errors are returned synchronously and nothing is enqueued.
+ * A failed launch returns FP2_ERR_CUDA.  Errors found on the device (a bad
+ * cu_seqlens, a page index outside the pool, a wait that ran out of time) are
+ * recorded in a flag inside the workspace; the kernels then skip the bad
+ * access and the call's results are undefined.  fp2_get_error() reads and
+ * clears that flag.
+ *
+ * All compute calls are asynchronous on `stream` (a cudaStream_t, NULL = the
+ * legacy default stream).  Calls sharing one workspace must be ordered on the
+ * device (same stream, or synchronised streams).
+ */
+#ifndef FP2_H
+#define FP2_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum fp2_status {
+    FP2_OK = 0,
+    FP2_ERR_INVALID_ARG = 1,   /* bad argument; nothing was enqueued */
+    FP2_ERR_UNSUPPORTED = 2,   /* valid but not implemented (e.g. head_dim != 128) */
+    FP2_ERR_WORKSPACE = 3,     /* workspace missing, misaligned or too small */
+    FP2_ERR_CUDA = 4,          /* a CUDA runtime/driver call or launch failed */
+    FP2_ERR_TIMEOUT = 5,       /* device: a pipeline wait exceeded its limit */
+    FP2_ERR_BAD_INDEX = 6      /* device: bad cu_seqlens or page index */
+} fp2_status;
+
+typedef enum fp2_dtype {
+    FP2_BF16 = 0,              /* q/k/v bf16 */
+    FP2_E4M3 = 1               /* q/k/v float8 e4m3 codes with per-head scales */
+} fp2_dtype;
+
+/* Problem parameters (read on the host). */
+typedef struct fp2_params {
+    int32_t num_q_heads;       /* Hq >= 1 */
+    int32_t num_kv_heads;      /* Hkv >= 1, Hq % Hkv == 0 (G = Hq / Hkv query heads per KV head) */
+    int32_t head_dim;          /* must be 128 */
+    int32_t block_size;        /* must be 128; also the KV page size */
+    float alpha;               /* threshold; <= 0 keeps every causal block; must be <= 1 */
+    float sm_scale;            /* softmax scale tau; 0 selects 1/sqrt(head_dim) */
+    int32_t correction;        /* 0: drop pruned blocks; 1: mean correction */
+    int32_t dtype;             /* fp2_dtype */
+    const float* q_scale;      /* e4m3 only: device [Hq] dequantisation scales */
+    const float* k_scale;      /* e4m3 only: device [Hkv] */
+    const float* v_scale;      /* e4m3 only: device [Hkv] */
+} fp2_params;
+
+/* Block metadata written by the estimator and read by the attention calls.
+ * All arrays are device memory owned by the caller. */
+typedef struct fp2_blockmeta {
+    int32_t* kept_cnt;         /* [max_blocks, Hkv]: number of kept key blocks */
+    int32_t* kept_idx;         /* [max_blocks, Hkv, nb_max]: kept key blocks of every
+                                  q-block, ascending, diagonal block last */
+    float* k_mean;             /* [max_blocks, Hkv, head_dim] fp32 dequantised block means */
+    float* v_mean;             /* [max_blocks, Hkv, head_dim] fp32; needed when correction != 0 */
+    float* score_dbg;          /* optional (NULL): [max_blocks, Hq, nb_max] s - m, fp32;
+                                  entries j > i are left untouched */
+    int32_t nb_max;            /* row stride of kept_idx / score_dbg, >= ceil(max_seqlen / block_size) */
+    int32_t max_blocks;        /* capacity in blocks, >= sum_b ceil(L_b / block_size) */
+} fp2_blockmeta;
+
+/* Upper bound of sum_b ceil(L_b / block_size) for any batch of `batch` requests
+ * holding `total_tokens` tokens: total_tokens / block_size + batch. */
+int64_t fp2_max_blocks(int32_t batch, int64_t total_tokens, int32_t block_size);
+
+/* Workspace bytes needed by every call below for this problem size (an upper
+ * bound independent of the lengths inside cu_seqlens).  Returns 0 for invalid
+ * arguments. */
+size_t fp2_workspace_bytes(const fp2_params* params, int32_t batch, int64_t total_tokens,
+                           int32_t max_seqlen);
+
+/* Clears the workspace's device error flag (enqueued on `stream`).  Call once
+ * on a new workspace before its first use. */
+fp2_status fp2_workspace_init(void* workspace, size_t ws_bytes, void* stream);
+
+/* Estimator (block means, block scores, row max, alpha threshold, GQA union,
+ * compaction).  Writes meta->kept_cnt, kept_idx, k_mean, v_mean (v_mean only
+ * when non-NULL) and score_dbg (when non-NULL).
+ *   q            [total_tokens, Hq, d]
+ *   k, v         contiguous [total_tokens, Hkv, d] when block_table == NULL,
+ *                else page pools [num_pages * block_size, Hkv, d]
+ *   block_table  NULL (contiguous) or [batch, max_blocks_per_seq] page indices
+ *   num_pages    pages in the pools (paged mode; ignored otherwise) */
+fp2_status fp2_estimate(const fp2_params* params, const void* q, const void* k, const void* v,
+                        const int32_t* cu_seqlens, int32_t batch, int64_t total_tokens,
+                        int32_t max_seqlen, const int32_t* block_table,
+                        int32_t max_blocks_per_seq, int32_t num_pages, fp2_blockmeta* meta,
+                        void* workspace, size_t ws_bytes, void* stream);
+
+/* Sparse attention over the kept blocks of `meta` (from fp2_estimate on the
+ * same inputs) with contiguous K/V, plus the mean correction when
+ * params->correction != 0.  Writes out (bf16) and, when non-NULL, lse. */
+fp2_status fp2_sparse_prefill(const fp2_params* params, const void* q, const void* k,
+                              const void* v, const int32_t* cu_seqlens, int32_t batch,
+                              int64_t total_tokens, int32_t max_seqlen,
+                              const fp2_blockmeta* meta, void* out, float* lse, void* workspace,
+                              size_t ws_bytes, void* stream);
+
+/* One whole prefill attention layer on a paged KV cache: fp2_estimate on the
+ * page pools (writing `meta`) followed by the sparse attention, whose K/V
+ * tiles are fetched page by page through block_table. */
+fp2_status fp2_prefill_paged(const fp2_params* params, const void* q, const void* k_pool,
+                             const void* v_pool, const int32_t* cu_seqlens, int32_t batch,
+                             int64_t total_tokens, int32_t max_seqlen, const int32_t* block_table,
+                             int32_t max_blocks_per_seq, int32_t num_pages, fp2_blockmeta* meta,
+                             void* out, float* lse, void* workspace, size_t ws_bytes,
+                             void* stream);
+
+/* Synchronises `stream`, returns the first device-side error recorded in the
+ * workspace since the last call (FP2_OK if none) and clears it. */
+fp2_status fp2_get_error(void* workspace, void* stream);
+
+/* Static description of a status code. */
+const char* fp2_status_string(fp2_status status);
+
+/* Library version (major * 10000 + minor * 100 + patch). */
+int32_t fp2_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP2_H */

@@ -1,0 +1,133 @@
+"""GPU (sm_100a) path against the CPU oracle, through the C ABI.
+
+Masks: bit-exact except at blocks whose oracle score lies within 1e-3
+(relative) of the threshold.  Outputs, given the GPU's mask (the oracle is
+re-run with it): bf16 max-abs 2e-2 and mean-abs 2e-3, e4m3 max-abs 6e-2.
+LSE (natural log): max-abs 2e-2 for bf16 and 6e-2 for e4m3 (the attention
+weights are rounded to the MMA precision before the PV product).
+"""
+import numpy as np
+import pytest
+import torch
+
+from gpu_helpers import (BF16_MAX_ABS, BF16_MEAN_ABS, E4M3_MAX_ABS, compare_masks, oracle,
+                         out_errors, rows_of_blocks, run_gpu, sample_blocks, tau)
+from workloads import make_config, make_workload
+
+pytestmark = pytest.mark.gpu
+
+
+def _kept(g):
+    return {"kept_cnt": g["kept_cnt"], "kept_idx": g["kept_idx"]}
+
+
+def _check_outputs(wl, g, correction, sel=None, max_abs=BF16_MAX_ABS, mean_abs=BF16_MEAN_ABS, lse_abs=2e-2):
+    orc = oracle()
+    ref = orc.run(wl, kept=_kept(g), correction=correction, sel=sel)
+    rows = None if sel is None else rows_of_blocks(wl.cu_seqlens, sel)
+    mx, mn = out_errors(g["o"], ref["o"], rows)
+    assert mx <= max_abs and mn <= mean_abs, f"output max-abs {mx:.3e} mean-abs {mn:.3e}"
+    if g["lse"] is not None:
+        lm, _ = out_errors(g["lse"], ref["lse"], rows)
+        assert lm < lse_abs, f"lse max-abs {lm:.3e}"
+    return mx, mn
+
+
+def _check_masks(wl, g, alpha=None):
+    orc = oracle()
+    a = wl.alpha if alpha is None else alpha
+    est = orc.run(wl, alpha=a, want_scores=True, sel=np.zeros(0, np.int64))
+    bad, near, total = compare_masks(g, est, a, wl.num_kv_heads)
+    assert bad == 0, f"{bad} kept-list entries differ outside the near-threshold band ({near} near, {total} total)"
+    # block means
+    assert np.abs(g["k_mean"] - est["kbar"]).max() < 1e-4 * max(1.0, np.abs(est["kbar"]).max())
+    return est
+
+
+@pytest.mark.parametrize("correction", [True, False])
+def test_tiny_config(correction):
+    wl = make_config(0)
+    g = run_gpu(wl, correction=correction)
+    _check_masks(wl, g)
+    _check_outputs(wl, g, correction)
+
+
+def test_dense_alpha_zero():
+    wl = make_workload([1000, 300], 4, 2, alpha=0.0, seed=3)
+    g = run_gpu(wl, alpha=0.0)
+    nb = [(L + 127) // 128 for L in wl.seqlens]
+    full = np.concatenate([np.arange(1, n + 1) for n in nb])
+    assert (g["kept_cnt"] == full[:, None]).all(), "alpha <= 0 must keep every causal block"
+    _check_outputs(wl, g, True)
+
+
+@pytest.mark.parametrize("G", [1, 2, 3, 4])
+def test_ragged_edges(G):
+    wl = make_workload([1, 127, 129, 200, 383, 700], 2 * G, 2, alpha=0.2, seed=10 + G, n_retrieval=1)
+    g = run_gpu(wl)
+    _check_masks(wl, g)
+    _check_outputs(wl, g, True)
+
+
+def test_llama_shape_4k():
+    wl = make_config(1, seqlen=4096)
+    g = run_gpu(wl, scores=True)
+    est = _check_masks(wl, g)
+    _check_outputs(wl, g, True)
+    # score_dbg = s - m
+    s_rel = est["s"] - est["m"][:, :, None]
+    m = ~np.isnan(s_rel)
+    assert np.abs(g["score_dbg"][m] - s_rel[m]).max() < 1e-3
+
+
+@pytest.mark.parametrize("alpha", [0.02, 0.05, 0.1, 0.2])
+def test_llama_shape_32k_sweep(alpha):
+    wl = make_config(1, alpha=alpha)
+    g = run_gpu(wl)
+    _check_masks(wl, g)
+    nblk = g["kept_cnt"].shape[0]
+    sel = sample_blocks(nblk, 12, seed=int(alpha * 1000), include=(0, nblk - 1))
+    _check_outputs(wl, g, True, sel=sel)
+
+
+def test_128k_bf16_sampled():
+    wl = make_config(2)
+    g = run_gpu(wl)
+    _check_masks(wl, g)
+    nblk = g["kept_cnt"].shape[0]
+    sel = sample_blocks(nblk, 16, seed=2, include=(0, nblk - 1))
+    _check_outputs(wl, g, True, sel=sel)
+
+
+def test_e4m3_4k():
+    wl = make_config(3, seqlen=4096)
+    g = run_gpu(wl)
+    _check_masks(wl, g)
+    _check_outputs(wl, g, True, max_abs=E4M3_MAX_ABS, mean_abs=1.0, lse_abs=E4M3_MAX_ABS)
+
+
+def test_128k_e4m3_sampled():
+    wl = make_config(3)
+    g = run_gpu(wl)
+    _check_masks(wl, g)
+    nblk = g["kept_cnt"].shape[0]
+    sel = sample_blocks(nblk, 16, seed=3, include=(0, nblk - 1))
+    _check_outputs(wl, g, True, sel=sel, max_abs=E4M3_MAX_ABS, mean_abs=1.0, lse_abs=E4M3_MAX_ABS)
+
+
+def test_paged_equals_contiguous_small():
+    wl = make_workload([900, 130, 2000, 1], 8, 2, alpha=0.1, seed=41, paged=True)
+    gp = run_gpu(wl, paged=True)
+    gc = run_gpu(wl, paged=False)
+    assert (gp["kept_cnt"] == gc["kept_cnt"]).all() and (gp["kept_idx"] == gc["kept_idx"]).all()
+    assert np.array_equal(gp["o"], gc["o"], equal_nan=True), "paged output differs from contiguous"
+    _check_outputs(wl, gp, True)
+
+
+def test_paged_ragged_batch_sampled():
+    wl = make_config(4, seqlen=32768)
+    g = run_gpu(wl, paged=True)
+    _check_masks(wl, g)
+    nblk = g["kept_cnt"].shape[0]
+    sel = sample_blocks(nblk, 16, seed=4, include=(0, nblk - 1))
+    _check_outputs(wl, g, True, sel=sel)
