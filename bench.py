@@ -1,0 +1,478 @@
+"""Benchmark of one block-sparse prefill attention layer on B200.
+
+One step = one whole layer of the path: fp2_estimate (block means, block
+scores, row max, alpha threshold, GQA union) followed by fp2_sparse_prefill
+(tcgen05 attention over the kept blocks plus the mean correction), on the
+128K-token Llama-3-8B-shaped workload (B=1, Hq=32, Hkv=8, d=128, bf16,
+alpha=0.05; seeded synthetic inputs, which are larger than the 126 MB L2).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line.  `value` is the effective TFLOP/s of the whole layer:
+the attention work on the kept blocks (4*d per query-key pair, the diagonal
+block counted causally) divided by the device time of estimator + attention.
+Under torchrun (N > 1) every rank runs its own independent layer (weak
+scaling, no collective on the data path); time is the max over ranks.
+`--impl reference` times the CPU oracle on a bounded sample of the same layer.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "ms/layer & effective TFLOP/s at 128K prefill (BF16/FP8); % of tensor-core peak"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+E4M3_OVER_BF16 = 2.0  # nominal dense ratio (4.5 / 2.25 PFLOP/s)
+
+
+def load_peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------------------
+# algorithmic work of a layer (from the kept lists)
+# ---------------------------------------------------------------------------
+def layer_work(seqlens, kept_cnt, kept_idx, hq, hkv, d=128, bs=128, correction=True):
+    """Returns (kept-pair flops, correction flops) for 4*d flops per pair."""
+    G = hq // hkv
+    pairs = 0
+    corr = 0
+    t = 0
+    for L in seqlens:
+        nb = (L + bs - 1) // bs
+        n = np.minimum(bs, L - np.arange(nb) * bs)              # rows of each block
+        for i in range(nb):
+            ni = int(n[i])
+            for g in range(hkv):
+                c = int(kept_cnt[t, g])
+                js = kept_idx[t, g, :c]
+                off = js[js < i]
+                p = ni * int(n[off].sum()) + ni * (ni + 1) // 2   # diagonal counted causally
+                pairs += G * p
+                if correction:
+                    corr += G * ni * (i - len(off))
+            t += 1
+    return 4.0 * d * pairs, 4.0 * d * corr
+
+
+# ---------------------------------------------------------------------------
+# clocks sampler (nvidia-smi, during the timed region)
+# ---------------------------------------------------------------------------
+class Clocks:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        import torch
+        self.proc = None
+        self.lines = []
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            ident = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+        except Exception:
+            ident = str(device_index)
+        self.ident = ident
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.ident, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        rows = [r.split(",") for r in out.strip().splitlines() if r.strip()]
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            r = [x.strip() for x in r]
+            if len(r) < 9:
+                continue
+            try:
+                sm.append(float(r[1]))
+                smax.append(float(r[2]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, r[5:9]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+def setup_layer(wl, dev):
+    import torch
+    import block_sparse_prefill_b200 as fp2
+    e4m3 = wl.dtype == "e4m3"
+    params = fp2.Params(num_q_heads=wl.num_q_heads, num_kv_heads=wl.num_kv_heads, alpha=wl.alpha,
+                        correction=True, dtype=fp2.FP2_E4M3 if e4m3 else fp2.FP2_BF16)
+    if e4m3:
+        params.q_scale = torch.from_numpy(wl.q_scale).to(dev)
+        params.k_scale = torch.from_numpy(wl.k_scale).to(dev)
+        params.v_scale = torch.from_numpy(wl.v_scale).to(dev)
+    T, B = wl.total_tokens, wl.batch
+    st = {
+        "params": params,
+        "q": wl.q.to(dev), "k": wl.k.to(dev), "v": wl.v.to(dev),
+        "cu": torch.from_numpy(wl.cu_seqlens).to(dev),
+        "meta": fp2.BlockMeta.empty(params, B, T, wl.max_seqlen, dev),
+        "ws": fp2.Workspace(params, B, T, wl.max_seqlen, dev),
+        "out": torch.empty((T, wl.num_q_heads, 128), dtype=torch.bfloat16, device=dev),
+        "lse": torch.empty((T, wl.num_q_heads), dtype=torch.float32, device=dev),
+    }
+    return st
+
+
+def run_layer(st, wl, stream, q=None, k=None, v=None):
+    import block_sparse_prefill_b200 as fp2
+    q = st["q"] if q is None else q
+    k = st["k"] if k is None else k
+    v = st["v"] if v is None else v
+    fp2.estimate(st["params"], q, k, v, st["cu"], wl.max_seqlen, st["meta"], st["ws"], stream=stream)
+    fp2.sparse_prefill(st["params"], q, k, v, st["cu"], wl.max_seqlen, st["meta"], st["out"], st["ws"],
+                       lse=st["lse"], stream=stream)
+
+
+def time_layer(st, wl, steps, warmup, dist_ctx, clocks=None):
+    """Device time of `steps` layers on one stream (CUDA events per call)."""
+    import torch
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        run_layer(st, wl, stream)
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dist_ctx.barrier()
+    torch.cuda.synchronize()
+    if clocks:
+        clocks.start()
+    e0.record(stream)
+    for s in range(steps):
+        ev[s][0].record(stream)
+        import block_sparse_prefill_b200 as fp2
+        fp2.estimate(st["params"], st["q"], st["k"], st["v"], st["cu"], wl.max_seqlen, st["meta"], st["ws"],
+                     stream=stream)
+        ev[s][1].record(stream)
+        fp2.sparse_prefill(st["params"], st["q"], st["k"], st["v"], st["cu"], wl.max_seqlen, st["meta"],
+                           st["out"], st["ws"], lse=st["lse"], stream=stream)
+        ev[s][2].record(stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop() if clocks else None
+    dist_ctx.barrier()
+    total = e0.elapsed_time(e1)
+    est = [ev[s][0].elapsed_time(ev[s][1]) for s in range(steps)]
+    att = [ev[s][1].elapsed_time(ev[s][2]) for s in range(steps)]
+    return total, est, att, clk
+
+
+def time_e2e(st, wl, steps, dist_ctx):
+    """Same layer through the C ABI with host buffers: pinned H2D of Q/K/V and
+    D2H of the output inside the timed region."""
+    import torch
+    stream = torch.cuda.current_stream()
+    hq = wl.q.pin_memory()
+    hk = wl.k.pin_memory()
+    hv = wl.v.pin_memory()
+    ho = torch.empty(st["out"].shape, dtype=st["out"].dtype).pin_memory()
+    dq, dk, dv = torch.empty_like(st["q"]), torch.empty_like(st["k"]), torch.empty_like(st["v"])
+
+    def one():
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        run_layer(st, wl, stream, dq, dk, dv)
+        ho.copy_(st["out"], non_blocking=True)
+
+    one()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dist_ctx.barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(steps):
+        one()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    dist_ctx.barrier()
+    h2d = hq.numel() * hq.element_size() + hk.numel() * hk.element_size() + hv.numel() * hv.element_size()
+    d2h = ho.numel() * ho.element_size()
+    return e0.elapsed_time(e1) / steps, h2d, d2h
+
+
+class DistCtx:
+    def __init__(self):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = None
+
+    def init(self, backend="nccl"):
+        if self.world > 1:
+            import datetime
+            import torch.distributed as dist
+            dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=600))
+            self.pg = dist
+
+    def barrier(self):
+        if self.pg is not None:
+            import torch
+            self.pg.barrier(device_ids=[torch.cuda.current_device()])
+
+    def max(self, x: float) -> float:
+        if self.pg is None:
+            return x
+        import torch
+        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg is not None:
+            self.pg.destroy_process_group()
+
+
+def cpu_baseline(wl, fracs=(0.25, 0.5)):
+    """The oracle (fp64, OpenMP over host cores) on a bounded sample of the
+    layer: the full estimator, plus attention on the q-blocks at the given
+    fractions of the sequence (all heads); the per-layer time is extrapolated
+    from the sample by its share of the layer's attention work."""
+    from oracle.oracle import Oracle
+    orc = Oracle()
+    q, k, v = wl.float_inputs()
+    cu = wl.cu_seqlens
+    t0 = time.perf_counter()
+    qb = orc.block_means(q, cu, 128, wl.q_scale)
+    kb = orc.block_means(k, cu, 128, wl.k_scale)
+    vb = orc.block_means(v, cu, 128, wl.v_scale)
+    est = orc.estimate(qb, kb, cu, 128, wl.alpha, 1.0 / math.sqrt(wl.head_dim))
+    t_est = time.perf_counter() - t0
+    nblk = est["kept_cnt"].shape[0]
+    sel = np.unique(np.array([min(nblk - 1, int(f * nblk)) for f in fracs], dtype=np.int64))
+    t1 = time.perf_counter()
+    orc.attend(q, k, v, cu, 128, 1.0 / math.sqrt(wl.head_dim), est["kept_cnt"], est["kept_idx"], correction=True,
+               kbar=kb, vbar=vb, q_scale=wl.q_scale, k_scale=wl.k_scale, v_scale=wl.v_scale, sel=sel)
+    t_att = time.perf_counter() - t1
+    # share of the layer's attention work inside the sample
+    flops_all, corr_all = layer_work(wl.seqlens, est["kept_cnt"], est["kept_idx"], wl.num_q_heads,
+                                     wl.num_kv_heads)
+    sub_cnt = est["kept_cnt"][sel]
+    sub_idx = est["kept_idx"][sel]
+    # work of the sampled blocks: rebuild per-block work with the block index i
+    G = wl.num_q_heads // wl.num_kv_heads
+    fs = 0.0
+    for r, t in enumerate(sel):
+        i = int(t)
+        for g in range(wl.num_kv_heads):
+            js = sub_idx[r, g, :sub_cnt[r, g]]
+            fs += G * (128 * 128 * int((js < i).sum()) + 128 * 129 // 2 + 128 * (i - int((js < i).sum())))
+    fs *= 4.0 * wl.head_dim
+    frac = fs / max(flops_all + corr_all, 1.0)
+    t_layer = t_est + t_att / max(frac, 1e-12)
+    cores = os.cpu_count() or 1
+    try:
+        cores = len(os.sched_getaffinity(0))
+    except AttributeError:
+        pass
+    omp = int(os.environ.get("OMP_NUM_THREADS", cores))
+    return {
+        "value": flops_all / t_layer / 1e12, "unit": "TFLOP/s", "cores": min(cores, omp), "kind": "oracle",
+        "ms_per_layer": t_layer * 1e3,
+        "sample": (f"fp64 oracle: full estimator ({t_est:.1f} s) + attention on {len(sel)} of {nblk} "
+                   f"q-blocks {sel.tolist()}, all heads ({t_att:.1f} s, {100 * frac:.2f}% of the layer's "
+                   "attention work); "
+                   "layer time extrapolated by work share"),
+    }
+
+
+def ours(args):
+    import torch
+    ctx = DistCtx()
+    torch.cuda.set_device(ctx.local_rank)
+    ctx.init("nccl")
+    dev = torch.device("cuda", ctx.local_rank)
+    from workloads import make_config
+    import block_sparse_prefill_b200 as fp2
+    peaks, peaks_kind = load_peaks()
+
+    wl = make_config(2, seed=1002 + ctx.rank, seqlen=args.seqlen)
+    st = setup_layer(wl, dev)
+    clocks = Clocks(ctx.local_rank)
+    total, est, att, clk = time_layer(st, wl, args.steps, args.warmup, ctx, clocks)
+    err = fp2.get_error(st["ws"])
+    if err != 0:
+        raise RuntimeError(f"device error: {fp2.status_string(err)}")
+    nblk = fp2.max_blocks(wl.batch, wl.total_tokens)
+    kept_cnt = st["meta"].kept_cnt.cpu().numpy()
+    kept_idx = st["meta"].kept_idx.cpu().numpy()
+    flops, corr_flops = layer_work(wl.seqlens, kept_cnt, kept_idx, wl.num_q_heads, wl.num_kv_heads)
+    nb = (wl.max_seqlen + 127) // 128
+    density = float(kept_cnt[:nb].sum()) / (wl.num_kv_heads * nb * (nb + 1) / 2)
+    ms_step = ctx.max(total / args.steps)
+    ms_est = statistics.mean(est)
+    ms_att = statistics.mean(att)
+    value = ctx.world * flops / (ms_step * 1e-3) / 1e12
+
+    e2e = None
+    if not args.no_e2e:
+        e2e_ms, h2d, d2h = time_e2e(st, wl, max(1, min(3, args.steps)), ctx)
+        e2e_ms = ctx.max(e2e_ms)
+        e2e = {"value": ctx.world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    # e4m3 variant of the same layer (config 3), kernel-timed
+    fp8 = None
+    if not args.no_fp8:
+        del st
+        torch.cuda.empty_cache()
+        wl8 = make_config(3, seed=1002 + ctx.rank, seqlen=args.seqlen)
+        st8 = setup_layer(wl8, dev)
+        tot8, est8, att8, _ = time_layer(st8, wl8, args.steps, args.warmup, ctx)
+        f8, c8 = layer_work(wl8.seqlens, st8["meta"].kept_cnt.cpu().numpy(), st8["meta"].kept_idx.cpu().numpy(),
+                            wl8.num_q_heads, wl8.num_kv_heads)
+        ms8 = ctx.max(tot8 / args.steps)
+        a8 = statistics.mean(att8)
+        peak8 = peaks["bf16_tflops"] * E4M3_OVER_BF16
+        fp8 = {
+            "config": f"{wl8.max_seqlen // 1024}K e4m3 (Hq=32, Hkv=8, d=128, alpha=0.05)",
+            "ms_per_layer": ms8, "ms_estimate": statistics.mean(est8), "ms_attention": a8,
+            "tflops_layer": ctx.world * f8 / (ms8 * 1e-3) / 1e12,
+            "tflops_attention": (f8 + c8) / (a8 * 1e-3) / 1e12,
+            "tensor_peak_tflops": peak8,
+            "frac_attention": (f8 + c8) / (a8 * 1e-3) / 1e12 / peak8,
+            "peak_note": f"e4m3 peak = {peaks_kind} bf16 burst x {E4M3_OVER_BF16} (nominal dense ratio)",
+        }
+        del st8
+
+    # roofline of the dominant kernel (the attention call: attention kernel +
+    # two small set-up launches) and the estimator (HBM)
+    ach_att = (flops + corr_flops) / (ms_att * 1e-3) / 1e12
+    est_bytes = wl.total_tokens * (wl.num_q_heads + 2 * wl.num_kv_heads) * 128 * 2
+    est_gbs = est_bytes / (ms_est * 1e-3) / 1e9
+    line = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "TFLOP/s",
+        "n_gpus": ctx.world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {
+            "workload": f"{wl.max_seqlen // 1024}K Llama-3-8B-shaped block-sparse prefill layer (B=1, "
+                        f"S={wl.max_seqlen}, Hq=32, Hkv=8, d=128, bf16, alpha=0.05, mean correction on)",
+            "global_batch": ctx.world, "seq_len": wl.max_seqlen, "parallelism": f"independent layers x{ctx.world}",
+            "l2": f"inputs ({est_bytes / 1e9:.2f} GB) larger than L2; no flush",
+            "kept_density": density,
+        },
+        "ms_per_layer": ms_step,
+        "ms_estimate": ms_est,
+        "ms_attention": ms_att,
+        "tflops_attention": ach_att,
+        "roofline": {
+            "bound": "tensor", "achieved": ach_att, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+            "frac": ach_att / peaks["bf16_tflops"], "traffic": None,
+            "kernel": "attention_kernel<bf16> (fp2_sparse_prefill call)",
+            "work": "4*d flops per kept causal query-key pair + 4*d per (row, pruned block) correction term",
+            "peak_kind": f"{peaks_kind} bf16 burst",
+        },
+        "estimator_roofline": {
+            "bound": "hbm", "achieved": est_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": est_gbs / peaks["hbm_gbs"], "bytes": est_bytes,
+            "kernel": "fp2_estimate call (pool + score kernels)",
+        },
+        "e2e": e2e,
+        "gpu_launches": args.steps * 6,
+        "clocks": clk,
+        "fp8": fp8,
+    }
+    if ctx.rank == 0 and ctx.world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl)
+    if ctx.rank == 0:
+        print(json.dumps(line), flush=True)
+    ctx.close()
+
+
+def reference(args):
+    """The CPU oracle as the reference arm, on bounded samples of the layer."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from workloads import make_config
+    wl = make_config(2)
+    vals = []
+    for _ in range(args.warmup):
+        pass  # the oracle has no warm-up state; warm-up steps are skipped
+    t0 = time.perf_counter()
+    last = None
+    for s in range(args.steps):
+        last = cpu_baseline(wl, fracs=((0.2 + 0.05 * (s % 4)), 0.5))
+        vals.append(last["value"])
+    wall = time.perf_counter() - t0
+    v = statistics.mean(vals)
+    line = {
+        "metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": int(os.environ.get("WORLD_SIZE", "1")),
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * wall / max(args.steps, 1),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "impl": "reference",
+        "config": {"workload": "128K Llama-3-8B-shaped block-sparse prefill layer (B=1, S=131072, Hq=32, Hkv=8, "
+                               "d=128, bf16 inputs, alpha=0.05, mean correction on)"},
+        "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": last["cores"], "kind": "oracle",
+                         "sample": last["sample"]},
+        "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-fp8", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--seqlen", type=int, default=None,
+                    help="shorter sequence for profiling runs (default: the 128K workload)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        reference(args)
+    else:
+        ours(args)
+
+
+if __name__ == "__main__":
+    main()

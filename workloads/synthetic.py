@@ -261,11 +261,14 @@ CONFIG_NAMES = {
 }
 
 
-def make_config(cid: int, alpha: Optional[float] = None, seqlen: Optional[int] = None) -> Workload:
+def make_config(cid: int, alpha: Optional[float] = None, seqlen: Optional[int] = None,
+                seed: Optional[int] = None) -> Workload:
     """The five workloads: tiny (0), 32K bf16 (1), 128K bf16 (2), 128K e4m3 (3),
-    paged ragged batch (4).  ``seqlen`` shrinks configs 1-3 for quick tests."""
+    paged ragged batch (4).  ``seqlen`` shrinks configs 1-3 for quick tests;
+    ``seed`` replaces the default seed (1000 + id; config 3 shares config 2's)."""
     # config 3 is config 2 encoded in e4m3, so both draw from seed 1002
-    seed = 1000 + (2 if cid == 3 else cid)
+    if seed is None:
+        seed = 1000 + (2 if cid == 3 else cid)
     if cid == 0:
         return make_workload([seqlen or 2048], 2, 1, alpha=0.1 if alpha is None else alpha,
                              seed=seed, n_retrieval=3, name=CONFIG_NAMES[0])
