@@ -22,7 +22,8 @@ from . import _lib
 from ._lib import FP2_BF16, FP2_E4M3, STATUS
 
 __all__ = ["Params", "BlockMeta", "Workspace", "FP2Error", "max_blocks", "workspace_bytes",
-           "estimate", "sparse_prefill", "prefill_paged", "get_error", "status_string", "version",
+           "estimate", "sparse_prefill", "sparse_prefill_noalloc", "prefill_paged", "get_error",
+           "status_string", "version",
            "FP2_BF16", "FP2_E4M3"]
 
 BLOCK = 128
@@ -171,6 +172,21 @@ def prefill_paged(params: Params, q, k_pool, v_pool, cu_seqlens, max_seqlen: int
                                          int(num_pages), ctypes.byref(m), _ptr(out), _ptr(lse), ws.ptr,
                                          ws.nbytes, _stream(stream)),
            "fp2_prefill_paged")
+
+
+def sparse_prefill_noalloc(params: Params, q, k, v, cu_seqlens, max_seqlen: int, meta: BlockMeta, out,
+                           lse=None, device_status=None, stream=None) -> None:
+    """``fp2_sparse_prefill_noalloc``: ``sparse_prefill`` without a workspace,
+    for callers that cannot allocate device memory where they run attention
+    (the library's own fixed device array serves as scratch).  The first call
+    on a device must come before any stream capture on it, and calls that
+    overlap on the GPU race on the shared array."""
+    p, m = params.c(), meta.c()
+    _check(_lib.load().fp2_sparse_prefill_noalloc(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens),
+                                                  int(cu_seqlens.numel()) - 1, int(q.shape[0]),
+                                                  int(max_seqlen), ctypes.byref(m), _ptr(out), _ptr(lse),
+                                                  _ptr(device_status), _stream(stream)),
+           "fp2_sparse_prefill_noalloc")
 
 
 def get_error(ws: Workspace, stream=None) -> int:

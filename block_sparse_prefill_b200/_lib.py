@@ -18,7 +18,9 @@ STATUS = {
 # every function the header declares
 EXPORTS = ["fp2_max_blocks", "fp2_workspace_bytes", "fp2_workspace_init", "fp2_estimate",
            "fp2_sparse_prefill", "fp2_prefill_paged", "fp2_get_error", "fp2_status_string",
-           "fp2_version"]
+           "fp2_version", "fp2_sparse_prefill_noalloc"]
+
+NOALLOC_SCRATCH_BYTES = 8 << 20  # FP2_NOALLOC_SCRATCH_BYTES
 
 
 class fp2_params(ctypes.Structure):
@@ -85,6 +87,8 @@ def load():
     lib.fp2_get_error.restype = ctypes.c_int
     lib.fp2_status_string.argtypes = [ctypes.c_int]
     lib.fp2_status_string.restype = ctypes.c_char_p
+    lib.fp2_sparse_prefill_noalloc.argtypes = [_PP, _P, _P, _P, _P, _I32, _I64, _I32, _PM, _P, _P, _P, _P]
+    lib.fp2_sparse_prefill_noalloc.restype = ctypes.c_int
     lib.fp2_version.argtypes = []
     lib.fp2_version.restype = _I32
     _lib = lib

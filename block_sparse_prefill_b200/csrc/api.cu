@@ -405,3 +405,95 @@ const char* fp2_status_string(fp2_status status) {
 int32_t fp2_version(void) { return 100; }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// fp2_sparse_prefill_noalloc: the same attention call with its scratch in a
+// file-scope device array instead of a caller workspace.
+// ---------------------------------------------------------------------------
+namespace {
+
+static __device__ __align__(256) uint8_t g_noalloc_scratch[FP2_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[kMaxDevices] = {};  // device address of the array, per device ordinal
+
+// Device address of the scratch array on the current device.  Host code must
+// not hand `g_noalloc_scratch` itself to a kernel: on the host that name is a
+// stand-in, not a device address.
+fp2_status noalloc_scratch(void** addr) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FP2_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_addr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return FP2_ERR_CUDA;
+        g_noalloc_addr[dev] = p;
+    }
+    *addr = g_noalloc_addr[dev];
+    return FP2_OK;
+}
+
+// The attention call reads no q-block means, so its scratch is the workspace
+// layout without that region.
+WsLayout noalloc_layout(const Problem& pr, const fp2_params* p) {
+    WsLayout w;
+    size_t off = 256;
+    w.cu_blocks = off;
+    off = align256(off + sizeof(int32_t) * (pr.batch + 1));
+    w.cu_tiles = off;
+    off = align256(off + sizeof(int32_t) * (pr.batch + 1));
+    w.blk_req = off;
+    off = align256(off + sizeof(int32_t) * pr.max_blocks);
+    w.qbar = off;
+    w.kbar_lp = off;
+    off = align256(off + size_t(esize(p)) * pr.max_blocks * p->num_kv_heads * kHeadDim);
+    w.vbar_lp = off;
+    off = align256(off + size_t(esize(p)) * pr.max_blocks * p->num_kv_heads * kHeadDim);
+    w.total = off;
+    return w;
+}
+
+}  // namespace
+
+extern "C" fp2_status fp2_sparse_prefill_noalloc(const fp2_params* params, const void* q,
+                                                 const void* k, const void* v,
+                                                 const int32_t* cu_seqlens, int32_t batch,
+                                                 int64_t total_tokens, int32_t max_seqlen,
+                                                 const fp2_blockmeta* meta, void* out, float* lse,
+                                                 int32_t* device_status, void* stream) {
+    fp2_status st = check_params(params);
+    if (st != FP2_OK) return st;
+    if (batch < 0 || total_tokens < 0 || max_seqlen < 0) return FP2_ERR_INVALID_ARG;
+    if (total_tokens > (int64_t(1) << 31) - 1) return FP2_ERR_UNSUPPORTED;
+    if (batch > 0 && !cu_seqlens) return FP2_ERR_INVALID_ARG;
+    if (total_tokens > 0 && (!q || !k || !v)) return FP2_ERR_INVALID_ARG;
+    if ((q && !aligned(q, 16)) || (k && !aligned(k, 16)) || (v && !aligned(v, 16)))
+        return FP2_ERR_INVALID_ARG;
+    if (total_tokens > 0 && (!out || !aligned(out, 16))) return FP2_ERR_INVALID_ARG;
+    if (lse && !aligned(lse, 4)) return FP2_ERR_INVALID_ARG;
+    if (device_status && !aligned(device_status, 4)) return FP2_ERR_INVALID_ARG;
+    Problem pr;
+    pr.batch = batch;
+    pr.total_tokens = total_tokens;
+    pr.max_seqlen = max_seqlen;
+    pr.max_blocks = fp2_max_blocks(batch, total_tokens, kBlock);
+    pr.nb_need = (max_seqlen + kBlock - 1) / kBlock;
+    pr.ws = noalloc_layout(pr, params);
+    if (pr.ws.total > FP2_NOALLOC_SCRATCH_BYTES) return FP2_ERR_WORKSPACE;  // over the static maximum
+    if ((st = check_meta(meta, params, pr, true)) != FP2_OK) return st;
+    void* scratch = nullptr;
+    if ((st = noalloc_scratch(&scratch)) != FP2_OK) return st;
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // the error flag is the only scratch state that must start at zero; every
+    // other region is rewritten by the kernels of this call
+    if (cudaMemsetAsync(scratch, 0, sizeof(WsHeader), s) != cudaSuccess) return FP2_ERR_CUDA;
+    st = run_attention(params, q, k, v, cu_seqlens, pr, nullptr, 0, 0, meta, out, lse, scratch, s,
+                       true);
+    if (st != FP2_OK) return st;
+    if (device_status &&
+        cudaMemcpyAsync(device_status, scratch, sizeof(int32_t), cudaMemcpyDeviceToDevice, s) !=
+            cudaSuccess)
+        return FP2_ERR_CUDA;
+    return FP2_OK;
+}

@@ -163,6 +163,39 @@ fp2_status fp2_get_error(void* workspace, void* stream);
 /* Static description of a status code. */
 const char* fp2_status_string(fp2_status status);
 
+/* Size of the device scratch array behind fp2_sparse_prefill_noalloc (8 MiB). */
+#define FP2_NOALLOC_SCRATCH_BYTES (8u << 20)
+
+/* Allocation-free form of fp2_sparse_prefill.  The FlashPrefill V2 write-ups
+ * have no counterpart of this call; it exists for callers that cannot allocate
+ * device memory at the point where they run attention: a plugin or operator
+ * inside a host framework that owns every device allocation (and forbids
+ * allocating behind its back), code whose memory budget is fixed up front, or
+ * latency-critical code that must avoid cudaMalloc's implicit device
+ * synchronisation.  Such callers pass no workspace.  Instead the library uses
+ * one file-scope device array of FP2_NOALLOC_SCRATCH_BYTES, which every GPU
+ * that loads the library holds until the process exits.
+ *   - Arguments, layouts and results are those of fp2_sparse_prefill.
+ *   - Returns FP2_ERR_WORKSPACE, without enqueuing anything, when the problem
+ *     needs more scratch than FP2_NOALLOC_SCRATCH_BYTES (about 4.2 MB for a
+ *     131072-token request with 8 KV heads).
+ *   - device_status: optional caller-owned DEVICE int32; when non-NULL it
+ *     receives (asynchronously, on `stream`) the device-side fp2_status of
+ *     this call (0 = none), since there is no workspace to query with
+ *     fp2_get_error.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress), so make that first call before any CUDA stream
+ *     capture on that device.
+ *   - All calls share the one array, and the array keeps the last call's
+ *     contents: calls that overlap on the GPU (different streams, or
+ *     different host threads, without ordering) race on it.
+ *   - It calls no cudaMalloc/cudaFree or allocating library routine. */
+fp2_status fp2_sparse_prefill_noalloc(const fp2_params* params, const void* q, const void* k,
+                                      const void* v, const int32_t* cu_seqlens, int32_t batch,
+                                      int64_t total_tokens, int32_t max_seqlen,
+                                      const fp2_blockmeta* meta, void* out, float* lse,
+                                      int32_t* device_status, void* stream);
+
 /* Library version (major * 10000 + minor * 100 + patch). */
 int32_t fp2_version(void);
 
