@@ -13,16 +13,25 @@
 //
 // Structure (one CTA = one q-block x two query heads of one KV head, so every
 // K/V tile fetched into shared memory serves both heads):
-//   warps 0-3  softmax of Q tile 0 (one thread per row, rows = TMEM lanes)
-//   warps 4-7  softmax of Q tile 1
-//   warp  8    TMA producer: Q tiles, then K/V (or mean-K/mean-V) tiles into a
-//              ring of shared-memory slots, following the kept list and, in
-//              paged mode, the block table
-//   warp  9    TMEM owner and MMA issuer: S_t = Q_t K^T (both operands in shared
-//              memory), O_t += P_t V (P_t from TMEM, V from shared memory)
+//   warpgroup 0 (warps 0-3)  softmax of Q tile 0 (one thread per row = TMEM lane)
+//   warpgroup 1 (warps 4-7)  softmax of Q tile 1
+//   warpgroup 2: warp 8      TMA producer: Q tiles, then K/V (or mean-K/mean-V)
+//                            tiles into a ring of shared-memory slots, following
+//                            the kept list and, in paged mode, the block table
+//                warp 9      TMEM owner and MMA issuer
+//                warps 10-11 idle (they only donate registers)
+// The softmax warpgroups raise their register budget (setmaxnreg) so that a
+// whole 128-column row of S stays in registers; warpgroup 2 lowers its own.
+//
 // TMEM columns: S_0 [0,128) S_1 [128,256) O_0 [256,384) O_1 [384,512); P_t is
-// written over the first columns of S_t.  The running max is only raised when
-// it grows by more than a threshold (log2 units), so O is rarely rescaled.
+// written over the first columns of S_t and read by the PV MMA from TMEM.
+// MMA issue order per kept tile n (tcgen05.mma from one thread run in issue
+// order, so S_t(n+1) may be issued right after PV_t(n), which still reads P_t
+// from the same columns):
+//   PV_0(n), S_0(n+1), PV_1(n), S_1(n+1)
+// so the softmax of one tile overlaps the other tile's two MMAs.
+// The running max is only raised when a row max exceeds it by more than a
+// threshold (log2 units), so O is rarely rescaled.
 // Tile order: diagonal block first (it fixes the causal mask and usually the
 // row max), then the other kept blocks from nearest to farthest, then the
 // correction tiles: 128 consecutive block means each, with the kept ones (and
@@ -36,10 +45,18 @@ namespace fp2 {
 
 namespace {
 
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr uint32_t kTmemCols = 512;
+// Registers per thread after the split.  setmaxnreg only redistributes the
+// registers the CTA was launched with (384 threads x 168 = 64512), so
+// 256 x kSoftmaxRegs + 128 x kOtherRegs must not exceed that: 53248 + 11264.
+constexpr int kLaunchRegs = 168;
+constexpr int kSoftmaxRegs = 208;
+constexpr int kOtherRegs = 88;
+static_assert(256 * kSoftmaxRegs + 128 * kOtherRegs <= kThreads * kLaunchRegs,
+              "register split exceeds the launch allocation");
 
 template <bool kE4M3>
 struct Cfg {
@@ -106,6 +123,45 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, WsHead
                                           volatile int32_t* abort, int32_t where) {
     const bool ok = mbar_wait(bar, parity, hdr, abort, where);
     return __all_sync(0xffffffffu, ok);
+}
+
+template <int kRegs>
+__device__ __forceinline__ void regs_inc() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(kRegs));
+}
+template <int kRegs>
+__device__ __forceinline__ void regs_dec() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(kRegs));
+}
+
+// S = Q_t K^T for one Q tile (kKSteps MMAs over d).
+template <bool kE4M3>
+__device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_addr, uint32_t k_addr) {
+    using C = Cfg<kE4M3>;
+#pragma unroll
+    for (int k = 0; k < C::kKSteps; ++k) {
+        if (kE4M3)
+            mma_f8_ss(d_tmem, kmajor_desc<true>(q_addr, k), kmajor_desc<true>(k_addr, k), C::kIdescQK,
+                      k > 0);
+        else
+            mma_bf16_ss(d_tmem, kmajor_desc<false>(q_addr, k), kmajor_desc<false>(k_addr, k),
+                        C::kIdescQK, k > 0);
+    }
+}
+
+// O += P V for one Q tile (P from TMEM, kKSteps MMAs over the 128 keys).
+template <bool kE4M3>
+__device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint32_t v_addr,
+                                         bool first) {
+    using C = Cfg<kE4M3>;
+#pragma unroll
+    for (int k = 0; k < C::kKSteps; ++k) {
+        const uint32_t acc = (!first || k > 0) ? 1u : 0u;
+        if (kE4M3)
+            mma_f8_ts(o_tmem, p_tmem + 8 * k, vmajor_desc<true>(v_addr, k), C::kIdescPV, acc);
+        else
+            mma_bf16_ts(o_tmem, p_tmem + 8 * k, vmajor_desc<false>(v_addr, k), C::kIdescPV, acc);
+    }
 }
 
 }  // namespace
@@ -224,7 +280,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int32_t ntot = cnt + ncorr;
 
     // ---- roles -------------------------------------------------------------
-    if (warp == kProducerWarp) {
+    if (warp >= 8) {
+      regs_dec<kOtherRegs>();
+      if (warp == kProducerWarp) {
         // lane 0 issues every TMA; the whole warp zeroes the V rows past the
         // request end of a partial diagonal block (a paged pool may hold
         // anything there, and zero attention weights times NaN is NaN)
@@ -304,68 +362,55 @@ __global__ void __launch_bounds__(kThreads, 1)
                     break;
             }
         }
-    } else if (warp == kMmaWarp) {
+      } else if (warp == kMmaWarp) {
         if (lane == 0) {
             const uint32_t q_addr = smem_u32(q_s);
             const uint32_t kv_addr = smem_u32(kv_s);
-            bool ok = mbar_wait(&bars.q_full, 0, hdr, abort, 300000);
-            tc_fence_after();
-            for (int32_t n = 0; ok && n < ntot; ++n) {
-                const int32_t ik = 2 * n, iv = 2 * n + 1;
-                const int32_t sk = ik % C::kSlots, sv = iv % C::kSlots;
-                if (!(ok = mbar_wait(&bars.kv_full[sk], (ik / C::kSlots) & 1, hdr, abort, 310000 + n)))
-                    break;
+            // tile n: K in ring entry 2n, V in ring entry 2n + 1
+            auto slot = [](int32_t idx) { return idx % C::kSlots; };
+            auto phase = [](int32_t idx) { return static_cast<uint32_t>((idx / C::kSlots) & 1); };
+            bool ok = mbar_wait(&bars.q_full, 0, hdr, abort, 300000) &&
+                      mbar_wait(&bars.kv_full[slot(0)], phase(0), hdr, abort, 301000);
+            if (ok) {
                 tc_fence_after();
-                for (int qt = 0; qt < ntiles && ok; ++qt) {
-                    if (n > 0) {
-                        if (!(ok = mbar_wait(&bars.o_done[qt], (n - 1) & 1, hdr, abort, 320000 + n)))
-                            break;
-                        tc_fence_after();
-                    }
-                    const uint32_t d_s = tmem + qt * 128;
-                    const uint32_t qb = q_addr + qt * C::kTileBytes;
-                    const uint32_t kb = kv_addr + sk * C::kTileBytes;
-#pragma unroll
-                    for (int k = 0; k < C::kKSteps; ++k) {
-                        if (kE4M3)
-                            mma_f8_ss(d_s, kmajor_desc<kE4M3>(qb, k), kmajor_desc<kE4M3>(kb, k),
-                                      C::kIdescQK, k > 0);
-                        else
-                            mma_bf16_ss(d_s, kmajor_desc<kE4M3>(qb, k), kmajor_desc<kE4M3>(kb, k),
-                                        C::kIdescQK, k > 0);
-                    }
+                for (int qt = 0; qt < ntiles; ++qt) {
+                    issue_qk<kE4M3>(tmem + qt * 128, q_addr + qt * C::kTileBytes,
+                                    kv_addr + slot(0) * C::kTileBytes);
                     mma_commit(&bars.s_full[qt]);
                 }
-                if (!ok) break;
-                mma_commit(&bars.kv_empty[sk]);
-                if (!(ok = mbar_wait(&bars.kv_full[sv], (iv / C::kSlots) & 1, hdr, abort, 330000 + n)))
+                mma_commit(&bars.kv_empty[slot(0)]);
+            }
+            for (int32_t n = 0; ok && n < ntot; ++n) {
+                const int32_t iv = 2 * n + 1, ik = 2 * n + 2;
+                const bool next = n + 1 < ntot;
+                if (!(ok = mbar_wait(&bars.kv_full[slot(iv)], phase(iv), hdr, abort, 330000 + n)))
                     break;
                 if (n == 0 && nrows < kBlock &&
                     !(ok = mbar_wait(&bars.v_tail, 0, hdr, abort, 335000)))
                     break;
-                tc_fence_after();
                 for (int qt = 0; qt < ntiles && ok; ++qt) {
                     if (!(ok = mbar_wait(&bars.p_full[qt], n & 1, hdr, abort, 340000 + n))) break;
                     tc_fence_after();
-                    const uint32_t d_o = tmem + 256 + qt * 128;
-                    const uint32_t p_t = tmem + qt * 128;
-                    const uint32_t vb = kv_addr + sv * C::kTileBytes;
-#pragma unroll
-                    for (int k = 0; k < C::kKSteps; ++k) {
-                        if (kE4M3)
-                            mma_f8_ts(d_o, p_t + 8 * k, vmajor_desc<kE4M3>(vb, k), C::kIdescPV,
-                                      (n > 0 || k > 0) ? 1u : 0u);
-                        else
-                            mma_bf16_ts(d_o, p_t + 8 * k, vmajor_desc<kE4M3>(vb, k), C::kIdescPV,
-                                        (n > 0 || k > 0) ? 1u : 0u);
-                    }
+                    issue_pv<kE4M3>(tmem + 256 + qt * 128, tmem + qt * 128,
+                                    kv_addr + slot(iv) * C::kTileBytes, n == 0);
                     mma_commit(&bars.o_done[qt]);
+                    if (next) {
+                        if (qt == 0 && !(ok = mbar_wait(&bars.kv_full[slot(ik)], phase(ik), hdr,
+                                                        abort, 310000 + n)))
+                            break;
+                        tc_fence_after();
+                        issue_qk<kE4M3>(tmem + qt * 128, q_addr + qt * C::kTileBytes,
+                                        kv_addr + slot(ik) * C::kTileBytes);
+                        mma_commit(&bars.s_full[qt]);
+                    }
                 }
                 if (!ok) break;
-                mma_commit(&bars.kv_empty[sv]);
+                if (next) mma_commit(&bars.kv_empty[slot(ik)]);
+                mma_commit(&bars.kv_empty[slot(iv)]);
             }
         }
-    } else if (warp / 4 < ntiles) {
+      }
+    } else if (regs_inc<kSoftmaxRegs>(), warp / 4 < ntiles) {
         // ---- softmax + epilogue of Q tile qt ---------------------------------
         const int qt = warp / 4;
         const int32_t r = tid & 127;
@@ -375,6 +420,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t o_addr = tmem + lane_off + 256 + qt * 128;
         float qk = a.scale_log2;
         if (kE4M3) qk *= a.q_scale[h] * a.k_scale[g];
+        // correction tiles: +log2(128) after scaling == +7/qk before it
+        const float corr_bias = 7.f / qk;
         float m_ref = -INFINITY;
         float l = 0.f;      // row sum of the weights the PV MMA uses (O normaliser)
         float l_lse = 0.f;  // row sum before P is rounded to the MMA precision (LSE)
@@ -382,36 +429,37 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int32_t n = 0; n < ntot; ++n) {
             if (!(ok = warp_wait(&bars.s_full[qt], n & 1, hdr, abort, 400000 + n))) break;
             tc_fence_after();
-            // logits of this tile in log2 units, masked entries -inf:
+            uint32_t sv[128];
+            tmem_ld32(s_addr + 0, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+            tmem_ld32(s_addr + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+            tmem_ld32(s_addr + 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[64]));
+            tmem_ld32(s_addr + 96, *reinterpret_cast<uint32_t(*)[32]>(&sv[96]));
+            tmem_wait_ld();
+            // masks (warp-uniform branch per tile kind):
             //   diagonal block (n == 0): keys c <= r
             //   kept block: every key
-            //   correction tile: pruned block means only, plus log2(128) for the 128 rows each stands for
-            const int kind = (n == 0) ? 0 : (n < cnt ? 1 : 2);
-            const int32_t w0 = (kind == 2) ? ctiles[n - cnt] * 4 : 0;
-            auto logit = [&](uint32_t raw, int c, uint32_t bits) -> float {
-                const float sx = __uint_as_float(raw);
-                if (kind == 0) return (c <= r) ? sx * qk : -INFINITY;
-                if (kind == 1) return sx * qk;
-                return ((bits >> (c & 31)) & 1u) ? fmaf(sx, qk, 7.f) : -INFINITY;
-            };
-            // pass 1: row max
-            float mx = -INFINITY;
+            //   correction tile: pruned block means only, weighted by 128
+            if (n == 0) {
 #pragma unroll
-            for (int c0 = 0; c0 < 128; c0 += 64) {
-                uint32_t sv[64];
-                tmem_ld32(s_addr + c0, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-                tmem_ld32(s_addr + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
-                tmem_wait_ld();
+                for (int c = 0; c < 128; ++c)
+                    if (c > r) sv[c] = __float_as_uint(-INFINITY);
+            } else if (n >= cnt) {
+                const int32_t w0 = ctiles[n - cnt] * 4;
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    const int cw = (c0 >> 5) + half;
-                    const uint32_t bits = (kind == 2 && w0 + cw < nwords) ? pruned[w0 + cw] : 0u;
+                for (int wi = 0; wi < 4; ++wi) {
+                    const uint32_t bits = (w0 + wi < nwords) ? pruned[w0 + wi] : 0u;
 #pragma unroll
                     for (int c = 0; c < 32; ++c)
-                        mx = fmaxf(mx, logit(sv[half * 32 + c], c0 + half * 32 + c, bits));
+                        sv[wi * 32 + c] =
+                            ((bits >> c) & 1u)
+                                ? __float_as_uint(__uint_as_float(sv[wi * 32 + c]) + corr_bias)
+                                : __float_as_uint(-INFINITY);
                 }
             }
-            const float m_new = fmaxf(m_ref, mx);
+            float mx = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < 128; ++c) mx = fmaxf(mx, __uint_as_float(sv[c]));
+            const float m_new = fmaxf(m_ref, mx * qk);
             const bool need = m_new > m_ref + C::kRescale;
             if (__any_sync(0xffffffffu, need)) {
                 const float f = need ? ex2(m_ref - m_new) : 1.f;
@@ -435,50 +483,38 @@ __global__ void __launch_bounds__(kThreads, 1)
                     m_ref = m_new;
                 }
             }
-            const float m_use = ((m_ref == -INFINITY) ? 0.f : m_ref) - C::kPOffset;
-            // pass 2: P = exp2(x - m) in the MMA precision, written over the
-            // already-consumed leading columns of S
-            float rs = 0.f, rs_q = 0.f;
+            // P = exp2(s * qk - m + offset) in the MMA precision, written over S
+            const float neg = C::kPOffset - ((m_ref == -INFINITY) ? 0.f : m_ref);
+            float rs = 0.f;
 #pragma unroll
-            for (int c0 = 0; c0 < 128; c0 += 64) {
-                uint32_t sv[64];
-                tmem_ld32(s_addr + c0, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-                tmem_ld32(s_addr + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
-                tmem_wait_ld();
-                float p[64];
-#pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    const int cw = (c0 >> 5) + half;
-                    const uint32_t bits = (kind == 2 && w0 + cw < nwords) ? pruned[w0 + cw] : 0u;
-#pragma unroll
-                    for (int c = 0; c < 32; ++c) {
-                        const int cc = half * 32 + c;
-                        p[cc] = ex2(logit(sv[cc], c0 + cc, bits) - m_use);
-                        rs += p[cc];
-                    }
-                }
-                if (kE4M3) {
-                    // the row sum takes the quantised weights the PV MMA sees, so
-                    // numerator and denominator use the same P
-                    uint32_t pk[16];
-                    __half2 hs = __float2half2_rn(0.f);
-#pragma unroll
-                    for (int c = 0; c < 16; ++c) {
-                        pk[c] = pack_e4m3x4(p[4 * c], p[4 * c + 1], p[4 * c + 2], p[4 * c + 3]);
-                        hs = __hadd2(hs, e4m3x4_sum2(pk[c]));
-                    }
-                    const float2 hf = __half22float2(hs);
-                    rs_q += hf.x + hf.y;
-                    tmem_st16(s_addr + c0 / 4, pk);
-                } else {
-                    uint32_t pk[32];
-#pragma unroll
-                    for (int c = 0; c < 32; ++c) pk[c] = pack_bf16(p[2 * c], p[2 * c + 1]);
-                    tmem_st32(s_addr + c0 / 2, pk);
-                }
+            for (int c = 0; c < 128; ++c) {
+                const float p = ex2(fmaf(__uint_as_float(sv[c]), qk, neg));
+                sv[c] = __float_as_uint(p);
+                rs += p;
             }
-            l += kE4M3 ? rs_q : rs;
             l_lse += rs;
+            if (kE4M3) {
+                // the O normaliser sums the quantised weights the PV MMA sees
+                __half2 hs = __float2half2_rn(0.f);
+#pragma unroll
+                for (int c = 0; c < 32; ++c) {
+                    const uint32_t pk =
+                        pack_e4m3x4(__uint_as_float(sv[4 * c]), __uint_as_float(sv[4 * c + 1]),
+                                    __uint_as_float(sv[4 * c + 2]), __uint_as_float(sv[4 * c + 3]));
+                    hs = __hadd2(hs, e4m3x4_sum2(pk));
+                    sv[c] = pk;
+                }
+                const float2 hf = __half22float2(hs);
+                l += hf.x + hf.y;
+                tmem_st32(s_addr, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+            } else {
+                l += rs;
+#pragma unroll
+                for (int c = 0; c < 64; ++c)
+                    sv[c] = pack_bf16(__uint_as_float(sv[2 * c]), __uint_as_float(sv[2 * c + 1]));
+                tmem_st32(s_addr, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+                tmem_st32(s_addr + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+            }
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&bars.p_full[qt]);
@@ -535,7 +571,13 @@ cudaError_t launch_attention(bool e4m3, const AttnArgs& a, const CUtensorMap& tq
     const size_t smem = attn_smem_bytes(e4m3, a.nb_cap);
     const int64_t grid = max_blocks * a.hkv * a.pairs;
     if (grid <= 0) return cudaSuccess;
-    cudaError_t err;
+    // the setmaxnreg split assumes the kernel was built with kLaunchRegs per
+    // thread; with fewer, the softmax warps' register request could never be met
+    cudaFuncAttributes fa;
+    cudaError_t err = e4m3 ? cudaFuncGetAttributes(&fa, attention_kernel<true>)
+                           : cudaFuncGetAttributes(&fa, attention_kernel<false>);
+    if (err != cudaSuccess) return err;
+    if (fa.numRegs < kLaunchRegs) return cudaErrorInvalidConfiguration;
     if (e4m3) {
         err = cudaFuncSetAttribute(attention_kernel<true>,
                                    cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
