@@ -153,11 +153,19 @@ fp2_status run_setup(const Problem& pr, void* ws, const int32_t* cu, int32_t qt,
     sa.paged = paged ? 1 : 0;
     sa.max_blocks_per_seq = mbps;
     sa.max_blocks = meta_blocks < pr.max_blocks ? meta_blocks : pr.max_blocks;
+    sa.nb_cap = pr.nb_need > 0 ? pr.nb_need : 1;
     sa.hdr = at<WsHeader>(ws, 0);
     sa.cu_blocks = at<int32_t>(ws, pr.ws.cu_blocks);
     sa.cu_tiles = at<int32_t>(ws, pr.ws.cu_tiles);
     sa.blk_req = at<int32_t>(ws, pr.ws.blk_req);
-    setup_kernel<<<1, 256, 0, s>>>(sa);
+    sa.order = at<int32_t>(ws, pr.ws.order);
+    const size_t hist_bytes = sizeof(int32_t) * (sa.nb_cap + 1);
+    if (hist_bytes > kMaxSmem) return FP2_ERR_UNSUPPORTED;
+    if (hist_bytes > 48 * 1024 &&
+        cudaFuncSetAttribute(setup_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(hist_bytes)) != cudaSuccess)
+        return FP2_ERR_CUDA;
+    setup_kernel<<<1, 256, hist_bytes, s>>>(sa);
     return launched(cudaGetLastError());
 }
 
@@ -279,6 +287,7 @@ fp2_status run_attention(const fp2_params* p, const void* q, const void* k, cons
     a.cu = cu;
     a.cu_blocks = at<int32_t>(ws, pr.ws.cu_blocks);
     a.blk_req = at<int32_t>(ws, pr.ws.blk_req);
+    a.order = at<int32_t>(ws, pr.ws.order);
     a.block_table = block_table;
     a.max_blocks_per_seq = mbps;
     a.num_pages = num_pages;
@@ -444,6 +453,8 @@ WsLayout noalloc_layout(const Problem& pr, const fp2_params* p) {
     w.cu_tiles = off;
     off = align256(off + sizeof(int32_t) * (pr.batch + 1));
     w.blk_req = off;
+    off = align256(off + sizeof(int32_t) * pr.max_blocks);
+    w.order = off;
     off = align256(off + sizeof(int32_t) * pr.max_blocks);
     w.qbar = off;
     w.kbar_lp = off;

@@ -48,6 +48,15 @@ namespace {
 constexpr int kThreads = 384;
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
+constexpr int kSchedWarp = 10;
+// When > 0, every kEmuEvery-th pair of attention weights is exponentiated on
+// the FMA pipe (exp2_poly2) instead of MUFU.  Measured on B200 at 128K (bf16,
+// attention call): off 4.77 ms, 1/8 4.77 ms, 1/4 5.08 ms, 1/2 5.90 ms -- the
+// softmax is bound by instruction issue, not by MUFU, so it is off.
+#ifndef FP2_EXP_EMU_EVERY
+#define FP2_EXP_EMU_EVERY 0
+#endif
+constexpr int kEmuEvery = FP2_EXP_EMU_EVERY;
 constexpr uint32_t kTmemCols = 512;
 // Registers per thread after the split.  setmaxnreg only redistributes the
 // registers the CTA was launched with (384 threads x 168 = 64512), so
@@ -79,20 +88,30 @@ struct Cfg {
 
 struct Bars {
     uint64_t q_full;
+    uint64_t q_empty;     // the last S MMA of a work item has read Q
     uint64_t s_full[2];
     uint64_t p_full[2];
     uint64_t o_done[2];
     uint64_t kv_full[8];
     uint64_t kv_empty[8];
     uint64_t v_tail;      // V rows past the request end zeroed (partial diagonal block)
+    uint64_t meta_full[2];
+    uint64_t meta_empty[2];
 };
 
 struct SmemMisc {
     Bars bars;
     uint32_t tmem_base;
     int32_t abort;
-    int32_t cnt;      // kept blocks
-    int32_t ncorr;    // correction tiles
+};
+
+// One work item (a q-block x up to two query heads of one KV head), prepared
+// by the scheduler warp into one of two shared-memory buffers.  The kept list,
+// the pruned-block bitmask and the correction tile list follow the header.
+struct ItemMeta {
+    int32_t stop;     // 1: no work left
+    int32_t t, b, i, g, h0, ntiles, nrows, qrow0, cb, cnt, ncorr, nwords;
+    int32_t pad[3];
 };
 
 template <bool kE4M3>
@@ -100,9 +119,11 @@ __host__ __device__ constexpr size_t tiles_bytes() {
     return static_cast<size_t>(2 + Cfg<kE4M3>::kSlots) * Cfg<kE4M3>::kTileBytes;
 }
 
-__host__ __device__ inline size_t lists_bytes(int32_t nb_max) {
-    // kept list + pruned bitmask + correction tile list
-    return sizeof(int32_t) * (nb_max + (nb_max + 31) / 32 + (nb_max + 127) / 128 + 4);
+// One metadata buffer: header, kept list, pruned bitmask, correction tile list.
+__host__ __device__ inline size_t meta_bytes(int32_t nb_cap) {
+    const size_t b = sizeof(ItemMeta) +
+                     sizeof(int32_t) * (nb_cap + (nb_cap + 31) / 32 + (nb_cap + 127) / 128 + 4);
+    return (b + 15) & ~size_t(15);
 }
 
 // Descriptor of K-major operand step k (Q or K tile at `base`).
@@ -179,35 +200,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t* q_s = smem;                                  // 2 tiles
     uint8_t* kv_s = smem + 2 * C::kTileBytes;             // kSlots tiles
     SmemMisc* misc = reinterpret_cast<SmemMisc*>(smem + tiles_bytes<kE4M3>());
-    int32_t* klist = reinterpret_cast<int32_t*>(misc + 1);
-    uint32_t* pruned = reinterpret_cast<uint32_t*>(klist + a.nb_cap);
-    int32_t* ctiles = reinterpret_cast<int32_t*>(pruned + (a.nb_cap + 31) / 32);
+    uint8_t* meta_base = reinterpret_cast<uint8_t*>(misc + 1);
+    const size_t meta_stride = meta_bytes(a.nb_cap);
     Bars& bars = misc->bars;
     volatile int32_t* abort = &misc->abort;
-
-    // ---- work item ---------------------------------------------------------
     WsHeader* hdr = a.hdr;
     if (!hdr->valid) return;
-    const int32_t total_blocks = hdr->total_blocks;
-    const int32_t per_blk = a.hkv * a.pairs;
-    const int32_t t_rev = blockIdx.x / per_blk;
-    if (t_rev >= total_blocks) return;
-    const int32_t t = total_blocks - 1 - t_rev;  // late q-blocks (long kept lists) first
-    const int32_t rem = blockIdx.x % per_blk;
-    const int32_t g = rem / a.pairs;
-    const int32_t hp = rem % a.pairs;
-    const int32_t h0 = g * a.G + 2 * hp;
-    const int32_t ntiles = min(2, a.G - 2 * hp);
-    const int32_t b = a.blk_req[t];
-    const int32_t cb = a.cu_blocks[b];
-    const int32_t i = t - cb;
-    const int32_t L = a.cu[b + 1] - a.cu[b];
-    const int32_t nrows = min(kBlock, L - i * kBlock);
-    const int32_t qrow0 = a.cu[b] + i * kBlock;
 
     const int32_t tid = threadIdx.x;
     const int32_t warp = tid >> 5;
     const int32_t lane = tid & 31;
+    const int32_t per_blk = a.hkv * a.pairs;
+    const int32_t n_items = hdr->total_blocks * per_blk;
+
+    auto meta = [&](int32_t buf) { return reinterpret_cast<ItemMeta*>(meta_base + buf * meta_stride); };
+    auto klist_of = [](ItemMeta* m) { return reinterpret_cast<int32_t*>(m + 1); };
+    auto pruned_of = [&](ItemMeta* m) { return reinterpret_cast<uint32_t*>(klist_of(m) + a.nb_cap); };
+    auto ctiles_of = [&](ItemMeta* m) {
+        return reinterpret_cast<int32_t*>(pruned_of(m) + (a.nb_cap + 31) / 32);
+    };
 
     // ---- set-up ------------------------------------------------------------
     if (warp == kMmaWarp) {
@@ -216,10 +227,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (tid == 0) {
         mbar_init(&bars.q_full, 1);
+        mbar_init(&bars.q_empty, 1);
         for (int s = 0; s < 2; ++s) {
             mbar_init(&bars.s_full[s], 1);
             mbar_init(&bars.p_full[s], 128);
             mbar_init(&bars.o_done[s], 1);
+            mbar_init(&bars.meta_full[s], 1);
+            mbar_init(&bars.meta_empty[s], 10);  // producer, MMA issuer, 8 softmax warps
         }
         for (int s = 0; s < C::kSlots; ++s) {
             mbar_init(&bars.kv_full[s], 1);
@@ -229,60 +243,104 @@ __global__ void __launch_bounds__(kThreads, 1)
         misc->abort = 0;
         fence_mbar_init();
     }
-    // kept list of (q-block t, KV head g)
-    const int64_t lrow = static_cast<int64_t>(t) * a.hkv + g;
-    int32_t cnt = a.kept_cnt[lrow];
-    const bool cnt_ok = cnt >= 1 && cnt <= i + 1;
-    if (!cnt_ok) cnt = 1;
-    const int32_t* src = a.kept_idx + lrow * a.nb_max;
-    for (int32_t e = tid; e < cnt; e += kThreads) klist[e] = cnt_ok ? src[e] : i;
-    const int32_t nwords = (i + 31) / 32;  // bits for key blocks j < i
-    for (int32_t w = tid; w < nwords; w += kThreads) {
-        const int32_t lo = w * 32;
-        const int32_t nbits = min(32, i - lo);
-        pruned[w] = (nbits == 32) ? 0xffffffffu : ((1u << nbits) - 1u);
-    }
-    __syncthreads();
-    if (tid == 0) {
-        bool ok = cnt_ok && klist[cnt - 1] == i;
-        for (int32_t e = 1; ok && e < cnt; ++e) ok = klist[e] > klist[e - 1] && klist[e - 1] >= 0;
-        if (!ok) {
-            set_error(hdr, FP2_ERR_BAD_INDEX, t);
-            klist[0] = i;
-            cnt = 1;
-        }
-        misc->cnt = cnt;
-    }
-    __syncthreads();
-    cnt = misc->cnt;
-    if (a.correction) {
-        for (int32_t e = tid; e < cnt - 1; e += kThreads) {
-            const int32_t j = klist[e];
-            atomicAnd(&pruned[j >> 5], ~(1u << (j & 31)));
-        }
-    }
-    __syncthreads();
-    if (tid == 0) {
-        int32_t nc = 0;
-        if (a.correction) {
-            for (int32_t ct = 0; ct * 128 < i; ++ct) {
-                uint32_t any = 0;
-                for (int32_t w = ct * 4; w < min(ct * 4 + 4, nwords); ++w) any |= pruned[w];
-                if (any) ctiles[nc++] = ct;
-            }
-        }
-        misc->ncorr = nc;
-    }
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = misc->tmem_base;
-    const int32_t ncorr = misc->ncorr;
-    const int32_t ntot = cnt + ncorr;
 
-    // ---- roles -------------------------------------------------------------
     if (warp >= 8) {
       regs_dec<kOtherRegs>();
-      if (warp == kProducerWarp) {
+      if (warp == kSchedWarp) {
+        // ---- scheduler: next work item -> metadata buffer ----------------
+        for (int32_t k = 0;; ++k) {
+            const int32_t buf = k & 1;
+            if (!warp_wait(&bars.meta_empty[buf], ((k >> 1) & 1) ^ 1, hdr, abort, 500000 + k)) break;
+            ItemMeta* m = meta(buf);
+            int32_t item = 0;
+            if (lane == 0) item = atomicAdd(&hdr->work_next, 1);
+            item = __shfl_sync(0xffffffffu, item, 0);
+            if (item >= n_items) {
+                if (lane == 0) {
+                    m->stop = 1;
+                    mbar_arrive(&bars.meta_full[buf]);
+                }
+                break;
+            }
+            const int32_t t = a.order[item / per_blk];
+            const int32_t rem = item % per_blk;
+            const int32_t g = rem / a.pairs;
+            const int32_t hp = rem % a.pairs;
+            const int32_t b = a.blk_req[t];
+            const int32_t cb = a.cu_blocks[b];
+            const int32_t i = t - cb;
+            const int32_t L = a.cu[b + 1] - a.cu[b];
+            int32_t* klist = klist_of(m);
+            uint32_t* pruned = pruned_of(m);
+            int32_t* ctiles = ctiles_of(m);
+            // kept list of (q-block t, KV head g), checked: ascending, in [0, i], ends at i
+            const int64_t lrow = static_cast<int64_t>(t) * a.hkv + g;
+            int32_t cnt = a.kept_cnt[lrow];
+            bool good = cnt >= 1 && cnt <= i + 1;
+            const int32_t* src = a.kept_idx + lrow * a.nb_max;
+            if (good)
+                for (int32_t e = lane; e < cnt; e += 32) klist[e] = src[e];
+            __syncwarp();
+            if (good) {
+                bool bad = false;
+                for (int32_t e = lane; e < cnt; e += 32)
+                    bad |= klist[e] < 0 || klist[e] > i || (e > 0 && klist[e] <= klist[e - 1]);
+                good = !__any_sync(0xffffffffu, bad) && klist[cnt - 1] == i;
+            }
+            if (!good) {
+                if (lane == 0) set_error(hdr, FP2_ERR_BAD_INDEX, t);
+                cnt = 1;
+                __syncwarp();
+                if (lane == 0) klist[0] = i;
+            }
+            // pruned blocks j < i (bit set) and the correction tiles holding any
+            const int32_t nwords = (i + 31) / 32;
+            for (int32_t w = lane; w < nwords; w += 32) {
+                const int32_t nbits = min(32, i - w * 32);
+                pruned[w] = (nbits == 32) ? 0xffffffffu : ((1u << nbits) - 1u);
+            }
+            __syncwarp();
+            for (int32_t e = lane; e < cnt - 1; e += 32) {
+                const int32_t j = klist[e];
+                atomicAnd(&pruned[j >> 5], ~(1u << (j & 31)));
+            }
+            __syncwarp();
+            int32_t nc = 0;
+            if (a.correction) {
+                const int32_t nct = (i + 127) / 128;
+                for (int32_t c0 = 0; c0 < nct; c0 += 32) {
+                    const int32_t ct = c0 + lane;
+                    uint32_t any = 0;
+                    if (ct < nct)
+                        for (int32_t w = ct * 4; w < min(ct * 4 + 4, nwords); ++w) any |= pruned[w];
+                    const uint32_t mask = __ballot_sync(0xffffffffu, any != 0);
+                    if (any) ctiles[nc + __popc(mask & ((1u << lane) - 1u))] = ct;
+                    nc += __popc(mask);
+                }
+            }
+            if (lane == 0) {
+                m->stop = 0;
+                m->t = t;
+                m->b = b;
+                m->i = i;
+                m->g = g;
+                m->h0 = g * a.G + 2 * hp;
+                m->ntiles = min(2, a.G - 2 * hp);
+                m->nrows = min(kBlock, L - i * kBlock);
+                m->qrow0 = a.cu[b] + i * kBlock;
+                m->cb = cb;
+                m->cnt = cnt;
+                m->ncorr = nc;
+                m->nwords = nwords;
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars.meta_full[buf]);
+        }
+      } else if (warp == kProducerWarp) {
+        // ---- TMA producer ----------------------------------------------------
         // lane 0 issues every TMA; the whole warp zeroes the V rows past the
         // request end of a partial diagonal block (a paged pool may hold
         // anything there, and zero attention weights times NaN is NaN)
@@ -291,67 +349,90 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_prefetch_desc(&tq);
             tma_prefetch_desc(&tk);
             tma_prefetch_desc(&tv);
-            mbar_arrive_expect_tx(&bars.q_full, ntiles * C::kTileBytes);
-            for (int qt = 0; qt < ntiles; ++qt)
-                for (int ch = 0; ch < C::kChunks; ++ch)
-                    tma_load_3d(q_s + qt * C::kTileBytes + ch * 16384, &tq, &bars.q_full, ch * 64,
-                                h0 + qt, qrow0);
         }
-        int32_t issued = 0;
-        for (int32_t n = 0; n < ntot && !*abort; ++n) {
-            const CUtensorMap* mk;
-            const CUtensorMap* mv;
-            int32_t row = 0;
-            if (n < cnt) {
-                const int32_t j = klist[cnt - 1 - n];
-                mk = &tk;
-                mv = &tv;
-                if (a.block_table) {
-                    int32_t page = a.block_table[static_cast<int64_t>(b) * a.max_blocks_per_seq + j];
-                    if (page < 0 || page >= a.num_pages) {
-                        if (leader) set_error(hdr, FP2_ERR_BAD_INDEX, t);
-                        page = 0;
-                    }
-                    row = page * kBlock;
-                } else {
-                    row = a.cu[b] + j * kBlock;
-                }
-            } else {
-                mk = &tkb;
-                mv = &tvb;
-                row = cb + ctiles[n - cnt] * 128;
-            }
+        int32_t issued = 0;  // K/V ring entries issued so far
+        for (int32_t k = 0; !*abort; ++k) {
+            const int32_t buf = k & 1;
+            if (!warp_wait(&bars.meta_full[buf], (k >> 1) & 1, hdr, abort, 510000 + k)) break;
+            ItemMeta* m = meta(buf);
+            if (m->stop) break;
+            const int32_t ntiles = m->ntiles, cnt = m->cnt, ntot = m->cnt + m->ncorr;
+            const int32_t nrows = m->nrows, g = m->g, b = m->b, t = m->t, cb = m->cb;
+            const int32_t* klist = klist_of(m);
+            const int32_t* ctiles = ctiles_of(m);
             bool ok = true;
-            for (int kv = 0; kv < 2 && ok; ++kv) {
-                const int32_t idx = 2 * n + kv;
-                const int32_t s = idx % C::kSlots;
-                if (leader) {
-                    ok = mbar_wait(&bars.kv_empty[s], ((idx / C::kSlots) & 1) ^ 1, hdr, abort,
-                                   100000 + idx);
-                    if (ok) {
-                        mbar_arrive_expect_tx(&bars.kv_full[s], C::kTileBytes);
+            for (int32_t n = 0; ok && n < ntot; ++n) {
+                if (n == 1 || (n == 0 && ntot == 1)) {
+                    // Q after the first K/V pair: those loads are already in flight
+                    // while the previous item's last MMAs still read the Q buffer
+                    if (leader) {
+                        if (k > 0) ok = mbar_wait(&bars.q_empty, (k - 1) & 1, hdr, abort, 520000 + k);
+                        if (ok) {
+                            mbar_arrive_expect_tx(&bars.q_full, ntiles * C::kTileBytes);
+                            for (int qt = 0; qt < ntiles; ++qt)
+                                for (int ch = 0; ch < C::kChunks; ++ch)
+                                    tma_load_3d(q_s + qt * C::kTileBytes + ch * 16384, &tq,
+                                                &bars.q_full, ch * 64, m->h0 + qt, m->qrow0);
+                        }
+                    }
+                    ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+                    if (!ok) break;
+                }
+                const CUtensorMap* mk;
+                const CUtensorMap* mv;
+                int32_t row = 0;
+                if (n < cnt) {
+                    const int32_t j = klist[cnt - 1 - n];
+                    mk = &tk;
+                    mv = &tv;
+                    if (a.block_table) {
+                        int32_t page = a.block_table[static_cast<int64_t>(b) * a.max_blocks_per_seq + j];
+                        if (page < 0 || page >= a.num_pages) {
+                            if (leader) set_error(hdr, FP2_ERR_BAD_INDEX, t);
+                            page = 0;
+                        }
+                        row = page * kBlock;
+                    } else {
+                        row = a.cu[b] + j * kBlock;
+                    }
+                } else {
+                    mk = &tkb;
+                    mv = &tvb;
+                    row = cb + ctiles[n - cnt] * 128;
+                }
+                for (int kv = 0; kv < 2 && ok; ++kv) {
+                    const int32_t idx = issued;
+                    const int32_t s = idx % C::kSlots;
+                    if (leader) {
+                        ok = mbar_wait(&bars.kv_empty[s], ((idx / C::kSlots) & 1) ^ 1, hdr, abort,
+                                       100000 + n);
+                        if (ok) {
+                            mbar_arrive_expect_tx(&bars.kv_full[s], C::kTileBytes);
+                            for (int ch = 0; ch < C::kChunks; ++ch)
+                                tma_load_3d(kv_s + s * C::kTileBytes + ch * 16384, kv ? mv : mk,
+                                            &bars.kv_full[s], ch * 64, g, row);
+                        }
+                    }
+                    ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+                    if (!ok) break;
+                    ++issued;
+                    if (kv == 1 && n == 0 && nrows < kBlock) {
+                        ok = warp_wait(&bars.kv_full[s], (idx / C::kSlots) & 1, hdr, abort, 150000);
+                        if (!ok) break;
+                        uint8_t* vt = kv_s + s * C::kTileBytes;
+                        const int32_t nz = (kBlock - nrows) * 8;  // 16-byte units per chunk
                         for (int ch = 0; ch < C::kChunks; ++ch)
-                            tma_load_3d(kv_s + s * C::kTileBytes + ch * 16384, kv ? mv : mk,
-                                        &bars.kv_full[s], ch * 64, g, row);
+                            for (int32_t e = lane; e < nz; e += 32)
+                                *reinterpret_cast<uint4*>(vt + ch * 16384 + nrows * 128 + e * 16) =
+                                    make_uint4(0u, 0u, 0u, 0u);
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (leader) mbar_arrive(&bars.v_tail);
                     }
                 }
-                ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-                if (!ok) break;
-                ++issued;
-                if (kv == 1 && n == 0 && nrows < kBlock) {
-                    ok = warp_wait(&bars.kv_full[s], (idx / C::kSlots) & 1, hdr, abort, 150000);
-                    if (!ok) break;
-                    uint8_t* vt = kv_s + s * C::kTileBytes;
-                    const int32_t nz = (kBlock - nrows) * 8;  // 16-byte units per chunk
-                    for (int ch = 0; ch < C::kChunks; ++ch)
-                        for (int32_t e = lane; e < nz; e += 32)
-                            *reinterpret_cast<uint4*>(vt + ch * 16384 + nrows * 128 + e * 16) =
-                                make_uint4(0u, 0u, 0u, 0u);
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                    if (leader) mbar_arrive(&bars.v_tail);
-                }
             }
+            __syncwarp();
+            if (leader) mbar_arrive(&bars.meta_empty[buf]);
             if (!ok) break;
         }
         // drain: every issued tile has been consumed and released
@@ -363,191 +444,252 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
       } else if (warp == kMmaWarp) {
+        // ---- MMA issuer ------------------------------------------------------
         if (lane == 0) {
             const uint32_t q_addr = smem_u32(q_s);
             const uint32_t kv_addr = smem_u32(kv_s);
-            // tile n: K in ring entry 2n, V in ring entry 2n + 1
             auto slot = [](int32_t idx) { return idx % C::kSlots; };
             auto phase = [](int32_t idx) { return static_cast<uint32_t>((idx / C::kSlots) & 1); };
-            bool ok = mbar_wait(&bars.q_full, 0, hdr, abort, 300000) &&
-                      mbar_wait(&bars.kv_full[slot(0)], phase(0), hdr, abort, 301000);
-            if (ok) {
+            int32_t base = 0;          // ring entry of the current item's first K tile
+            int32_t it[2] = {0, 0};    // PV iterations issued per Q tile
+            int32_t vt = 0;            // partial diagonal blocks seen
+            bool ok = true;
+            for (int32_t k = 0; ok; ++k) {
+                const int32_t buf = k & 1;
+                if (!(ok = mbar_wait(&bars.meta_full[buf], (k >> 1) & 1, hdr, abort, 530000 + k))) break;
+                ItemMeta* m = meta(buf);
+                if (m->stop) break;
+                const int32_t ntiles = m->ntiles, ntot = m->cnt + m->ncorr;
+                const bool partial = m->nrows < kBlock;
+                ok = mbar_wait(&bars.q_full, k & 1, hdr, abort, 300000) &&
+                     mbar_wait(&bars.kv_full[slot(base)], phase(base), hdr, abort, 301000);
+                if (!ok) break;
                 tc_fence_after();
                 for (int qt = 0; qt < ntiles; ++qt) {
                     issue_qk<kE4M3>(tmem + qt * 128, q_addr + qt * C::kTileBytes,
-                                    kv_addr + slot(0) * C::kTileBytes);
+                                    kv_addr + slot(base) * C::kTileBytes);
                     mma_commit(&bars.s_full[qt]);
                 }
-                mma_commit(&bars.kv_empty[slot(0)]);
-            }
-            for (int32_t n = 0; ok && n < ntot; ++n) {
-                const int32_t iv = 2 * n + 1, ik = 2 * n + 2;
-                const bool next = n + 1 < ntot;
-                if (!(ok = mbar_wait(&bars.kv_full[slot(iv)], phase(iv), hdr, abort, 330000 + n)))
-                    break;
-                if (n == 0 && nrows < kBlock &&
-                    !(ok = mbar_wait(&bars.v_tail, 0, hdr, abort, 335000)))
-                    break;
-                for (int qt = 0; qt < ntiles && ok; ++qt) {
-                    if (!(ok = mbar_wait(&bars.p_full[qt], n & 1, hdr, abort, 340000 + n))) break;
-                    tc_fence_after();
-                    issue_pv<kE4M3>(tmem + 256 + qt * 128, tmem + qt * 128,
-                                    kv_addr + slot(iv) * C::kTileBytes, n == 0);
-                    mma_commit(&bars.o_done[qt]);
-                    if (next) {
-                        if (qt == 0 && !(ok = mbar_wait(&bars.kv_full[slot(ik)], phase(ik), hdr,
-                                                        abort, 310000 + n)))
-                            break;
-                        tc_fence_after();
-                        issue_qk<kE4M3>(tmem + qt * 128, q_addr + qt * C::kTileBytes,
-                                        kv_addr + slot(ik) * C::kTileBytes);
-                        mma_commit(&bars.s_full[qt]);
+                mma_commit(&bars.kv_empty[slot(base)]);
+                for (int32_t n = 0; ok && n < ntot; ++n) {
+                    const int32_t iv = base + 2 * n + 1, ik = base + 2 * n + 2;
+                    const bool next = n + 1 < ntot;
+                    if (!(ok = mbar_wait(&bars.kv_full[slot(iv)], phase(iv), hdr, abort, 330000 + n)))
+                        break;
+                    if (n == 0 && partial) {
+                        if (!(ok = mbar_wait(&bars.v_tail, vt & 1, hdr, abort, 335000))) break;
+                        ++vt;
                     }
+                    for (int qt = 0; qt < ntiles && ok; ++qt) {
+                        if (!(ok = mbar_wait(&bars.p_full[qt], it[qt] & 1, hdr, abort, 340000 + n))) break;
+                        ++it[qt];
+                        tc_fence_after();
+                        issue_pv<kE4M3>(tmem + 256 + qt * 128, tmem + qt * 128,
+                                        kv_addr + slot(iv) * C::kTileBytes, n == 0);
+                        mma_commit(&bars.o_done[qt]);
+                        if (next) {
+                            if (qt == 0 && !(ok = mbar_wait(&bars.kv_full[slot(ik)], phase(ik), hdr,
+                                                            abort, 310000 + n)))
+                                break;
+                            tc_fence_after();
+                            issue_qk<kE4M3>(tmem + qt * 128, q_addr + qt * C::kTileBytes,
+                                            kv_addr + slot(ik) * C::kTileBytes);
+                            mma_commit(&bars.s_full[qt]);
+                        }
+                    }
+                    if (!ok) break;
+                    if (next) mma_commit(&bars.kv_empty[slot(ik)]);
+                    mma_commit(&bars.kv_empty[slot(iv)]);
                 }
-                if (!ok) break;
-                if (next) mma_commit(&bars.kv_empty[slot(ik)]);
-                mma_commit(&bars.kv_empty[slot(iv)]);
+                // every S MMA of this item has been issued: Q is free once they finish
+                mma_commit(&bars.q_empty);
+                base += 2 * ntot;
+                mbar_arrive(&bars.meta_empty[buf]);
             }
         }
       }
-    } else if (regs_inc<kSoftmaxRegs>(), warp / 4 < ntiles) {
+    } else {
+        regs_inc<kSoftmaxRegs>();
         // ---- softmax + epilogue of Q tile qt ---------------------------------
         const int qt = warp / 4;
         const int32_t r = tid & 127;
-        const int32_t h = h0 + qt;
         const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
         const uint32_t s_addr = tmem + lane_off + qt * 128;
         const uint32_t o_addr = tmem + lane_off + 256 + qt * 128;
-        float qk = a.scale_log2;
-        if (kE4M3) qk *= a.q_scale[h] * a.k_scale[g];
-        // correction tiles: +log2(128) after scaling == +7/qk before it
-        const float corr_bias = 7.f / qk;
-        float m_ref = -INFINITY;
-        float l = 0.f;      // row sum of the weights the PV MMA uses (O normaliser)
-        float l_lse = 0.f;  // row sum before P is rounded to the MMA precision (LSE)
+        int32_t it = 0;  // iterations of this Q tile so far (barrier phases)
         bool ok = true;
-        for (int32_t n = 0; n < ntot; ++n) {
-            if (!(ok = warp_wait(&bars.s_full[qt], n & 1, hdr, abort, 400000 + n))) break;
-            tc_fence_after();
-            uint32_t sv[128];
-            tmem_ld32(s_addr + 0, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-            tmem_ld32(s_addr + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
-            tmem_ld32(s_addr + 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[64]));
-            tmem_ld32(s_addr + 96, *reinterpret_cast<uint32_t(*)[32]>(&sv[96]));
-            tmem_wait_ld();
-            // masks (warp-uniform branch per tile kind):
-            //   diagonal block (n == 0): keys c <= r
-            //   kept block: every key
-            //   correction tile: pruned block means only, weighted by 128
-            if (n == 0) {
-#pragma unroll
-                for (int c = 0; c < 128; ++c)
-                    if (c > r) sv[c] = __float_as_uint(-INFINITY);
-            } else if (n >= cnt) {
-                const int32_t w0 = ctiles[n - cnt] * 4;
-#pragma unroll
-                for (int wi = 0; wi < 4; ++wi) {
-                    const uint32_t bits = (w0 + wi < nwords) ? pruned[w0 + wi] : 0u;
-#pragma unroll
-                    for (int c = 0; c < 32; ++c)
-                        sv[wi * 32 + c] =
-                            ((bits >> c) & 1u)
-                                ? __float_as_uint(__uint_as_float(sv[wi * 32 + c]) + corr_bias)
-                                : __float_as_uint(-INFINITY);
-                }
+        for (int32_t k = 0; ok; ++k) {
+            const int32_t buf = k & 1;
+            if (!(ok = warp_wait(&bars.meta_full[buf], (k >> 1) & 1, hdr, abort, 540000 + k))) break;
+            ItemMeta* m = meta(buf);
+            if (m->stop) break;
+            if (qt >= m->ntiles) {
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars.meta_empty[buf]);
+                continue;
             }
-            float mx = -INFINITY;
-#pragma unroll
-            for (int c = 0; c < 128; ++c) mx = fmaxf(mx, __uint_as_float(sv[c]));
-            const float m_new = fmaxf(m_ref, mx * qk);
-            const bool need = m_new > m_ref + C::kRescale;
-            if (__any_sync(0xffffffffu, need)) {
-                const float f = need ? ex2(m_ref - m_new) : 1.f;
-                if (n > 0) {
-                    if (!(ok = warp_wait(&bars.o_done[qt], (n - 1) & 1, hdr, abort, 410000 + n))) break;
-                    tc_fence_after();
-#pragma unroll
-                    for (int c0 = 0; c0 < 128; c0 += 32) {
-                        uint32_t ov[32];
-                        tmem_ld32(o_addr + c0, ov);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int c = 0; c < 32; ++c) ov[c] = __float_as_uint(__uint_as_float(ov[c]) * f);
-                        tmem_st32(o_addr + c0, ov);
-                    }
-                    tmem_wait_st();
-                }
-                if (need) {
-                    l *= f;
-                    l_lse *= f;
-                    m_ref = m_new;
-                }
-            }
-            // P = exp2(s * qk - m + offset) in the MMA precision, written over S
-            const float neg = C::kPOffset - ((m_ref == -INFINITY) ? 0.f : m_ref);
-            float rs = 0.f;
-#pragma unroll
-            for (int c = 0; c < 128; ++c) {
-                const float p = ex2(fmaf(__uint_as_float(sv[c]), qk, neg));
-                sv[c] = __float_as_uint(p);
-                rs += p;
-            }
-            l_lse += rs;
-            if (kE4M3) {
-                // the O normaliser sums the quantised weights the PV MMA sees
-                __half2 hs = __float2half2_rn(0.f);
-#pragma unroll
-                for (int c = 0; c < 32; ++c) {
-                    const uint32_t pk =
-                        pack_e4m3x4(__uint_as_float(sv[4 * c]), __uint_as_float(sv[4 * c + 1]),
-                                    __uint_as_float(sv[4 * c + 2]), __uint_as_float(sv[4 * c + 3]));
-                    hs = __hadd2(hs, e4m3x4_sum2(pk));
-                    sv[c] = pk;
-                }
-                const float2 hf = __half22float2(hs);
-                l += hf.x + hf.y;
-                tmem_st32(s_addr, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-            } else {
-                l += rs;
-#pragma unroll
-                for (int c = 0; c < 64; ++c)
-                    sv[c] = pack_bf16(__uint_as_float(sv[2 * c]), __uint_as_float(sv[2 * c + 1]));
-                tmem_st32(s_addr, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-                tmem_st32(s_addr + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
-            }
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(&bars.p_full[qt]);
-        }
-        // ---- epilogue: O / l -> bf16 ----------------------------------------
-        if (ok && ntot > 0 && warp_wait(&bars.o_done[qt], (ntot - 1) & 1, hdr, abort, 420000)) {
-            tc_fence_after();
-            float inv = 1.f / l;
-            if (kE4M3) inv *= a.v_scale[g];
-            uint16_t* orow = static_cast<uint16_t*>(a.out) +
-                             (static_cast<int64_t>(qrow0 + r) * a.hq + h) * kHeadDim;
-#pragma unroll
-            for (int c0 = 0; c0 < 128; c0 += 32) {
-                uint32_t ov[32];
-                tmem_ld32(o_addr + c0, ov);
+            const int32_t cnt = m->cnt, ntot = m->cnt + m->ncorr, nwords = m->nwords;
+            const int32_t g = m->g, h = m->h0 + qt, nrows = m->nrows, qrow0 = m->qrow0;
+            const uint32_t* pruned = pruned_of(m);
+            const int32_t* ctiles = ctiles_of(m);
+            float qk = a.scale_log2;
+            if (kE4M3) qk *= a.q_scale[h] * a.k_scale[g];
+            // correction tiles: +log2(128) after scaling == +7/qk before it
+            const float corr_bias = 7.f / qk;
+            float m_ref = -INFINITY;
+            float l = 0.f;      // row sum of the weights the PV MMA uses (O normaliser)
+            float l_lse = 0.f;  // row sum before P is rounded to the MMA precision (LSE)
+            for (int32_t n = 0; n < ntot; ++n) {
+                if (!(ok = warp_wait(&bars.s_full[qt], it & 1, hdr, abort, 400000 + n))) break;
+                tc_fence_after();
+                uint32_t sv[128];
+                tmem_ld32(s_addr + 0, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+                tmem_ld32(s_addr + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+                tmem_ld32(s_addr + 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[64]));
+                tmem_ld32(s_addr + 96, *reinterpret_cast<uint32_t(*)[32]>(&sv[96]));
                 tmem_wait_ld();
-                if (r < nrows) {
-                    uint32_t pk[16];
+                // masks (warp-uniform branch per tile kind):
+                //   diagonal block (n == 0): keys c <= r
+                //   kept block: every key
+                //   correction tile: pruned block means only, weighted by 128
+                if (n == 0) {
 #pragma unroll
-                    for (int c = 0; c < 16; ++c)
-                        pk[c] = pack_bf16(__uint_as_float(ov[2 * c]) * inv,
-                                          __uint_as_float(ov[2 * c + 1]) * inv);
-                    uint4* dst = reinterpret_cast<uint4*>(orow + c0);
+                    for (int c = 0; c < 128; ++c)
+                        if (c > r) sv[c] = __float_as_uint(-INFINITY);
+                } else if (n >= cnt) {
+                    const int32_t w0 = ctiles[n - cnt] * 4;
 #pragma unroll
-                    for (int c = 0; c < 4; ++c)
-                        dst[c] = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+                    for (int wi = 0; wi < 4; ++wi) {
+                        const uint32_t bits = (w0 + wi < nwords) ? pruned[w0 + wi] : 0u;
+#pragma unroll
+                        for (int c = 0; c < 32; ++c)
+                            sv[wi * 32 + c] =
+                                ((bits >> c) & 1u)
+                                    ? __float_as_uint(__uint_as_float(sv[wi * 32 + c]) + corr_bias)
+                                    : __float_as_uint(-INFINITY);
+                    }
+                }
+                // row max over 4 independent 3-input max chains
+                float mxp[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) mxp[j] = -INFINITY;
+#pragma unroll
+                for (int c = 0; c < 128; c += 2)
+                    mxp[(c >> 1) & 3] =
+                        fmax3(mxp[(c >> 1) & 3], __uint_as_float(sv[c]), __uint_as_float(sv[c + 1]));
+                const float mx = fmax3(mxp[0], mxp[1], fmaxf(mxp[2], mxp[3]));
+                const float m_new = fmaxf(m_ref, mx * qk);
+                const bool need = m_new > m_ref + C::kRescale;
+                if (__any_sync(0xffffffffu, need)) {
+                    const float f = need ? ex2(m_ref - m_new) : 1.f;
+                    if (n > 0) {
+                        if (!(ok = warp_wait(&bars.o_done[qt], (it - 1) & 1, hdr, abort, 410000 + n)))
+                            break;
+                        tc_fence_after();
+#pragma unroll
+                        for (int c0 = 0; c0 < 128; c0 += 32) {
+                            uint32_t ov[32];
+                            tmem_ld32(o_addr + c0, ov);
+                            tmem_wait_ld();
+#pragma unroll
+                            for (int c = 0; c < 32; ++c)
+                                ov[c] = __float_as_uint(__uint_as_float(ov[c]) * f);
+                            tmem_st32(o_addr + c0, ov);
+                        }
+                        tmem_wait_st();
+                    }
+                    if (need) {
+                        l *= f;
+                        l_lse *= f;
+                        m_ref = m_new;
+                    }
+                }
+                // P = exp2(s * qk - m + offset) in the MMA precision, written over S
+                const float neg = C::kPOffset - ((m_ref == -INFINITY) ? 0.f : m_ref);
+                // exp2 of packed pairs (MUFU; optionally some pairs on the FMA pipe)
+                float2 rsp[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) rsp[j] = make_float2(0.f, 0.f);
+#pragma unroll
+                for (int c = 0; c < 128; c += 2) {
+                    float2 x = ffma2(make_float2(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])),
+                                     make_float2(qk, qk), make_float2(neg, neg));
+                    if (kEmuEvery > 0 && ((c >> 1) % (kEmuEvery > 0 ? kEmuEvery : 1)) == kEmuEvery - 1) {
+                        x = exp2_poly2(x);
+                    } else {
+                        x.x = ex2(x.x);
+                        x.y = ex2(x.y);
+                    }
+                    sv[c] = __float_as_uint(x.x);
+                    sv[c + 1] = __float_as_uint(x.y);
+                    rsp[(c >> 1) & 3] = fadd2(rsp[(c >> 1) & 3], x);
+                }
+                const float2 rs2 = fadd2(fadd2(rsp[0], rsp[1]), fadd2(rsp[2], rsp[3]));
+                const float rs = rs2.x + rs2.y;
+                l_lse += rs;
+                if (kE4M3) {
+                    // the O normaliser sums the quantised weights the PV MMA sees
+                    __half2 hs[4];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) hs[j] = __float2half2_rn(0.f);
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) {
+                        const uint32_t pk = pack_e4m3x4(
+                            __uint_as_float(sv[4 * c]), __uint_as_float(sv[4 * c + 1]),
+                            __uint_as_float(sv[4 * c + 2]), __uint_as_float(sv[4 * c + 3]));
+                        hs[c & 3] = __hadd2(hs[c & 3], e4m3x4_sum2(pk));
+                        sv[c] = pk;
+                    }
+                    const float2 h01 = __half22float2(hs[0]), h23 = __half22float2(hs[1]);
+                    const float2 h45 = __half22float2(hs[2]), h67 = __half22float2(hs[3]);
+                    l += ((h01.x + h01.y) + (h23.x + h23.y)) + ((h45.x + h45.y) + (h67.x + h67.y));
+                    tmem_st32(s_addr, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+                } else {
+                    l += rs;
+#pragma unroll
+                    for (int c = 0; c < 64; ++c)
+                        sv[c] = pack_bf16(__uint_as_float(sv[2 * c]), __uint_as_float(sv[2 * c + 1]));
+                    tmem_st32(s_addr, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+                    tmem_st32(s_addr + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(&bars.p_full[qt]);
+                ++it;
+            }
+            // ---- epilogue: O / l -> bf16 ------------------------------------
+            if (ok && ntot > 0 && (ok = warp_wait(&bars.o_done[qt], (it - 1) & 1, hdr, abort, 420000))) {
+                tc_fence_after();
+                float inv = 1.f / l;
+                if (kE4M3) inv *= a.v_scale[g];
+                uint16_t* orow = static_cast<uint16_t*>(a.out) +
+                                 (static_cast<int64_t>(qrow0 + r) * a.hq + h) * kHeadDim;
+#pragma unroll
+                for (int c0 = 0; c0 < 128; c0 += 32) {
+                    uint32_t ov[32];
+                    tmem_ld32(o_addr + c0, ov);
+                    tmem_wait_ld();
+                    if (r < nrows) {
+                        uint32_t pk[16];
+#pragma unroll
+                        for (int c = 0; c < 16; ++c)
+                            pk[c] = pack_bf16(__uint_as_float(ov[2 * c]) * inv,
+                                              __uint_as_float(ov[2 * c + 1]) * inv);
+                        uint4* dst = reinterpret_cast<uint4*>(orow + c0);
+#pragma unroll
+                        for (int c = 0; c < 4; ++c)
+                            dst[c] = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+                    }
+                }
+                if (a.lse && r < nrows) {
+                    const float m_use = ((m_ref == -INFINITY) ? 0.f : m_ref) - C::kPOffset;
+                    a.lse[static_cast<int64_t>(qrow0 + r) * a.hq + h] =
+                        (m_use + __log2f(l_lse)) * 0.69314718055994530942f;
                 }
             }
-            if (a.lse && r < nrows) {
-                const float m_use = ((m_ref == -INFINITY) ? 0.f : m_ref) - C::kPOffset;
-                a.lse[static_cast<int64_t>(qrow0 + r) * a.hq + h] =
-                    (m_use + __log2f(l_lse)) * 0.69314718055994530942f;
-            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars.meta_empty[buf]);
         }
     }
 
@@ -562,15 +704,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 size_t attn_smem_bytes(bool e4m3, int32_t nb_cap) {
     const size_t tiles = e4m3 ? tiles_bytes<true>() : tiles_bytes<false>();
-    return 1024 + tiles + sizeof(SmemMisc) + lists_bytes(nb_cap);
+    return 1024 + tiles + sizeof(SmemMisc) + 2 * meta_bytes(nb_cap);
 }
 
 cudaError_t launch_attention(bool e4m3, const AttnArgs& a, const CUtensorMap& tq,
                              const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tkb,
                              const CUtensorMap& tvb, int64_t max_blocks, cudaStream_t stream) {
     const size_t smem = attn_smem_bytes(e4m3, a.nb_cap);
-    const int64_t grid = max_blocks * a.hkv * a.pairs;
-    if (grid <= 0) return cudaSuccess;
+    const int64_t items = max_blocks * a.hkv * a.pairs;
+    if (items <= 0) return cudaSuccess;
     // the setmaxnreg split assumes the kernel was built with kLaunchRegs per
     // thread; with fewer, the softmax warps' register request could never be met
     cudaFuncAttributes fa;
@@ -578,18 +720,22 @@ cudaError_t launch_attention(bool e4m3, const AttnArgs& a, const CUtensorMap& tq
                            : cudaFuncGetAttributes(&fa, attention_kernel<false>);
     if (err != cudaSuccess) return err;
     if (fa.numRegs < kLaunchRegs) return cudaErrorInvalidConfiguration;
+    // persistent: one CTA per SM, work items taken from a counter in the workspace
+    int dev = 0, sms = 0;
+    if ((err = cudaGetDevice(&dev)) != cudaSuccess) return err;
+    if ((err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+        return err;
+    const unsigned grid = static_cast<unsigned>(items < sms ? items : sms);
     if (e4m3) {
         err = cudaFuncSetAttribute(attention_kernel<true>,
                                    cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
         if (err != cudaSuccess) return err;
-        attention_kernel<true><<<dim3(static_cast<unsigned>(grid)), kThreads, smem, stream>>>(
-            a, tq, tk, tv, tkb, tvb);
+        attention_kernel<true><<<grid, kThreads, smem, stream>>>(a, tq, tk, tv, tkb, tvb);
     } else {
         err = cudaFuncSetAttribute(attention_kernel<false>,
                                    cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
         if (err != cudaSuccess) return err;
-        attention_kernel<false><<<dim3(static_cast<unsigned>(grid)), kThreads, smem, stream>>>(
-            a, tq, tk, tv, tkb, tvb);
+        attention_kernel<false><<<grid, kThreads, smem, stream>>>(a, tq, tk, tv, tkb, tvb);
     }
     return cudaGetLastError();
 }

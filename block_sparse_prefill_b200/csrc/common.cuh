@@ -19,6 +19,7 @@ struct WsHeader {
     int32_t detail;        // detail of that error (offending index, ...)
     int32_t valid;         // 1 when the last setup pass accepted cu_seqlens
     int32_t total_blocks;  // sum_b ceil(L_b / block_size) of the last setup pass
+    int32_t work_next;     // next work item of the persistent attention kernel
 };
 
 // Byte offsets of the workspace regions (all 256-byte aligned).
@@ -26,6 +27,7 @@ struct WsLayout {
     size_t cu_blocks;   // int32 [batch + 1]
     size_t cu_tiles;    // int32 [batch + 1] (estimator q-tiles)
     size_t blk_req;     // int32 [max_blocks]
+    size_t order;       // int32 [max_blocks]: global blocks by block index in the request, descending
     size_t qbar;        // fp32  [max_blocks, Hq, d]
     size_t kbar_lp;     // bf16 / e4m3 [max_blocks, Hkv, d] (operands of the correction MMA)
     size_t vbar_lp;     // bf16 / e4m3 [max_blocks, Hkv, d]
@@ -43,6 +45,8 @@ __host__ __device__ inline WsLayout ws_layout(int32_t batch, int64_t max_blocks,
     w.cu_tiles = off;
     off = align256(off + sizeof(int32_t) * (batch + 1));
     w.blk_req = off;
+    off = align256(off + sizeof(int32_t) * max_blocks);
+    w.order = off;
     off = align256(off + sizeof(int32_t) * max_blocks);
     w.qbar = off;
     off = align256(off + sizeof(float) * max_blocks * hq * kHeadDim);

@@ -25,6 +25,7 @@ namespace fp2 {
 // set-up
 // ---------------------------------------------------------------------------
 __global__ void setup_kernel(SetupArgs a) {
+    extern __shared__ int32_t hist[];  // [nb_cap + 1]
     __shared__ int32_t ok;
     if (threadIdx.x == 0) {
         int32_t good = 1, bad = -1;
@@ -46,14 +47,34 @@ __global__ void setup_kernel(SetupArgs a) {
         if (good && nb_acc > a.max_blocks) { good = 0; bad = a.batch; }
         a.hdr->valid = good;
         a.hdr->total_blocks = good ? nb_acc : 0;
+        a.hdr->work_next = 0;
         if (!good) set_error(a.hdr, FP2_ERR_BAD_INDEX, bad);
         ok = good;
     }
+    for (int32_t e = threadIdx.x; e <= a.nb_cap; e += blockDim.x) hist[e] = 0;
     __syncthreads();
     if (!ok) return;
     for (int32_t b = 0; b < a.batch; ++b)
-        for (int32_t t = a.cu_blocks[b] + threadIdx.x; t < a.cu_blocks[b + 1]; t += blockDim.x)
+        for (int32_t t = a.cu_blocks[b] + threadIdx.x; t < a.cu_blocks[b + 1]; t += blockDim.x) {
             a.blk_req[t] = b;
+            atomicAdd(&hist[t - a.cu_blocks[b]], 1);
+        }
+    __syncthreads();
+    // order: blocks sorted by their index in the request, largest first (the
+    // causal kept lists grow with it), so the persistent attention kernel
+    // takes the longest work items first
+    if (threadIdx.x == 0) {
+        int32_t run = 0;
+        for (int32_t j = a.nb_cap - 1; j >= 0; --j) {
+            const int32_t c = hist[j];
+            hist[j] = run;
+            run += c;
+        }
+    }
+    __syncthreads();
+    for (int32_t b = 0; b < a.batch; ++b)
+        for (int32_t t = a.cu_blocks[b] + threadIdx.x; t < a.cu_blocks[b + 1]; t += blockDim.x)
+            a.order[atomicAdd(&hist[t - a.cu_blocks[b]], 1)] = t;
 }
 
 // ---------------------------------------------------------------------------

@@ -20,10 +20,12 @@ struct SetupArgs {
     int32_t paged;
     int32_t max_blocks_per_seq;
     int64_t max_blocks;
+    int32_t nb_cap;  // >= blocks of the longest request (histogram bins)
     WsHeader* hdr;
     int32_t* cu_blocks;
     int32_t* cu_tiles;
     int32_t* blk_req;
+    int32_t* order;
 };
 
 struct PoolArgs {
@@ -76,6 +78,7 @@ struct AttnArgs {
     const int32_t* cu;
     const int32_t* cu_blocks;
     const int32_t* blk_req;
+    const int32_t* order;        // global blocks, heaviest (largest block index) first
     const int32_t* block_table;  // NULL = contiguous K/V
     int32_t max_blocks_per_seq;
     int32_t num_pages;

@@ -261,6 +261,56 @@ __device__ __forceinline__ uint32_t pack_e4m3x4(float x0, float x1, float x2, fl
     return static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
 }
 
+// ---------------------------------------------------------------------------
+// Packed fp32 pairs (sm_100 f32x2 instructions) and 3-input max
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+    float2 r;
+    asm("{.reg .b64 ra, rb, rc, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;}"
+        : "=f"(r.x), "=f"(r.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return r;
+}
+
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+    float2 r;
+    asm("{.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;}"
+        : "=f"(r.x), "=f"(r.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return r;
+}
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+// 2^x for a pair of inputs on the FMA pipe instead of MUFU: x = n + f with
+// n = round(x) (the 1.5 * 2^23 rounding constant) and f in [-1/2, 1/2];
+// 2^f by a degree-3 polynomial with minimax relative error 7.5e-5 on that
+// interval (Remez exchange; coefficients from exp2_poly.py); 2^n added to the
+// exponent field.  Inputs are clamped at -126 so that the exponent cannot wrap
+// (the result there is ~1e-38, i.e. zero for the attention weights).
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+    constexpr float kRound = 12582912.f;  // 1.5 * 2^23
+    x.x = fmaxf(x.x, -126.f);
+    x.y = fmaxf(x.y, -126.f);
+    const float2 t = fadd2(x, make_float2(kRound, kRound));
+    const float2 n = fadd2(t, make_float2(-kRound, -kRound));
+    const float2 f = ffma2(n, make_float2(-1.f, -1.f), x);
+    float2 p = ffma2(make_float2(5.517166853e-02f, 5.517166853e-02f), f,
+                     make_float2(2.426111251e-01f, 2.426111251e-01f));
+    p = ffma2(p, f, make_float2(6.932609677e-01f, 6.932609677e-01f));
+    p = ffma2(p, f, make_float2(9.999280572e-01f, 9.999280572e-01f));
+    return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
+                       __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
+}
+
 // Sum of the four e4m3 values packed in `w` (exact decode to f16x2, f16x2 adds).
 __device__ __forceinline__ __half2 e4m3x4_sum2(uint32_t w) {
     uint32_t lo, hi;
