@@ -53,6 +53,19 @@ bool make_map(CUtensorMap* m, const void* base, bool e4m3, int64_t heads, int64_
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 2-D bf16 map over [rows, 128] with 128-byte-swizzled boxes of 128 rows x 64 columns.
+bool make_map_2d(CUtensorMap* m, const void* base, int64_t rows) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kHeadDim), static_cast<cuuint64_t>(rows > 0 ? rows : 1)};
+    const cuuint64_t strides[1] = {kHeadDim * 2};
+    const cuuint32_t box[2] = {64, 128};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 int32_t esize(const fp2_params* p) { return p->dtype == FP2_E4M3 ? 1 : 2; }
@@ -122,24 +135,11 @@ T* at(void* ws, size_t off) {
 
 fp2_status launched(cudaError_t e) { return e == cudaSuccess ? FP2_OK : FP2_ERR_CUDA; }
 
-// Score-kernel tiling: q-blocks per tile so that the score rows fit in shared memory.
-bool score_tiling(int32_t G, int32_t nb_need, int32_t* qt, int32_t* rp, int32_t* ncap, size_t* smem) {
-    const int32_t cap = ((nb_need + kScoreKC - 1) / kScoreKC) * kScoreKC;
-    int32_t q = G >= 32 ? 1 : 32 / G;
-    while (true) {
-        const int32_t r = ((q * G + 3) / 4) * 4;
-        const size_t bytes = sizeof(float) * (size_t(kHeadDim) * r + size_t(kHeadDim) * (kScoreKC + 4) +
-                                              size_t(r) * cap + r);
-        if (r <= 64 && bytes <= kMaxSmem) {
-            *qt = q;
-            *rp = r;
-            *ncap = cap > 0 ? cap : kScoreKC;
-            *smem = bytes;
-            return true;
-        }
-        if (q == 1) return false;
-        q /= 2;
-    }
+// Score-kernel tiling: q-blocks per 128-row tile (rows = q-block x query head).
+bool score_tiling(int32_t G, int32_t* qt) {
+    if (G < 1 || G > 128) return false;
+    *qt = 128 / G;
+    return true;
 }
 
 fp2_status run_setup(const Problem& pr, void* ws, const int32_t* cu, int32_t qt, bool paged,
@@ -174,9 +174,8 @@ fp2_status run_estimate(const fp2_params* p, const void* q, const void* k, const
                         int32_t mbps, int32_t num_pages, fp2_blockmeta* meta, void* ws,
                         cudaStream_t s) {
     const int32_t G = p->num_q_heads / p->num_kv_heads;
-    int32_t qt, rp, ncap;
-    size_t score_smem;
-    if (!score_tiling(G, pr.nb_need, &qt, &rp, &ncap, &score_smem)) return FP2_ERR_UNSUPPORTED;
+    int32_t qt;
+    if (!score_tiling(G, &qt)) return FP2_ERR_UNSUPPORTED;
     fp2_status st = run_setup(pr, ws, cu, qt, block_table != nullptr, mbps, meta->max_blocks, s);
     if (st != FP2_OK || pr.batch == 0 || pr.max_blocks == 0) return st;
 
@@ -187,9 +186,13 @@ fp2_status run_estimate(const fp2_params* p, const void* q, const void* k, const
     pa.x[0] = q;
     pa.x[1] = k;
     pa.x[2] = v;
-    pa.out[0] = at<float>(ws, pr.ws.qbar);
+    pa.out[0] = nullptr;
     pa.out[1] = meta->k_mean;
     pa.out[2] = meta->v_mean;
+    pa.split[0] = at<uint16_t>(ws, pr.ws.qsplit);
+    pa.split[1] = at<uint16_t>(ws, pr.ws.ksplit);
+    pa.G = G;
+    pa.max_blocks = pr.max_blocks;
     pa.scale[0] = e4m3 ? p->q_scale : nullptr;
     pa.scale[1] = e4m3 ? p->k_scale : nullptr;
     pa.scale[2] = e4m3 ? p->v_scale : nullptr;
@@ -217,8 +220,6 @@ fp2_status run_estimate(const fp2_params* p, const void* q, const void* k, const
     if ((st = launched(cudaGetLastError())) != FP2_OK) return st;
 
     ScoreArgs sa;
-    sa.qbar = at<float>(ws, pr.ws.qbar);
-    sa.kbar = meta->k_mean;
     sa.cu_blocks = at<int32_t>(ws, pr.ws.cu_blocks);
     sa.cu_tiles = at<int32_t>(ws, pr.ws.cu_tiles);
     sa.batch = pr.batch;
@@ -226,8 +227,7 @@ fp2_status run_estimate(const fp2_params* p, const void* q, const void* k, const
     sa.hkv = p->num_kv_heads;
     sa.G = G;
     sa.qt = qt;
-    sa.rp = rp;
-    sa.ncap = ncap;
+    sa.max_blocks = pr.max_blocks;
     sa.nb_max = meta->nb_max;
     sa.tau = tau_of(p);
     sa.keep_all = p->alpha <= 0.f ? 1 : 0;
@@ -236,12 +236,21 @@ fp2_status run_estimate(const fp2_params* p, const void* q, const void* k, const
     sa.kept_idx = meta->kept_idx;
     sa.score_dbg = meta->score_dbg;
     sa.hdr = hdr;
+    uint16_t* qs = at<uint16_t>(ws, pr.ws.qsplit);
+    uint16_t* ks = at<uint16_t>(ws, pr.ws.ksplit);
+    const int64_t qrows = pr.max_blocks * p->num_q_heads;
+    const int64_t krows = pr.max_blocks * p->num_kv_heads;
+    CUtensorMap tqh, tql, tkh, tkl;
+    if (!make_map_2d(&tqh, qs, qrows) || !make_map_2d(&tql, qs + qrows * kHeadDim, qrows) ||
+        !make_map_2d(&tkh, ks, krows) || !make_map_2d(&tkl, ks + krows * kHeadDim, krows))
+        return FP2_ERR_CUDA;
+    const size_t smem = score_smem_bytes();
     if (cudaFuncSetAttribute(score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(score_smem)) != cudaSuccess)
+                             static_cast<int>(smem)) != cudaSuccess)
         return FP2_ERR_CUDA;
     const int64_t tiles = (pr.max_blocks + qt - 1) / qt + pr.batch;
     score_kernel<<<dim3(static_cast<unsigned>(tiles), static_cast<unsigned>(p->num_kv_heads)),
-                   rp * 8, score_smem, s>>>(sa);
+                   kScoreThreads, smem, s>>>(sa, tqh, tql, tkh, tkl);
     return launched(cudaGetLastError());
 }
 
@@ -443,8 +452,8 @@ fp2_status noalloc_scratch(void** addr) {
     return FP2_OK;
 }
 
-// The attention call reads no q-block means, so its scratch is the workspace
-// layout without that region.
+// The attention call reads none of the estimator's split means, so its
+// scratch is the workspace layout without those regions.
 WsLayout noalloc_layout(const Problem& pr, const fp2_params* p) {
     WsLayout w;
     size_t off = 256;
@@ -456,7 +465,8 @@ WsLayout noalloc_layout(const Problem& pr, const fp2_params* p) {
     off = align256(off + sizeof(int32_t) * pr.max_blocks);
     w.order = off;
     off = align256(off + sizeof(int32_t) * pr.max_blocks);
-    w.qbar = off;
+    w.qsplit = off;
+    w.ksplit = off;
     w.kbar_lp = off;
     off = align256(off + size_t(esize(p)) * pr.max_blocks * p->num_kv_heads * kHeadDim);
     w.vbar_lp = off;

@@ -28,7 +28,9 @@ struct WsLayout {
     size_t cu_tiles;    // int32 [batch + 1] (estimator q-tiles)
     size_t blk_req;     // int32 [max_blocks]
     size_t order;       // int32 [max_blocks]: global blocks by block index in the request, descending
-    size_t qbar;        // fp32  [max_blocks, Hq, d]
+    size_t qsplit;      // bf16 [2][Hkv][max_blocks * G][d]: q-block means as hi + lo parts,
+                        // rows of one KV head's query heads grouped (row = block * G + head)
+    size_t ksplit;      // bf16 [2][Hkv][max_blocks][d]: key-block means as hi + lo parts
     size_t kbar_lp;     // bf16 / e4m3 [max_blocks, Hkv, d] (operands of the correction MMA)
     size_t vbar_lp;     // bf16 / e4m3 [max_blocks, Hkv, d]
     size_t total;
@@ -48,8 +50,10 @@ __host__ __device__ inline WsLayout ws_layout(int32_t batch, int64_t max_blocks,
     off = align256(off + sizeof(int32_t) * max_blocks);
     w.order = off;
     off = align256(off + sizeof(int32_t) * max_blocks);
-    w.qbar = off;
-    off = align256(off + sizeof(float) * max_blocks * hq * kHeadDim);
+    w.qsplit = off;
+    off = align256(off + 2 * sizeof(uint16_t) * max_blocks * hq * kHeadDim);
+    w.ksplit = off;
+    off = align256(off + 2 * sizeof(uint16_t) * max_blocks * hkv * kHeadDim);
     w.kbar_lp = off;
     off = align256(off + size_t(esize) * max_blocks * hkv * kHeadDim);
     w.vbar_lp = off;

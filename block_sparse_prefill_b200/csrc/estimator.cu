@@ -187,26 +187,94 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(PoolArgs a) {
             for (int e = 0; e < N; ++e) acc[e] += red[g][tc][e];
         const int32_t h = col / kHeadDim;
         const float s = (a.scale[x] ? a.scale[x][h] : 1.f) / static_cast<float>(n);
-        float* out = a.out[x] + static_cast<int64_t>(t) * ncols + col;
 #pragma unroll
-        for (int e = 0; e < N; e += 4)
-            *reinterpret_cast<float4*>(out + e) =
-                make_float4(acc[e] * s, acc[e + 1] * s, acc[e + 2] * s, acc[e + 3] * s);
+        for (int e = 0; e < N; ++e) acc[e] *= s;
+        if (a.out[x]) {
+            float* out = a.out[x] + static_cast<int64_t>(t) * ncols + col;
+#pragma unroll
+            for (int e = 0; e < N; e += 4)
+                *reinterpret_cast<float4*>(out + e) = make_float4(acc[e], acc[e + 1], acc[e + 2], acc[e + 3]);
+        }
+        if (x < 2) {
+            // hi + lo bf16 parts for the score MMAs: hi = bf16(m), lo = bf16(m - hi)
+            int64_t row;
+            if (x == 0) {
+                const int32_t g = h / a.G, hh = h % a.G;
+                row = (static_cast<int64_t>(g) * a.max_blocks + t) * a.G + hh;
+            } else {
+                row = static_cast<int64_t>(h) * a.max_blocks + t;
+            }
+            const int64_t plane = (x == 0 ? static_cast<int64_t>(a.heads[0]) : a.heads[1]) * a.max_blocks * kHeadDim;
+            uint16_t* hi = a.split[x] + row * kHeadDim + (col % kHeadDim);
+            uint16_t* lo = hi + plane;
+            uint32_t ph[N / 2], pl[N / 2];
+#pragma unroll
+            for (int e = 0; e < N; e += 2) {
+                const uint32_t hp = pack_bf16(acc[e], acc[e + 1]);
+                const float h0 = __uint_as_float(hp << 16), h1 = __uint_as_float(hp & 0xFFFF0000u);
+                ph[e / 2] = hp;
+                pl[e / 2] = pack_bf16(acc[e] - h0, acc[e + 1] - h1);
+            }
+#pragma unroll
+            for (int e = 0; e < N / 2; e += 4) {
+                *reinterpret_cast<uint4*>(hi + 2 * e) = make_uint4(ph[e], ph[e + 1], ph[e + 2], ph[e + 3]);
+                *reinterpret_cast<uint4*>(lo + 2 * e) = make_uint4(pl[e], pl[e + 1], pl[e + 2], pl[e + 3]);
+            }
+        }
     }
 }
 
 // ---------------------------------------------------------------------------
-// scores, threshold, union, compaction
+// scores, threshold, union, compaction (tcgen05)
+//
+// One CTA = one KV head g x one tile of qt = floor(128 / G) q-blocks of one
+// request: 128 rows (q-block, query head) of qbar against all causal key
+// blocks, 128 key blocks per chunk.  s = tau * qbar . kbar is computed on the
+// tensor cores as hi.hi + hi.lo + lo.hi with bf16 hi/lo parts of the fp32
+// means (relative error about 2^-16, the fp32 accumulation in TMEM).
+//   pass 1: row max m over j <= i
+//   pass 2: the same scores again; keep bit = exp(s - m) >= alpha (or j == i);
+//           OR over the G rows of each q-block; ascending compaction.
+// warps 0-3: epilogue (row r = TMEM lane r); warp 4: TMA loads and MMA issue.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) score_kernel(ScoreArgs a) {
-    extern __shared__ __align__(16) float smem[];
-    const int32_t RP = a.rp;                  // padded rows (multiple of 4)
-    float* qs = smem;                         // [d][RP]
-    float* ks = qs + kHeadDim * RP;           // [d][KC + 4]
-    float* sc = ks + kHeadDim * (kScoreKC + 4);  // [RP][ncap]
-    float* rowmax = sc + static_cast<size_t>(RP) * a.ncap;  // [RP]
+namespace {
+constexpr int kTileQ = 32768;   // one 128 x 128 bf16 operand (two 64-column chunks)
 
-    if (!a.hdr->valid) return;
+struct ScoreSmem {
+    uint64_t q_full;
+    uint64_t kv_full[2];
+    uint64_t kv_empty[2];
+    uint64_t acc_full[2];
+    uint64_t acc_empty[2];
+    uint32_t tmem_base;
+    int32_t abort;
+    uint32_t keep[128][4];
+};
+
+__device__ __forceinline__ uint64_t score_desc(uint32_t base, int k) {
+    return sdesc_sw128(base + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024);
+}
+
+__device__ __forceinline__ void named_sync_epi() {
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+}
+}  // namespace
+
+__global__ void __launch_bounds__(kScoreThreads, 1)
+    score_kernel(const __grid_constant__ ScoreArgs a, const __grid_constant__ CUtensorMap tqh,
+                 const __grid_constant__ CUtensorMap tql, const __grid_constant__ CUtensorMap tkh,
+                 const __grid_constant__ CUtensorMap tkl) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+    uint8_t* qh = sm;
+    uint8_t* ql = sm + kTileQ;
+    uint8_t* kh = sm + 2 * kTileQ;      // 2 stages
+    uint8_t* kl = sm + 4 * kTileQ;      // 2 stages
+    ScoreSmem* ss = reinterpret_cast<ScoreSmem*>(sm + 6 * kTileQ);
+    volatile int32_t* abort = &ss->abort;
+    WsHeader* hdr = a.hdr;
+    if (!hdr->valid) return;
     const int32_t total_tiles = a.cu_tiles[a.batch];
     if (static_cast<int32_t>(blockIdx.x) >= total_tiles) return;
     const int32_t tile = total_tiles - 1 - blockIdx.x;  // late (long-row) tiles first
@@ -221,97 +289,158 @@ __global__ void __launch_bounds__(256) score_kernel(ScoreArgs a) {
     const int32_t cb = a.cu_blocks[b];
     const int32_t nb = a.cu_blocks[b + 1] - cb;
     const int32_t i0 = (tile - a.cu_tiles[b]) * a.qt;
-    const int32_t nqb = min(a.qt, nb - i0);
-    const int32_t nrows = nqb * G;
-    const int32_t ncols = i0 + nqb;
-    const int32_t tid = threadIdx.x;
-    const int32_t nthr = blockDim.x;
+    const int32_t nq = min(a.qt, nb - i0);
+    const int32_t nrows = nq * G;
+    const int32_t nchunk = (i0 + nq - 1) / 128 + 1;
+    const int32_t steps = 2 * nchunk;
+    const int32_t tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
-    // q rows, transposed: qs[c][rho], rho = ii * G + hh
-    for (int32_t e = tid; e < RP * kHeadDim; e += nthr) {
-        const int32_t rho = e / kHeadDim, c = e % kHeadDim;
-        float v = 0.f;
-        if (rho < nrows) {
-            const int32_t ii = rho / G, hh = rho % G;
-            v = a.qbar[(static_cast<int64_t>(cb + i0 + ii) * a.hq + g * G + hh) * kHeadDim + c];
-        }
-        qs[c * RP + rho] = v;
+    if (warp == 4) {
+        tmem_alloc(&ss->tmem_base, 256);
+        tmem_relinquish();
     }
-    const int32_t tr = tid / 32;  // 4-row group
-    const int32_t tcg = tid % 32;  // 2-column group
-    for (int32_t kc0 = 0; kc0 < ncols; kc0 += kScoreKC) {
-        __syncthreads();
-        for (int32_t e = tid; e < kScoreKC * kHeadDim; e += nthr) {
-            const int32_t jj = e / kHeadDim, c = e % kHeadDim;
-            const int32_t j = kc0 + jj;
-            ks[c * (kScoreKC + 4) + jj] =
-                j < ncols ? a.kbar[(static_cast<int64_t>(cb + j) * a.hkv + g) * kHeadDim + c] : 0.f;
+    if (tid == 0) {
+        mbar_init(&ss->q_full, 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&ss->kv_full[s], 1);
+            mbar_init(&ss->kv_empty[s], 1);
+            mbar_init(&ss->acc_full[s], 1);
+            mbar_init(&ss->acc_empty[s], 128);
         }
-        __syncthreads();
-        float acc[4][2] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
-#pragma unroll 8
-        for (int32_t c = 0; c < kHeadDim; ++c) {
-            const float4 q4 = *reinterpret_cast<const float4*>(qs + c * RP + 4 * tr);
-            const float2 k2 = *reinterpret_cast<const float2*>(ks + c * (kScoreKC + 4) + 2 * tcg);
-            acc[0][0] = fmaf(q4.x, k2.x, acc[0][0]);
-            acc[0][1] = fmaf(q4.x, k2.y, acc[0][1]);
-            acc[1][0] = fmaf(q4.y, k2.x, acc[1][0]);
-            acc[1][1] = fmaf(q4.y, k2.y, acc[1][1]);
-            acc[2][0] = fmaf(q4.z, k2.x, acc[2][0]);
-            acc[2][1] = fmaf(q4.z, k2.y, acc[2][1]);
-            acc[3][0] = fmaf(q4.w, k2.x, acc[3][0]);
-            acc[3][1] = fmaf(q4.w, k2.y, acc[3][1]);
-        }
-#pragma unroll
-        for (int r = 0; r < 4; ++r)
-#pragma unroll
-            for (int cc = 0; cc < 2; ++cc) {
-                const int32_t j = kc0 + 2 * tcg + cc;
-                if (j < a.ncap) sc[(4 * tr + r) * a.ncap + j] = a.tau * acc[r][cc];
+        ss->abort = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = ss->tmem_base;
+
+    if (warp == 4) {
+        if (lane == 0) {
+            const int32_t qrow = (g * static_cast<int32_t>(a.max_blocks) + cb + i0) * G;
+            const int32_t krow = g * static_cast<int32_t>(a.max_blocks) + cb;
+            mbar_arrive_expect_tx(&ss->q_full, 2 * kTileQ);
+            for (int ch = 0; ch < 2; ++ch) {
+                tma_load_2d(qh + ch * 16384, &tqh, &ss->q_full, ch * 64, qrow);
+                tma_load_2d(ql + ch * 16384, &tql, &ss->q_full, ch * 64, qrow);
             }
-    }
-    __syncthreads();
-
-    const int32_t warp = tid / 32, lane = tid % 32, nwarps = nthr / 32;
-    for (int32_t rho = warp; rho < nrows; rho += nwarps) {
-        const int32_t i = i0 + rho / G;
-        float m = -INFINITY;
-        for (int32_t j = lane; j <= i; j += 32) m = fmaxf(m, sc[rho * a.ncap + j]);
+            auto load = [&](int32_t idx) -> bool {
+                const int32_t s = idx & 1;
+                if (!mbar_wait(&ss->kv_empty[s], ((idx >> 1) & 1) ^ 1, hdr, abort, 600000 + idx))
+                    return false;
+                const int32_t row = krow + (idx % nchunk) * 128;
+                mbar_arrive_expect_tx(&ss->kv_full[s], 2 * kTileQ);
+                for (int ch = 0; ch < 2; ++ch) {
+                    tma_load_2d(kh + s * kTileQ + ch * 16384, &tkh, &ss->kv_full[s], ch * 64, row);
+                    tma_load_2d(kl + s * kTileQ + ch * 16384, &tkl, &ss->kv_full[s], ch * 64, row);
+                }
+                return true;
+            };
+            bool ok = load(0) && mbar_wait(&ss->q_full, 0, hdr, abort, 610000);
+            const uint32_t idesc = idesc_make(kFmtBF16, 0, 128);
+            for (int32_t idx = 0; ok && idx < steps; ++idx) {
+                const int32_t s = idx & 1;
+                if (idx + 1 < steps && !(ok = load(idx + 1))) break;
+                if (!(ok = mbar_wait(&ss->kv_full[s], (idx >> 1) & 1, hdr, abort, 620000 + idx) &&
+                           mbar_wait(&ss->acc_empty[s], ((idx >> 1) & 1) ^ 1, hdr, abort, 630000 + idx)))
+                    break;
+                tc_fence_after();
+                const uint32_t d = tmem + s * 128;
+                const uint32_t ah = smem_u32(qh), al = smem_u32(ql);
+                const uint32_t bh = smem_u32(kh + s * kTileQ), bl = smem_u32(kl + s * kTileQ);
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-        if (lane == 0) rowmax[rho] = m;
-        if (a.score_dbg) {
-            const int32_t h = g * G + rho % G;
-            float* dst = a.score_dbg + (static_cast<int64_t>(cb + i) * a.hq + h) * a.nb_max;
-            for (int32_t j = lane; j <= i; j += 32) dst[j] = sc[rho * a.ncap + j] - m;
+                for (int k = 0; k < 8; ++k) mma_bf16_ss(d, score_desc(ah, k), score_desc(bh, k), idesc, k > 0);
+#pragma unroll
+                for (int k = 0; k < 8; ++k) mma_bf16_ss(d, score_desc(ah, k), score_desc(bl, k), idesc, 1);
+#pragma unroll
+                for (int k = 0; k < 8; ++k) mma_bf16_ss(d, score_desc(al, k), score_desc(bh, k), idesc, 1);
+                mma_commit(&ss->acc_full[s]);
+                mma_commit(&ss->kv_empty[s]);
+            }
+            // all loads consumed before the CTA exits
+            for (int32_t idx = max(0, steps - 2); ok && idx < steps; ++idx)
+                ok = mbar_wait(&ss->kv_empty[idx & 1], (idx >> 1) & 1, hdr, abort, 640000 + idx);
         }
-    }
-    __syncthreads();
-    for (int32_t ii = warp; ii < nqb; ii += nwarps) {
+    } else {
+        // ---- epilogue: row r of the tile ---------------------------------------
+        const int32_t r = tid;
+        const bool valid = r < nrows;
+        const int32_t ii = valid ? r / G : 0;
+        const int32_t hh = valid ? r % G : 0;
         const int32_t i = i0 + ii;
-        const int64_t row = static_cast<int64_t>(cb + i) * a.hkv + g;
-        int32_t* dst = a.kept_idx + row * a.nb_max;
-        int32_t base = 0;
-        for (int32_t j0 = 0; j0 <= i; j0 += 32) {
-            const int32_t j = j0 + lane;
-            bool keep = false;
-            if (j <= i) {
-                if (a.keep_all || j == i) {
-                    keep = true;
-                } else {
-                    for (int32_t hh = 0; hh < G; ++hh) {
-                        const int32_t rho = ii * G + hh;
-                        keep |= (sc[rho * a.ncap + j] - rowmax[rho]) >= a.ln_alpha;
+        const int32_t h = g * G + hh;
+        const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+        float m = -INFINITY;
+        int32_t cnt = 0;  // kept blocks of q-block i0 + r (thread r < nq owns it)
+        const int64_t own_row = static_cast<int64_t>(cb + i0 + r) * a.hkv + g;
+        // every epilogue thread runs all steps even after a failed wait (the
+        // waits then return at once): the named barriers below have no timeout,
+        // so all four warps must reach each of them
+        bool ok = true;
+        for (int32_t idx = 0; idx < steps; ++idx) {
+            const int32_t s = idx & 1;
+            const int32_t c = idx % nchunk;
+            const bool pass2 = idx >= nchunk;
+            ok = __all_sync(0xffffffffu, mbar_wait(&ss->acc_full[s], (idx >> 1) & 1, hdr, abort,
+                                                   650000 + idx)) && ok;
+            tc_fence_after();
+            uint32_t v[128];
+            const uint32_t addr = tmem + lane_off + s * 128;
+            tmem_ld32(addr + 0, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+            tmem_ld32(addr + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+            tmem_ld32(addr + 64, *reinterpret_cast<uint32_t(*)[32]>(&v[64]));
+            tmem_ld32(addr + 96, *reinterpret_cast<uint32_t(*)[32]>(&v[96]));
+            tmem_wait_ld();
+            tc_fence_before();
+            mbar_arrive(&ss->acc_empty[s]);
+            const int32_t j0 = c * 128;
+            if (!pass2) {
+#pragma unroll
+                for (int e = 0; e < 128; ++e)
+                    if (j0 + e <= i) m = fmaxf(m, __uint_as_float(v[e]) * a.tau);
+                continue;
+            }
+            uint32_t bits[4] = {0u, 0u, 0u, 0u};
+            if (valid) {
+                float* dbg = a.score_dbg
+                                 ? a.score_dbg + (static_cast<int64_t>(cb + i) * a.hq + h) * a.nb_max
+                                 : nullptr;
+#pragma unroll
+                for (int e = 0; e < 128; ++e) {
+                    const int32_t j = j0 + e;
+                    const float sv = __uint_as_float(v[e]) * a.tau;
+                    const bool keep = j <= i && (a.keep_all || j == i || sv - m >= a.ln_alpha);
+                    bits[e >> 5] |= keep ? (1u << (e & 31)) : 0u;
+                    if (dbg && j <= i) dbg[j] = sv - m;
+                }
+            }
+#pragma unroll
+            for (int w = 0; w < 4; ++w) ss->keep[r][w] = bits[w];
+            named_sync_epi();
+            if (ok && r < nq) {
+#pragma unroll
+                for (int w = 0; w < 4; ++w) {
+                    uint32_t u = 0;
+                    for (int32_t q = 0; q < G; ++q) u |= ss->keep[r * G + q][w];
+                    while (u) {
+                        const int bit = __ffs(u) - 1;
+                        u &= u - 1;
+                        a.kept_idx[own_row * a.nb_max + cnt++] = j0 + w * 32 + bit;
                     }
                 }
             }
-            const uint32_t mask = __ballot_sync(0xffffffffu, keep);
-            if (keep) dst[base + __popc(mask & ((1u << lane) - 1u))] = j;
-            base += __popc(mask);
+            named_sync_epi();
         }
-        if (lane == 0) a.kept_cnt[row] = base;
+        if (ok && r < nq) a.kept_cnt[own_row] = cnt;
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 4) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 256);
     }
 }
+
+size_t score_smem_bytes() { return 1024 + 6 * kTileQ + sizeof(ScoreSmem); }
 
 // ---------------------------------------------------------------------------
 // block means -> MMA operand precision

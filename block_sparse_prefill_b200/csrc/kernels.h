@@ -9,7 +9,7 @@
 namespace fp2 {
 
 constexpr int kPoolThreads = 512;  // 4 row groups x 128 column lanes
-constexpr int kScoreKC = 64;       // key blocks per shared-memory chunk in score_kernel
+constexpr int kScoreThreads = 160; // score_kernel: 4 epilogue warps + 1 TMA/MMA warp
 
 struct SetupArgs {
     const int32_t* cu;
@@ -30,7 +30,8 @@ struct SetupArgs {
 
 struct PoolArgs {
     const void* x[3];        // q, k, v (k/v may be page pools)
-    float* out[3];           // qbar, k_mean, v_mean
+    float* out[3];           // fp32 means (NULL = not written): -, k_mean, v_mean
+    uint16_t* split[2];      // bf16 hi/lo means of q (grouped rows) and k, see WsLayout
     const float* scale[3];   // per-head dequantisation scales (NULL = 1)
     int32_t heads[3];
     int32_t slabs[3];        // CTAs per block along the columns of each tensor
@@ -42,17 +43,19 @@ struct PoolArgs {
     const int32_t* block_table;
     int32_t max_blocks_per_seq;
     int32_t num_pages;
+    int32_t G;                 // query heads per KV head
+    int64_t max_blocks;        // row capacity of the split arrays
     WsHeader* hdr;
 };
 
 struct ScoreArgs {
-    const float* qbar;   // [max_blocks, Hq, d]
-    const float* kbar;   // [max_blocks, Hkv, d]
     const int32_t* cu_blocks;
     const int32_t* cu_tiles;
     int32_t batch;
     int32_t hq, hkv, G;
-    int32_t qt, rp, ncap, nb_max;
+    int32_t qt;          // q-blocks per tile: floor(128 / G)
+    int64_t max_blocks;  // row capacity of the split mean arrays
+    int32_t nb_max;
     float tau, ln_alpha;
     int32_t keep_all;
     int32_t* kept_cnt;
@@ -100,7 +103,12 @@ struct AttnArgs {
 __global__ void setup_kernel(SetupArgs a);
 template <bool kE4M3>
 __global__ void pool_kernel(PoolArgs a);
-__global__ void score_kernel(ScoreArgs a);
+__global__ void score_kernel(const __grid_constant__ ScoreArgs a,
+                             const __grid_constant__ CUtensorMap tqh,
+                             const __grid_constant__ CUtensorMap tql,
+                             const __grid_constant__ CUtensorMap tkh,
+                             const __grid_constant__ CUtensorMap tkl);
+size_t score_smem_bytes();
 __global__ void meanlp_kernel(MeanLpArgs a);
 
 // Shared-memory bytes of the attention kernel for a kept-list capacity.
