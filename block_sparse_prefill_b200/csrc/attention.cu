@@ -94,7 +94,9 @@ struct Bars {
     uint64_t o_done[2];
     uint64_t kv_full[8];
     uint64_t kv_empty[8];
-    uint64_t v_tail;      // V rows past the request end zeroed (partial diagonal block)
+    uint64_t v_tail[2];   // per metadata buffer: V rows past the request end zeroed
+                          // (partial diagonal block); per buffer so that a waiter can
+                          // never be two phases behind
     uint64_t meta_full[2];
     uint64_t meta_empty[2];
 };
@@ -239,7 +241,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&bars.kv_full[s], 1);
             mbar_init(&bars.kv_empty[s], 1);
         }
-        mbar_init(&bars.v_tail, 1);
+        mbar_init(&bars.v_tail[0], 1);
+        mbar_init(&bars.v_tail[1], 1);
         misc->abort = 0;
         fence_mbar_init();
     }
@@ -427,7 +430,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                     make_uint4(0u, 0u, 0u, 0u);
                         fence_proxy_async_smem();
                         __syncwarp();
-                        if (leader) mbar_arrive(&bars.v_tail);
+                        if (leader) mbar_arrive(&bars.v_tail[buf]);
                     }
                 }
             }
@@ -452,7 +455,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             auto phase = [](int32_t idx) { return static_cast<uint32_t>((idx / C::kSlots) & 1); };
             int32_t base = 0;          // ring entry of the current item's first K tile
             int32_t it[2] = {0, 0};    // PV iterations issued per Q tile
-            int32_t vt = 0;            // partial diagonal blocks seen
+            int32_t vt[2] = {0, 0};    // partial items seen per metadata buffer
             bool ok = true;
             for (int32_t k = 0; ok; ++k) {
                 const int32_t buf = k & 1;
@@ -477,8 +480,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (!(ok = mbar_wait(&bars.kv_full[slot(iv)], phase(iv), hdr, abort, 330000 + n)))
                         break;
                     if (n == 0 && partial) {
-                        if (!(ok = mbar_wait(&bars.v_tail, vt & 1, hdr, abort, 335000))) break;
-                        ++vt;
+                        if (!(ok = mbar_wait(&bars.v_tail[buf], vt[buf] & 1, hdr, abort, 335000))) break;
+                        ++vt[buf];
                     }
                     for (int qt = 0; qt < ntiles && ok; ++qt) {
                         if (!(ok = mbar_wait(&bars.p_full[qt], it[qt] & 1, hdr, abort, 340000 + n))) break;
