@@ -227,11 +227,16 @@ def time_e2e(st, wl, steps, dist_ctx):
 
 
 class DistCtx:
+    """One process per GPU: rank, world size and the two host-side collectives
+    the benchmark needs (a barrier around the timed region and the max of the
+    per-rank times).  Nothing on the data path is collective."""
+
     def __init__(self):
         self.world = int(os.environ.get("WORLD_SIZE", "1"))
         self.rank = int(os.environ.get("RANK", "0"))
         self.local_rank = int(os.environ.get("LOCAL_RANK", "0"))
         self.pg = None
+        self.backend = None
 
     def init(self, backend="nccl"):
         if self.world > 1:
@@ -239,23 +244,39 @@ class DistCtx:
             import torch.distributed as dist
             dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=600))
             self.pg = dist
+            self.backend = backend
 
     def barrier(self):
         if self.pg is not None:
-            import torch
-            self.pg.barrier(device_ids=[torch.cuda.current_device()])
+            if self.backend == "nccl":
+                import torch
+                self.pg.barrier(device_ids=[torch.cuda.current_device()])
+            else:
+                self.pg.barrier()
 
     def max(self, x: float) -> float:
         if self.pg is None:
             return x
         import torch
-        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        dev = "cuda" if self.backend == "nccl" else "cpu"
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
         self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
         return float(t.item())
 
     def close(self):
         if self.pg is not None:
             self.pg.destroy_process_group()
+            self.pg = None
+
+
+def rank_seed(rank: int) -> int:
+    """Each rank runs its own independent 128K layer (weak scaling)."""
+    return 1002 + rank
+
+
+def weak_scaling_value(world: int, flops_per_rank: float, ms_max: float) -> float:
+    """Whole-job TFLOP/s: the work of all ranks over the slowest rank's time."""
+    return world * flops_per_rank / (ms_max * 1e-3) / 1e12
 
 
 def cpu_baseline(wl, fracs=(0.25, 0.5)):
@@ -321,7 +342,7 @@ def ours(args):
     import block_sparse_prefill_b200 as fp2
     peaks, peaks_kind = load_peaks()
 
-    wl = make_config(2, seed=1002 + ctx.rank, seqlen=args.seqlen)
+    wl = make_config(2, seed=rank_seed(ctx.rank), seqlen=args.seqlen)
     st = setup_layer(wl, dev)
     clocks = Clocks(ctx.local_rank)
     total, est, att, clk = time_layer(st, wl, args.steps, args.warmup, ctx, clocks)
@@ -337,13 +358,13 @@ def ours(args):
     ms_step = ctx.max(total / args.steps)
     ms_est = statistics.mean(est)
     ms_att = statistics.mean(att)
-    value = ctx.world * flops / (ms_step * 1e-3) / 1e12
+    value = weak_scaling_value(ctx.world, flops, ms_step)
 
     e2e = None
     if not args.no_e2e:
         e2e_ms, h2d, d2h = time_e2e(st, wl, max(1, min(3, args.steps)), ctx)
         e2e_ms = ctx.max(e2e_ms)
-        e2e = {"value": ctx.world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
+        e2e = {"value": weak_scaling_value(ctx.world, flops, e2e_ms), "unit": "TFLOP/s", "ms_per_step": e2e_ms,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     # e4m3 variant of the same layer (config 3), kernel-timed
@@ -351,7 +372,7 @@ def ours(args):
     if not args.no_fp8:
         del st
         torch.cuda.empty_cache()
-        wl8 = make_config(3, seed=1002 + ctx.rank, seqlen=args.seqlen)
+        wl8 = make_config(3, seed=rank_seed(ctx.rank), seqlen=args.seqlen)
         st8 = setup_layer(wl8, dev)
         tot8, est8, att8, _ = time_layer(st8, wl8, args.steps, args.warmup, ctx)
         f8, c8 = layer_work(wl8.seqlens, st8["meta"].kept_cnt.cpu().numpy(), st8["meta"].kept_idx.cpu().numpy(),
@@ -362,7 +383,7 @@ def ours(args):
         fp8 = {
             "config": f"{wl8.max_seqlen // 1024}K e4m3 (Hq=32, Hkv=8, d=128, alpha=0.05)",
             "ms_per_layer": ms8, "ms_estimate": statistics.mean(est8), "ms_attention": a8,
-            "tflops_layer": ctx.world * f8 / (ms8 * 1e-3) / 1e12,
+            "tflops_layer": weak_scaling_value(ctx.world, f8, ms8),
             "tflops_attention": (f8 + c8) / (a8 * 1e-3) / 1e12,
             "tensor_peak_tflops": peak8,
             "frac_attention": (f8 + c8) / (a8 * 1e-3) / 1e12 / peak8,

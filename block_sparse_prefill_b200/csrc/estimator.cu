@@ -362,6 +362,10 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         }
     } else {
         // ---- epilogue: row r of the tile ---------------------------------------
+        // keep bit for key block j <= i: s - m >= ln(alpha), tested on the raw
+        // accumulator as acc >= (m + ln(alpha)) / tau (tau > 0).  The G rows of a
+        // q-block are G consecutive lanes when G divides 32 (warp shuffles OR
+        // them); otherwise they meet in shared memory.
         const int32_t r = tid;
         const bool valid = r < nrows;
         const int32_t ii = valid ? r / G : 0;
@@ -369,12 +373,13 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         const int32_t i = i0 + ii;
         const int32_t h = g * G + hh;
         const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+        const bool lanes_group = (32 % G) == 0;
         float m = -INFINITY;
-        int32_t cnt = 0;  // kept blocks of q-block i0 + r (thread r < nq owns it)
-        const int64_t own_row = static_cast<int64_t>(cb + i0 + r) * a.hkv + g;
-        // every epilogue thread runs all steps even after a failed wait (the
-        // waits then return at once): the named barriers below have no timeout,
-        // so all four warps must reach each of them
+        float thr_raw = 0.f;
+        int32_t cnt = 0;  // kept blocks of this q-block (group leader lane / owner thread)
+        const bool leader = lanes_group ? (valid && hh == 0) : (r < nq);
+        const int32_t lead_i = lanes_group ? i : i0 + r;
+        const int64_t own_row = static_cast<int64_t>(cb + (lead_i - i0) + i0) * a.hkv + g;
         bool ok = true;
         for (int32_t idx = 0; idx < steps; ++idx) {
             const int32_t s = idx & 1;
@@ -393,44 +398,85 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
             tc_fence_before();
             mbar_arrive(&ss->acc_empty[s]);
             const int32_t j0 = c * 128;
+            const bool full = j0 + 127 <= i;  // every column of the chunk is causal for this row
             if (!pass2) {
+                float mp[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+                if (full) {
 #pragma unroll
-                for (int e = 0; e < 128; ++e)
-                    if (j0 + e <= i) m = fmaxf(m, __uint_as_float(v[e]) * a.tau);
+                    for (int e = 0; e < 128; ++e) mp[e & 3] = fmaxf(mp[e & 3], __uint_as_float(v[e]));
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 128; ++e)
+                        if (j0 + e <= i) mp[e & 3] = fmaxf(mp[e & 3], __uint_as_float(v[e]));
+                }
+                m = fmaxf(m, fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])));
+                if (idx == nchunk - 1) {
+                    m *= a.tau;                       // row max of s
+                    thr_raw = (m + a.ln_alpha) / a.tau;
+                }
                 continue;
             }
             uint32_t bits[4] = {0u, 0u, 0u, 0u};
             if (valid) {
-                float* dbg = a.score_dbg
-                                 ? a.score_dbg + (static_cast<int64_t>(cb + i) * a.hq + h) * a.nb_max
-                                 : nullptr;
+                if (a.keep_all) {
 #pragma unroll
-                for (int e = 0; e < 128; ++e) {
-                    const int32_t j = j0 + e;
-                    const float sv = __uint_as_float(v[e]) * a.tau;
-                    const bool keep = j <= i && (a.keep_all || j == i || sv - m >= a.ln_alpha);
-                    bits[e >> 5] |= keep ? (1u << (e & 31)) : 0u;
-                    if (dbg && j <= i) dbg[j] = sv - m;
+                    for (int w = 0; w < 4; ++w) {
+                        const int32_t lim = i - (j0 + 32 * w);   // keep j <= i
+                        bits[w] = lim >= 31 ? 0xffffffffu : (lim < 0 ? 0u : ((2u << lim) - 1u));
+                    }
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 128; ++e)
+                        bits[e >> 5] |= (__uint_as_float(v[e]) >= thr_raw) ? (1u << (e & 31)) : 0u;
+                    if (!full) {
+#pragma unroll
+                        for (int w = 0; w < 4; ++w) {
+                            const int32_t lim = i - (j0 + 32 * w);
+                            bits[w] &= lim >= 31 ? 0xffffffffu : (lim < 0 ? 0u : ((2u << lim) - 1u));
+                        }
+                    }
+                    if (i >= j0 && i < j0 + 128) bits[(i - j0) >> 5] |= 1u << ((i - j0) & 31);  // diagonal
+                }
+                if (a.score_dbg) {
+                    float* dbg = a.score_dbg + (static_cast<int64_t>(cb + i) * a.hq + h) * a.nb_max;
+#pragma unroll
+                    for (int e = 0; e < 128; ++e)
+                        if (j0 + e <= i) dbg[j0 + e] = __uint_as_float(v[e]) * a.tau - m;
                 }
             }
-#pragma unroll
-            for (int w = 0; w < 4; ++w) ss->keep[r][w] = bits[w];
-            named_sync_epi();
-            if (ok && r < nq) {
+            uint32_t u[4];
+            if (lanes_group) {
 #pragma unroll
                 for (int w = 0; w < 4; ++w) {
-                    uint32_t u = 0;
-                    for (int32_t q = 0; q < G; ++q) u |= ss->keep[r * G + q][w];
-                    while (u) {
-                        const int bit = __ffs(u) - 1;
-                        u &= u - 1;
-                        a.kept_idx[own_row * a.nb_max + cnt++] = j0 + w * 32 + bit;
+                    u[w] = bits[w];
+                    for (int o = 1; o < G; o <<= 1) u[w] |= __shfl_xor_sync(0xffffffffu, u[w], o);
+                }
+            } else {
+#pragma unroll
+                for (int w = 0; w < 4; ++w) ss->keep[r][w] = bits[w];
+                named_sync_epi();
+#pragma unroll
+                for (int w = 0; w < 4; ++w) {
+                    u[w] = 0;
+                    if (r < nq)
+                        for (int32_t q = 0; q < G; ++q) u[w] |= ss->keep[r * G + q][w];
+                }
+                named_sync_epi();
+            }
+            if (ok && leader) {
+                int32_t* dst = a.kept_idx + own_row * a.nb_max;
+#pragma unroll
+                for (int w = 0; w < 4; ++w) {
+                    uint32_t x = u[w];
+                    while (x) {
+                        const int bit = __ffs(x) - 1;
+                        x &= x - 1;
+                        dst[cnt++] = j0 + w * 32 + bit;
                     }
                 }
             }
-            named_sync_epi();
         }
-        if (ok && r < nq) a.kept_cnt[own_row] = cnt;
+        if (ok && leader) a.kept_cnt[own_row] = cnt;
     }
     tc_fence_before();
     __syncthreads();
