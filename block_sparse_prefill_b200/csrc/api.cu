@@ -54,6 +54,23 @@ bool make_map(CUtensorMap* m, const void* base, bool e4m3, int64_t heads, int64_
 }
 
 // 2-D bf16 map over [rows, 128] with 128-byte-swizzled boxes of 128 rows x 64 columns.
+// [rows, heads, d] without swizzle, box of 32 rows x hb heads x d (the pooling stages).
+bool make_map_pool(CUtensorMap* m, const void* base, bool e4m3, int64_t heads, int64_t rows,
+                   int32_t hb) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    const cuuint64_t esz = e4m3 ? 1 : 2;
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kHeadDim), static_cast<cuuint64_t>(heads),
+                                static_cast<cuuint64_t>(rows > 0 ? rows : 1)};
+    const cuuint64_t strides[2] = {kHeadDim * esz, kHeadDim * esz * static_cast<cuuint64_t>(heads)};
+    const cuuint32_t box[3] = {static_cast<cuuint32_t>(kHeadDim), static_cast<cuuint32_t>(hb), 32};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, e4m3 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+               const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool make_map_2d(CUtensorMap* m, const void* base, int64_t rows) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return false;
@@ -183,9 +200,6 @@ fp2_status run_estimate(const fp2_params* p, const void* q, const void* k, const
     WsHeader* hdr = at<WsHeader>(ws, 0);
     PoolArgs pa;
     memset(&pa, 0, sizeof(pa));
-    pa.x[0] = q;
-    pa.x[1] = k;
-    pa.x[2] = v;
     pa.out[0] = nullptr;
     pa.out[1] = meta->k_mean;
     pa.out[2] = meta->v_mean;
@@ -199,11 +213,16 @@ fp2_status run_estimate(const fp2_params* p, const void* q, const void* k, const
     pa.heads[0] = p->num_q_heads;
     pa.heads[1] = p->num_kv_heads;
     pa.heads[2] = p->num_kv_heads;
-    const int32_t per_cta = 128 * (e4m3 ? 16 : 8);
-    for (int x = 0; x < 3; ++x) pa.slabs[x] = (pa.heads[x] * kHeadDim + per_cta - 1) / per_cta;
+    // a slab is at most 2 KB of a row (8 bf16 or 16 e4m3 heads): 32 rows = one 64 KB stage
+    const int32_t hb_max = e4m3 ? 16 : 8;
+    for (int x = 0; x < 3; ++x) {
+        pa.hb[x] = pa.heads[x] < hb_max ? pa.heads[x] : hb_max;
+        pa.slabs[x] = (pa.heads[x] + pa.hb[x] - 1) / pa.hb[x];
+    }
     pa.paged[0] = 0;
     pa.paged[1] = pa.paged[2] = block_table ? 1 : 0;
-    pa.ntensors = meta->v_mean ? 3 : 2;
+    pa.first = 0;
+    pa.last = meta->v_mean ? 3 : 2;
     pa.cu = cu;
     pa.cu_blocks = at<int32_t>(ws, pr.ws.cu_blocks);
     pa.blk_req = at<int32_t>(ws, pr.ws.blk_req);
@@ -211,12 +230,29 @@ fp2_status run_estimate(const fp2_params* p, const void* q, const void* k, const
     pa.max_blocks_per_seq = mbps;
     pa.num_pages = num_pages;
     pa.hdr = hdr;
-    const int32_t ys = pa.slabs[0] + pa.slabs[1] + (pa.ntensors == 3 ? pa.slabs[2] : 0);
-    dim3 pgrid(static_cast<unsigned>(pr.max_blocks), static_cast<unsigned>(ys));
+    const int32_t ys = pa.slabs[0] + pa.slabs[1] + (pa.last == 3 ? pa.slabs[2] : 0);
+    const int64_t kv_rows = block_table ? int64_t(num_pages) * kBlock : pr.total_tokens;
+    CUtensorMap pq, pk, pv;
+    if (!make_map_pool(&pq, q, e4m3, p->num_q_heads, pr.total_tokens, pa.hb[0]) ||
+        !make_map_pool(&pk, k, e4m3, p->num_kv_heads, kv_rows, pa.hb[1]) ||
+        !make_map_pool(&pv, v, e4m3, p->num_kv_heads, kv_rows, pa.hb[2]))
+        return FP2_ERR_CUDA;
+    // persistent: one CTA per SM (the stage ring fills most of shared memory)
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return FP2_ERR_CUDA;
+    const int64_t units = pr.max_blocks * ys;
+    const unsigned pgrid = static_cast<unsigned>(units < sms ? units : sms);
+    const size_t psmem = pool_smem_bytes(e4m3);
+    if (cudaFuncSetAttribute(e4m3 ? pool_kernel<true> : pool_kernel<false>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(psmem)) != cudaSuccess)
+        return FP2_ERR_CUDA;
     if (e4m3)
-        pool_kernel<true><<<pgrid, kPoolThreads, 0, s>>>(pa);
+        pool_kernel<true><<<pgrid, kPoolThreads, psmem, s>>>(pa, pq, pk, pv);
     else
-        pool_kernel<false><<<pgrid, kPoolThreads, 0, s>>>(pa);
+        pool_kernel<false><<<pgrid, kPoolThreads, psmem, s>>>(pa, pq, pk, pv);
     if ((st = launched(cudaGetLastError())) != FP2_OK) return st;
 
     ScoreArgs sa;
@@ -249,7 +285,8 @@ fp2_status run_estimate(const fp2_params* p, const void* q, const void* k, const
                              static_cast<int>(smem)) != cudaSuccess)
         return FP2_ERR_CUDA;
     const int64_t tiles = (pr.max_blocks + qt - 1) / qt + pr.batch;
-    score_kernel<<<dim3(static_cast<unsigned>(tiles), static_cast<unsigned>(p->num_kv_heads)),
+    if (tiles > 65535) return FP2_ERR_UNSUPPORTED;
+    score_kernel<<<dim3(static_cast<unsigned>(p->num_kv_heads), static_cast<unsigned>(tiles)),
                    kScoreThreads, smem, s>>>(sa, tqh, tql, tkh, tkl);
     return launched(cudaGetLastError());
 }

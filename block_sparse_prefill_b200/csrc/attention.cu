@@ -19,7 +19,9 @@
 //                            tiles into a ring of shared-memory slots, following
 //                            the kept list and, in paged mode, the block table
 //                warp 9      TMEM owner and MMA issuer
-//                warps 10-11 idle (they only donate registers)
+//                warp 10     scheduler: takes work items from a global counter and
+//                            prepares their kept lists in shared memory
+//                warp 11     idle (it only donates registers)
 // The softmax warpgroups raise their register budget (setmaxnreg) so that a
 // whole 128-column row of S stays in registers; warpgroup 2 lowers its own.
 //
@@ -50,13 +52,15 @@ constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr int kSchedWarp = 10;
 // When > 0, every kEmuEvery-th pair of attention weights is exponentiated on
-// the FMA pipe (exp2_poly2) instead of MUFU.  Measured on B200 at 128K (bf16,
-// attention call): off 4.77 ms, 1/8 4.77 ms, 1/4 5.08 ms, 1/2 5.90 ms -- the
-// softmax is bound by instruction issue, not by MUFU, so it is off.
-#ifndef FP2_EXP_EMU_EVERY
-#define FP2_EXP_EMU_EVERY 0
+// the FMA pipe (exp2_poly2) instead of MUFU (per dtype).  Measured on B200 at
+// 128K (bf16, attention call): off 4.77 ms, 1/8 4.77 ms, 1/4 5.08 ms, 1/2
+// 5.90 ms -- the bf16 softmax is bound by instruction issue, not by MUFU.
+#ifndef FP2_EXP_EMU_BF16
+#define FP2_EXP_EMU_BF16 0
 #endif
-constexpr int kEmuEvery = FP2_EXP_EMU_EVERY;
+#ifndef FP2_EXP_EMU_E4M3
+#define FP2_EXP_EMU_E4M3 0
+#endif
 constexpr uint32_t kTmemCols = 512;
 // Registers per thread after the split.  setmaxnreg only redistributes the
 // registers the CTA was launched with (384 threads x 168 = 64512), so
@@ -84,6 +88,7 @@ struct Cfg {
     // bf16: no offset, and O is rescaled only for jumps above 2^8.
     static constexpr float kPOffset = kE4M3 ? 8.f : 0.f;
     static constexpr float kRescale = kE4M3 ? 0.75f : 8.f;
+    static constexpr int kEmuEvery = kE4M3 ? FP2_EXP_EMU_E4M3 : FP2_EXP_EMU_BF16;
 };
 
 struct Bars {
@@ -91,7 +96,7 @@ struct Bars {
     uint64_t q_empty;     // the last S MMA of a work item has read Q
     uint64_t s_full[2];
     uint64_t p_full[2];
-    uint64_t o_done[2];
+    uint64_t o_done[2];   // the last PV of Q tile t in a work item has finished
     uint64_t kv_full[8];
     uint64_t kv_empty[8];
     uint64_t v_tail[2];   // per metadata buffer: V rows past the request end zeroed
@@ -489,7 +494,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tc_fence_after();
                         issue_pv<kE4M3>(tmem + 256 + qt * 128, tmem + qt * 128,
                                         kv_addr + slot(iv) * C::kTileBytes, n == 0);
-                        mma_commit(&bars.o_done[qt]);
+                        // O_t is complete after the item's last PV.  Within the
+                        // item no O-done signal is needed: S_t(n+1) is issued after
+                        // PV_t(n), and a commit tracks every earlier MMA, so the
+                        // softmax's S-ready wait also covers PV_t(n).  (Each commit
+                        // costs tensor-pipe time.)
+                        if (!next) mma_commit(&bars.o_done[qt]);
                         if (next) {
                             if (qt == 0 && !(ok = mbar_wait(&bars.kv_full[slot(ik)], phase(ik), hdr,
                                                             abort, 310000 + n)))
@@ -519,7 +529,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
         const uint32_t s_addr = tmem + lane_off + qt * 128;
         const uint32_t o_addr = tmem + lane_off + 256 + qt * 128;
-        int32_t it = 0;  // iterations of this Q tile so far (barrier phases)
+        int32_t it = 0;     // tile steps of this Q tile so far (s_full phases)
+        int32_t items = 0;  // work items of this Q tile so far (o_done phases)
         bool ok = true;
         for (int32_t k = 0; ok; ++k) {
             const int32_t buf = k & 1;
@@ -586,9 +597,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (__any_sync(0xffffffffu, need)) {
                     const float f = need ? ex2(m_ref - m_new) : 1.f;
                     if (n > 0) {
-                        if (!(ok = warp_wait(&bars.o_done[qt], (it - 1) & 1, hdr, abort, 410000 + n)))
-                            break;
-                        tc_fence_after();
+                        // PV_t(n-1) has finished: S_t(n) was issued after it
 #pragma unroll
                         for (int c0 = 0; c0 < 128; c0 += 32) {
                             uint32_t ov[32];
@@ -617,7 +626,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int c = 0; c < 128; c += 2) {
                     float2 x = ffma2(make_float2(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])),
                                      make_float2(qk, qk), make_float2(neg, neg));
-                    if (kEmuEvery > 0 && ((c >> 1) % (kEmuEvery > 0 ? kEmuEvery : 1)) == kEmuEvery - 1) {
+                    if (C::kEmuEvery > 0 &&
+                        ((c >> 1) % (C::kEmuEvery > 0 ? C::kEmuEvery : 1)) == C::kEmuEvery - 1) {
                         x = exp2_poly2(x);
                     } else {
                         x.x = ex2(x.x);
@@ -661,7 +671,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ++it;
             }
             // ---- epilogue: O / l -> bf16 ------------------------------------
-            if (ok && ntot > 0 && (ok = warp_wait(&bars.o_done[qt], (it - 1) & 1, hdr, abort, 420000))) {
+            if (ok && ntot > 0 && (ok = warp_wait(&bars.o_done[qt], (items++) & 1, hdr, abort, 420000))) {
                 tc_fence_after();
                 float inv = 1.f / l;
                 if (kE4M3) inv *= a.v_scale[g];

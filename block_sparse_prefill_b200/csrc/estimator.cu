@@ -7,7 +7,7 @@
 //
 //   setup_kernel   validates cu_seqlens, numbers the blocks of the ragged batch
 //   pool_kernel    block means of Q, K, V (HBM-bound streaming pass, every input
-//                  byte read once with 16-byte loads)
+//                  byte read once, TMA into a ring of shared-memory stages)
 //   score_kernel   s = tau * qbar . kbar for the causal block pairs of a tile of
 //                  q-blocks (fp32 FMA from shared memory), per-head row max,
 //                  exp(s - m) >= alpha threshold, union over the G query heads of
@@ -62,10 +62,37 @@ __global__ void setup_kernel(SetupArgs a) {
     __syncthreads();
     // order: blocks sorted by their index in the request, largest first (the
     // causal kept lists grow with it), so the persistent attention kernel
-    // takes the longest work items first
-    if (threadIdx.x == 0) {
-        int32_t run = 0;
-        for (int32_t j = a.nb_cap - 1; j >= 0; --j) {
+    // takes the longest work items first.  Exclusive scan of the histogram in
+    // descending index order: each thread scans a contiguous run of bins, the
+    // runs' totals are scanned across the block.
+    {
+        __shared__ int32_t wsum[32];
+        const int32_t tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+        const int32_t nwarps = (blockDim.x + 31) >> 5;
+        const int32_t per = (a.nb_cap + blockDim.x - 1) / blockDim.x;
+        const int32_t p0 = min(a.nb_cap, tid * per), p1 = min(a.nb_cap, p0 + per);
+        int32_t local = 0;
+        for (int32_t p = p0; p < p1; ++p) local += hist[a.nb_cap - 1 - p];
+        int32_t incl = local;
+        for (int32_t o = 1; o < 32; o <<= 1) {
+            const int32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        if (lane == 31) wsum[warp] = incl;
+        __syncthreads();
+        if (warp == 0) {
+            const int32_t v = lane < nwarps ? wsum[lane] : 0;
+            int32_t vi = v;
+            for (int32_t o = 1; o < 32; o <<= 1) {
+                const int32_t y = __shfl_up_sync(0xffffffffu, vi, o);
+                if (lane >= o) vi += y;
+            }
+            wsum[lane] = vi - v;
+        }
+        __syncthreads();
+        int32_t run = wsum[warp] + incl - local;
+        for (int32_t p = p0; p < p1; ++p) {
+            const int32_t j = a.nb_cap - 1 - p;
             const int32_t c = hist[j];
             hist[j] = run;
             run += c;
@@ -79,14 +106,53 @@ __global__ void setup_kernel(SetupArgs a) {
 
 // ---------------------------------------------------------------------------
 // pooling: mean over the valid rows of every block, per column
+//
+// Persistent: one CTA per SM walks the units (block t, column slab y of
+// tensor x).  A producer warp streams each unit's rows into a ring of
+// shared-memory stages with TMA (32 rows of one slab, up to 64 KB per stage),
+// so the bytes in flight per SM do not depend on the consumers' registers.
+// 16 consumer warps (4 row groups x 128 lanes of 16 bytes) accumulate in fp32
+// and, after the unit's last stage, reduce the row groups through shared
+// memory.  Rows past a request's end are loaded (or zero-filled past the
+// tensor) but not summed; pages are checked against the pool size.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ uint4 ld_stream16(const void* p) {
-    uint4 r;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-                 : "l"(p));
-    return r;
+namespace {
+constexpr int kPoolStages = 3;
+constexpr int kPoolStageRows = 32;
+constexpr int kPoolStageBytes = 65536;
+constexpr int kPoolConsumers = kPoolThreads - 32;
+static_assert(kPoolConsumers == 512, "4 row groups x 128 column lanes");
+
+struct PoolSmem {
+    uint64_t full[kPoolStages];
+    uint64_t empty[kPoolStages];
+    int32_t abort;
+};
+
+struct PoolUnit {
+    int32_t x, y, t, b, j, n;
+};
+
+// unit u -> (tensor, slab, block, request, block index in the request, valid rows)
+__device__ __forceinline__ PoolUnit pool_unit(const PoolArgs& a, int32_t u, int32_t ys) {
+    PoolUnit p;
+    p.t = u / ys;
+    p.y = u % ys;
+    p.x = a.first;
+    while (p.x < a.last - 1 && p.y >= a.slabs[p.x]) {
+        p.y -= a.slabs[p.x];
+        ++p.x;
+    }
+    p.b = a.blk_req[p.t];
+    p.j = p.t - a.cu_blocks[p.b];
+    p.n = min(kBlock, a.cu[p.b + 1] - a.cu[p.b] - p.j * kBlock);
+    return p;
 }
+
+__device__ __forceinline__ void named_sync_pool() {
+    asm volatile("bar.sync 1, %0;" ::"n"(kPoolConsumers) : "memory");
+}
+}  // namespace
 
 template <bool kE4M3>
 struct PoolVec;
@@ -123,103 +189,158 @@ struct PoolVec<true> {  // 16 e4m3 per 16 bytes
     }
 };
 
+size_t pool_smem_bytes(bool e4m3) {
+    const int n = e4m3 ? 16 : 8;
+    return 1024 + static_cast<size_t>(kPoolStages) * kPoolStageBytes +
+           sizeof(float) * 3 * 128 * (n + 1) + sizeof(PoolSmem);
+}
+
 template <bool kE4M3>
-__global__ void __launch_bounds__(kPoolThreads) pool_kernel(PoolArgs a) {
+__global__ void __launch_bounds__(kPoolThreads, 1)
+    pool_kernel(const __grid_constant__ PoolArgs a, const __grid_constant__ CUtensorMap tq,
+                const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv) {
     using V = PoolVec<kE4M3>;
     constexpr int N = V::N;
-    constexpr int kRowGroups = kPoolThreads / 128;
-    __shared__ float red[kRowGroups - 1][128][N + 1];
-
-    const int32_t t = blockIdx.x;
-    if (!a.hdr->valid || t >= a.hdr->total_blocks) return;
-    // which tensor / column slab
-    int32_t y = blockIdx.y, x = 0;
-    while (x < 2 && y >= a.slabs[x]) { y -= a.slabs[x]; ++x; }
-    if (x >= a.ntensors) return;
-    const int32_t b = a.blk_req[t];
-    const int32_t j = t - a.cu_blocks[b];
-    const int32_t L = a.cu[b + 1] - a.cu[b];
-    const int32_t n = min(kBlock, L - j * kBlock);
-    const int32_t ncols = a.heads[x] * kHeadDim;
-    const int32_t tc = threadIdx.x & 127;
-    const int32_t rg = threadIdx.x >> 7;
-    const int32_t col = (y * 128 + tc) * N;
-    const bool active = col < ncols;
-
-    int64_t row0;
-    if (a.paged[x]) {
-        int32_t page = a.block_table[static_cast<int64_t>(b) * a.max_blocks_per_seq + j];
-        if (page < 0 || page >= a.num_pages) {
-            if (threadIdx.x == 0) set_error(a.hdr, FP2_ERR_BAD_INDEX, t);
-            page = 0;
+    constexpr int kEsz = kE4M3 ? 1 : 2;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* stages = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                 ~uintptr_t(1023));
+    float(*red)[128][N + 1] =
+        reinterpret_cast<float(*)[128][N + 1]>(stages + kPoolStages * kPoolStageBytes);
+    PoolSmem* ps = reinterpret_cast<PoolSmem*>(stages + kPoolStages * kPoolStageBytes +
+                                               sizeof(float) * 3 * 128 * (N + 1));
+    volatile int32_t* abort = &ps->abort;
+    WsHeader* hdr = a.hdr;
+    if (!hdr->valid) return;
+    int32_t ys = 0;
+    for (int x = a.first; x < a.last; ++x) ys += a.slabs[x];
+    const int32_t units = hdr->total_blocks * ys;
+    const int32_t tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    if (tid == 0) {
+        for (int st = 0; st < kPoolStages; ++st) {
+            mbar_init(&ps->full[st], 1);
+            mbar_init(&ps->empty[st], kPoolConsumers / 32);
         }
-        row0 = static_cast<int64_t>(page) * kBlock;
-    } else {
-        row0 = a.cu[b] + static_cast<int64_t>(j) * kBlock;
-    }
-
-    float acc[N];
-#pragma unroll
-    for (int e = 0; e < N; ++e) acc[e] = 0.f;
-    if (active) {
-        const char* base = static_cast<const char*>(a.x[x]) +
-                           (row0 * ncols + col) * static_cast<int64_t>(kE4M3 ? 1 : 2);
-        const int64_t rstride = static_cast<int64_t>(ncols) * (kE4M3 ? 1 : 2);
-        int32_t r = rg;
-        for (; r + 7 * kRowGroups < n; r += 8 * kRowGroups) {
-            uint4 v[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) v[u] = ld_stream16(base + (r + u * kRowGroups) * rstride);
-#pragma unroll
-            for (int u = 0; u < 8; ++u) V::add(acc, v[u]);
-        }
-        for (; r < n; r += kRowGroups) V::add(acc, ld_stream16(base + r * rstride));
-    }
-    if (rg > 0) {
-#pragma unroll
-        for (int e = 0; e < N; ++e) red[rg - 1][tc][e] = acc[e];
+        ps->abort = 0;
+        fence_mbar_init();
     }
     __syncthreads();
-    if (rg == 0 && active) {
-#pragma unroll
-        for (int g = 0; g < kRowGroups - 1; ++g)
-#pragma unroll
-            for (int e = 0; e < N; ++e) acc[e] += red[g][tc][e];
-        const int32_t h = col / kHeadDim;
-        const float s = (a.scale[x] ? a.scale[x][h] : 1.f) / static_cast<float>(n);
-#pragma unroll
-        for (int e = 0; e < N; ++e) acc[e] *= s;
-        if (a.out[x]) {
-            float* out = a.out[x] + static_cast<int64_t>(t) * ncols + col;
-#pragma unroll
-            for (int e = 0; e < N; e += 4)
-                *reinterpret_cast<float4*>(out + e) = make_float4(acc[e], acc[e + 1], acc[e + 2], acc[e + 3]);
+
+    if (warp == kPoolConsumers / 32) {
+        // ---- producer ---------------------------------------------------------
+        if (lane == 0) {
+            const CUtensorMap* maps[3] = {&tq, &tk, &tv};
+            int32_t cnt = 0;
+            bool ok = true;
+            for (int32_t u = blockIdx.x; ok && u < units; u += gridDim.x) {
+                const PoolUnit p = pool_unit(a, u, ys);
+                int64_t row0;
+                if (a.paged[p.x]) {
+                    int32_t page = a.block_table[static_cast<int64_t>(p.b) * a.max_blocks_per_seq + p.j];
+                    if (page < 0 || page >= a.num_pages) {
+                        set_error(hdr, FP2_ERR_BAD_INDEX, p.t);
+                        page = 0;
+                    }
+                    row0 = static_cast<int64_t>(page) * kBlock;
+                } else {
+                    row0 = a.cu[p.b] + static_cast<int64_t>(p.j) * kBlock;
+                }
+                const uint32_t bytes = static_cast<uint32_t>(a.hb[p.x]) * kHeadDim * kEsz * kPoolStageRows;
+                const int32_t nsub = (p.n + kPoolStageRows - 1) / kPoolStageRows;
+                for (int32_t sub = 0; sub < nsub; ++sub, ++cnt) {
+                    const int32_t st = cnt % kPoolStages;
+                    if (!(ok = mbar_wait(&ps->empty[st], ((cnt / kPoolStages) & 1) ^ 1, hdr, abort,
+                                         700000 + sub)))
+                        break;
+                    mbar_arrive_expect_tx(&ps->full[st], bytes);
+                    tma_load_3d(stages + st * kPoolStageBytes, maps[p.x], &ps->full[st], 0,
+                                p.y * a.hb[p.x], static_cast<int32_t>(row0 + sub * kPoolStageRows));
+                }
+            }
         }
-        if (x < 2) {
-            // hi + lo bf16 parts for the score MMAs: hi = bf16(m), lo = bf16(m - hi)
-            int64_t row;
-            if (x == 0) {
-                const int32_t g = h / a.G, hh = h % a.G;
-                row = (static_cast<int64_t>(g) * a.max_blocks + t) * a.G + hh;
-            } else {
-                row = static_cast<int64_t>(h) * a.max_blocks + t;
-            }
-            const int64_t plane = (x == 0 ? static_cast<int64_t>(a.heads[0]) : a.heads[1]) * a.max_blocks * kHeadDim;
-            uint16_t* hi = a.split[x] + row * kHeadDim + (col % kHeadDim);
-            uint16_t* lo = hi + plane;
-            uint32_t ph[N / 2], pl[N / 2];
+    } else {
+        // ---- consumers: thread (row group rg, 16-byte column lane tc) -----------
+        const int32_t tc = tid & 127;
+        const int32_t rg = tid >> 7;
+        int32_t cnt = 0;
+        bool ok = true;
+        for (int32_t u = blockIdx.x; u < units; u += gridDim.x) {
+            const PoolUnit p = pool_unit(a, u, ys);
+            const int32_t x = p.x;
+            const int32_t row_bytes = a.hb[x] * kHeadDim * kEsz;   // one row of the slab
+            const int32_t ncols = a.heads[x] * kHeadDim;
+            const int32_t col = p.y * a.hb[x] * kHeadDim + tc * N;
+            const bool active = tc * 16 < row_bytes && col < ncols;
+            float acc[N];
 #pragma unroll
-            for (int e = 0; e < N; e += 2) {
-                const uint32_t hp = pack_bf16(acc[e], acc[e + 1]);
-                const float h0 = __uint_as_float(hp << 16), h1 = __uint_as_float(hp & 0xFFFF0000u);
-                ph[e / 2] = hp;
-                pl[e / 2] = pack_bf16(acc[e] - h0, acc[e + 1] - h1);
+            for (int e = 0; e < N; ++e) acc[e] = 0.f;
+            const int32_t nsub = (p.n + kPoolStageRows - 1) / kPoolStageRows;
+            for (int32_t sub = 0; sub < nsub; ++sub, ++cnt) {
+                const int32_t st = cnt % kPoolStages;
+                // after a failed wait nothing more is read, but every consumer
+                // still passes the same named barriers
+                if (ok) ok = mbar_wait(&ps->full[st], (cnt / kPoolStages) & 1, hdr, abort, 710000 + sub);
+                if (ok && active) {
+                    const uint8_t* base = stages + st * kPoolStageBytes + tc * 16;
+                    const int32_t nr = min(kPoolStageRows, p.n - sub * kPoolStageRows);
+#pragma unroll 4
+                    for (int32_t rr = rg; rr < nr; rr += 4)
+                        V::add(acc, *reinterpret_cast<const uint4*>(base + rr * row_bytes));
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&ps->empty[st]);
             }
+            if (rg > 0) {
 #pragma unroll
-            for (int e = 0; e < N / 2; e += 4) {
-                *reinterpret_cast<uint4*>(hi + 2 * e) = make_uint4(ph[e], ph[e + 1], ph[e + 2], ph[e + 3]);
-                *reinterpret_cast<uint4*>(lo + 2 * e) = make_uint4(pl[e], pl[e + 1], pl[e + 2], pl[e + 3]);
+                for (int e = 0; e < N; ++e) red[rg - 1][tc][e] = acc[e];
             }
+            named_sync_pool();
+            if (rg == 0 && active && ok) {
+#pragma unroll
+                for (int g = 0; g < 3; ++g)
+#pragma unroll
+                    for (int e = 0; e < N; ++e) acc[e] += red[g][tc][e];
+                const int32_t h = col / kHeadDim;
+                const float sc = (a.scale[x] ? a.scale[x][h] : 1.f) / static_cast<float>(p.n);
+#pragma unroll
+                for (int e = 0; e < N; ++e) acc[e] *= sc;
+                const int32_t t = p.t;
+                if (a.out[x]) {
+                    float* out = a.out[x] + static_cast<int64_t>(t) * ncols + col;
+#pragma unroll
+                    for (int e = 0; e < N; e += 4)
+                        *reinterpret_cast<float4*>(out + e) =
+                            make_float4(acc[e], acc[e + 1], acc[e + 2], acc[e + 3]);
+                }
+                if (x < 2) {
+                    // hi + lo bf16 parts for the score MMAs: hi = bf16(m), lo = bf16(m - hi)
+                    int64_t row;
+                    if (x == 0) {
+                        const int32_t g = h / a.G, hh = h % a.G;
+                        row = (static_cast<int64_t>(g) * a.max_blocks + t) * a.G + hh;
+                    } else {
+                        row = static_cast<int64_t>(h) * a.max_blocks + t;
+                    }
+                    const int64_t plane =
+                        static_cast<int64_t>(a.heads[x]) * a.max_blocks * kHeadDim;
+                    uint16_t* hi = a.split[x] + row * kHeadDim + (col % kHeadDim);
+                    uint16_t* lo = hi + plane;
+                    uint32_t ph[N / 2], pl[N / 2];
+#pragma unroll
+                    for (int e = 0; e < N; e += 2) {
+                        const uint32_t hp = pack_bf16(acc[e], acc[e + 1]);
+                        const float h0 = __uint_as_float(hp << 16), h1 = __uint_as_float(hp & 0xFFFF0000u);
+                        ph[e / 2] = hp;
+                        pl[e / 2] = pack_bf16(acc[e] - h0, acc[e + 1] - h1);
+                    }
+#pragma unroll
+                    for (int e = 0; e < N / 2; e += 4) {
+                        *reinterpret_cast<uint4*>(hi + 2 * e) = make_uint4(ph[e], ph[e + 1], ph[e + 2], ph[e + 3]);
+                        *reinterpret_cast<uint4*>(lo + 2 * e) = make_uint4(pl[e], pl[e + 1], pl[e + 2], pl[e + 3]);
+                    }
+                }
+            }
+            named_sync_pool();  // red is reused by the next unit
         }
     }
 }
@@ -276,15 +397,17 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
     WsHeader* hdr = a.hdr;
     if (!hdr->valid) return;
     const int32_t total_tiles = a.cu_tiles[a.batch];
-    if (static_cast<int32_t>(blockIdx.x) >= total_tiles) return;
-    const int32_t tile = total_tiles - 1 - blockIdx.x;  // late (long-row) tiles first
+    if (static_cast<int32_t>(blockIdx.y) >= total_tiles) return;
+    // grid (KV head, tile): CTAs start in launch order, so with heads fastest
+    // the late (long-row) tiles of every head start first
+    const int32_t tile = total_tiles - 1 - blockIdx.y;
     int32_t lo = 0, hi = a.batch - 1;                   // request owning this tile
     while (lo < hi) {
         const int32_t mid = (lo + hi + 1) >> 1;
         if (a.cu_tiles[mid] <= tile) lo = mid; else hi = mid - 1;
     }
     const int32_t b = lo;
-    const int32_t g = blockIdx.y;
+    const int32_t g = blockIdx.x;
     const int32_t G = a.G;
     const int32_t cb = a.cu_blocks[b];
     const int32_t nb = a.cu_blocks[b + 1] - cb;
@@ -518,7 +641,13 @@ __global__ void meanlp_kernel(MeanLpArgs a) {
     }
 }
 
-template __global__ void pool_kernel<false>(PoolArgs);
-template __global__ void pool_kernel<true>(PoolArgs);
+template __global__ void pool_kernel<false>(const __grid_constant__ PoolArgs,
+                                            const __grid_constant__ CUtensorMap,
+                                            const __grid_constant__ CUtensorMap,
+                                            const __grid_constant__ CUtensorMap);
+template __global__ void pool_kernel<true>(const __grid_constant__ PoolArgs,
+                                           const __grid_constant__ CUtensorMap,
+                                           const __grid_constant__ CUtensorMap,
+                                           const __grid_constant__ CUtensorMap);
 
 }  // namespace fp2

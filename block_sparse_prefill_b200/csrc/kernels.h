@@ -8,7 +8,7 @@
 
 namespace fp2 {
 
-constexpr int kPoolThreads = 512;  // 4 row groups x 128 column lanes
+constexpr int kPoolThreads = 544;  // 16 consumer warps (4 row groups x 128 column lanes) + TMA warp
 constexpr int kScoreThreads = 160; // score_kernel: 4 epilogue warps + 1 TMA/MMA warp
 
 struct SetupArgs {
@@ -29,14 +29,14 @@ struct SetupArgs {
 };
 
 struct PoolArgs {
-    const void* x[3];        // q, k, v (k/v may be page pools)
     float* out[3];           // fp32 means (NULL = not written): -, k_mean, v_mean
     uint16_t* split[2];      // bf16 hi/lo means of q (grouped rows) and k, see WsLayout
     const float* scale[3];   // per-head dequantisation scales (NULL = 1)
     int32_t heads[3];
-    int32_t slabs[3];        // CTAs per block along the columns of each tensor
+    int32_t hb[3];           // heads per column slab (one TMA box: 32 rows x hb heads x d)
+    int32_t slabs[3];        // column slabs per block of each tensor
     int32_t paged[3];
-    int32_t ntensors;        // 2 (q, k) or 3 (q, k, v)
+    int32_t first, last;     // tensors [first, last) of q, k, v are pooled
     const int32_t* cu;
     const int32_t* cu_blocks;
     const int32_t* blk_req;
@@ -102,7 +102,10 @@ struct AttnArgs {
 
 __global__ void setup_kernel(SetupArgs a);
 template <bool kE4M3>
-__global__ void pool_kernel(PoolArgs a);
+__global__ void pool_kernel(const __grid_constant__ PoolArgs a, const __grid_constant__ CUtensorMap tq,
+                            const __grid_constant__ CUtensorMap tk,
+                            const __grid_constant__ CUtensorMap tv);
+size_t pool_smem_bytes(bool e4m3);
 __global__ void score_kernel(const __grid_constant__ ScoreArgs a,
                              const __grid_constant__ CUtensorMap tqh,
                              const __grid_constant__ CUtensorMap tql,
