@@ -93,7 +93,9 @@ struct Cfg {
 
 struct Bars {
     uint64_t q_full;
-    uint64_t q_empty;     // the last S MMA of a work item has read Q
+    uint64_t q_empty;     // the last S MMAs of a work item have read Q (committed right
+                          // after them, so the next item's Q loads during the item's
+                          // last tile step)
     uint64_t s_full[2];
     uint64_t p_full[2];
     uint64_t o_done[2];   // the last PV of Q tile t in a work item has finished
@@ -479,6 +481,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mma_commit(&bars.s_full[qt]);
                 }
                 mma_commit(&bars.kv_empty[slot(base)]);
+                if (ntot == 1) mma_commit(&bars.q_empty);
                 for (int32_t n = 0; ok && n < ntot; ++n) {
                     const int32_t iv = base + 2 * n + 1, ik = base + 2 * n + 2;
                     const bool next = n + 1 < ntot;
@@ -511,11 +514,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                     }
                     if (!ok) break;
+                    if (n + 2 == ntot) mma_commit(&bars.q_empty);  // S_t(ntot-1) were the last
                     if (next) mma_commit(&bars.kv_empty[slot(ik)]);
                     mma_commit(&bars.kv_empty[slot(iv)]);
                 }
-                // every S MMA of this item has been issued: Q is free once they finish
-                mma_commit(&bars.q_empty);
                 base += 2 * ntot;
                 mbar_arrive(&bars.meta_empty[buf]);
             }
