@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 
 #include <cmath>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -346,6 +347,8 @@ fp2_status run_attention(const fp2_params* p, const void* q, const void* k, cons
     a.G = p->num_q_heads / p->num_kv_heads;
     a.pairs = (a.G + 1) / 2;
     a.correction = p->correction;
+    // test hook (tests/test_gpu_errors.py): make one bounded wait run out
+    a.test_wait_timeout = std::getenv("FP2_TEST_WAIT_TIMEOUT") != nullptr ? 1 : 0;
     a.scale_log2 = tau_of(p) * 1.4426950408889634f;
     a.q_scale = p->q_scale;
     a.k_scale = p->k_scale;

@@ -106,6 +106,7 @@ struct Bars {
                           // never be two phases behind
     uint64_t meta_full[2];
     uint64_t meta_empty[2];
+    uint64_t never;       // completed by nothing (the timeout test hook waits on it)
 };
 
 struct SmemMisc {
@@ -248,6 +249,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&bars.kv_full[s], 1);
             mbar_init(&bars.kv_empty[s], 1);
         }
+        mbar_init(&bars.never, 1);
         mbar_init(&bars.v_tail[0], 1);
         mbar_init(&bars.v_tail[1], 1);
         misc->abort = 0;
@@ -361,6 +363,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_prefetch_desc(&tv);
         }
         int32_t issued = 0;  // K/V ring entries issued so far
+        int32_t nq = 0;      // Q loads issued so far
         for (int32_t k = 0; !*abort; ++k) {
             const int32_t buf = k & 1;
             if (!warp_wait(&bars.meta_full[buf], (k >> 1) & 1, hdr, abort, 510000 + k)) break;
@@ -378,6 +381,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (leader) {
                         if (k > 0) ok = mbar_wait(&bars.q_empty, (k - 1) & 1, hdr, abort, 520000 + k);
                         if (ok) {
+                            ++nq;
                             mbar_arrive_expect_tx(&bars.q_full, ntiles * C::kTileBytes);
                             for (int qt = 0; qt < ntiles; ++qt)
                                 for (int ch = 0; ch < C::kChunks; ++ch)
@@ -445,12 +449,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (leader) mbar_arrive(&bars.meta_empty[buf]);
             if (!ok) break;
         }
-        // drain: every issued tile has been consumed and released
+        // drain: every issued tile has been consumed and released; after an
+        // abort, at least every issued copy has landed
         if (leader) {
-            for (int32_t idx = max(0, issued - C::kSlots); idx < issued; ++idx) {
+            bool drained = true;
+            for (int32_t idx = max(0, issued - C::kSlots); drained && idx < issued; ++idx) {
                 const int32_t s = idx % C::kSlots;
-                if (!mbar_wait(&bars.kv_empty[s], (idx / C::kSlots) & 1, hdr, abort, 200000 + idx))
-                    break;
+                drained = mbar_wait(&bars.kv_empty[s], (idx / C::kSlots) & 1, hdr, abort, 200000 + idx);
+            }
+            if (!drained) {
+                for (int32_t idx = max(0, issued - C::kSlots); idx < issued; ++idx)
+                    mbar_wait_drain(&bars.kv_full[idx % C::kSlots], (idx / C::kSlots) & 1);
+                if (nq > 0) mbar_wait_drain(&bars.q_full, (nq - 1) & 1);
             }
         }
       } else if (warp == kMmaWarp) {
@@ -471,6 +481,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (m->stop) break;
                 const int32_t ntiles = m->ntiles, ntot = m->cnt + m->ncorr;
                 const bool partial = m->nrows < kBlock;
+                if (a.test_wait_timeout && k == 0 &&
+                    !(ok = mbar_wait(&bars.never, 0, hdr, abort, 900000)))
+                    break;
                 ok = mbar_wait(&bars.q_full, k & 1, hdr, abort, 300000) &&
                      mbar_wait(&bars.kv_full[slot(base)], phase(base), hdr, abort, 301000);
                 if (!ok) break;

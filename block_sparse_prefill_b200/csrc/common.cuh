@@ -88,4 +88,13 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, WsHead
     }
 }
 
+// Bounded wait that ignores the abort flag: a role that stops early still waits
+// (at most ~2^31 cycles) for the TMA copies it issued to land before the CTA exits.
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) {
+    const long long start = clock64();
+    while (!mbar_try_wait(bar, parity))
+        if (clock64() - start > (1ll << 31)) return false;
+    return true;
+}
+
 }  // namespace fp2

@@ -257,6 +257,10 @@ __global__ void __launch_bounds__(kPoolThreads, 1)
                                 p.y * a.hb[p.x], static_cast<int32_t>(row0 + sub * kPoolStageRows));
                 }
             }
+            // the issued copies land before the CTA exits (the consumers may have
+            // stopped waiting after an abort)
+            for (int32_t c = max(0, cnt - kPoolStages); c < cnt; ++c)
+                mbar_wait_drain(&ps->full[c % kPoolStages], (c / kPoolStages) & 1);
         }
     } else {
         // ---- consumers: thread (row group rg, 16-byte column lane tc) -----------
@@ -446,6 +450,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
                 tma_load_2d(qh + ch * 16384, &tqh, &ss->q_full, ch * 64, qrow);
                 tma_load_2d(ql + ch * 16384, &tql, &ss->q_full, ch * 64, qrow);
             }
+            int32_t nload = 0;  // K chunk loads issued
             auto load = [&](int32_t idx) -> bool {
                 const int32_t s = idx & 1;
                 if (!mbar_wait(&ss->kv_empty[s], ((idx >> 1) & 1) ^ 1, hdr, abort, 600000 + idx))
@@ -456,6 +461,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
                     tma_load_2d(kh + s * kTileQ + ch * 16384, &tkh, &ss->kv_full[s], ch * 64, row);
                     tma_load_2d(kl + s * kTileQ + ch * 16384, &tkl, &ss->kv_full[s], ch * 64, row);
                 }
+                ++nload;
                 return true;
             };
             bool ok = load(0) && mbar_wait(&ss->q_full, 0, hdr, abort, 610000);
@@ -479,9 +485,14 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
                 mma_commit(&ss->acc_full[s]);
                 mma_commit(&ss->kv_empty[s]);
             }
-            // all loads consumed before the CTA exits
+            // all loads consumed before the CTA exits; after an abort, at least landed
             for (int32_t idx = max(0, steps - 2); ok && idx < steps; ++idx)
                 ok = mbar_wait(&ss->kv_empty[idx & 1], (idx >> 1) & 1, hdr, abort, 640000 + idx);
+            if (!ok) {
+                for (int32_t idx = max(0, nload - 2); idx < nload; ++idx)
+                    mbar_wait_drain(&ss->kv_full[idx & 1], (idx >> 1) & 1);
+                mbar_wait_drain(&ss->q_full, 0);
+            }
         }
     } else {
         // ---- epilogue: row r of the tile ---------------------------------------

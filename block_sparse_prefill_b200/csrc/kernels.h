@@ -91,6 +91,8 @@ struct AttnArgs {
     int32_t nb_cap;              // >= key blocks of the longest request (shared-memory lists)
     int32_t hq, hkv, G, pairs;   // pairs = ceil(G / 2) CTAs per (q-block, KV head)
     int32_t correction;
+    int32_t test_wait_timeout;   // 1: the MMA issuer waits on a barrier nothing completes
+                                 // (tests the bounded-wait timeout and abort path)
     float scale_log2;            // tau * log2(e)
     const float* q_scale;        // e4m3 only
     const float* k_scale;

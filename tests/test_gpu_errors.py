@@ -82,3 +82,33 @@ def test_corrupt_kept_list_is_reported():
     fp2.sparse_prefill(params, q, k, v, cu, wl.max_seqlen, meta, out, ws)
     assert fp2.get_error(ws) == BAD_INDEX
     assert torch.isfinite(out.float()).all()
+
+
+TIMEOUT = 5
+
+
+def test_wait_timeout_is_reported_and_the_context_stays_usable(monkeypatch):
+    """The attention kernel's bounded waits: with the FP2_TEST_WAIT_TIMEOUT hook its MMA issuer
+    waits on a barrier that nothing completes.  After about a second (2^31 cycles) the wait
+    gives up, records FP2_ERR_TIMEOUT and sets the CTA's abort flag; every role stops, the
+    issued TMA copies land, TMEM is freed and the kernel returns.  The same context and
+    workspace then run the call again with a bit-identical result."""
+    wl = make_workload([1000, 700], 4, 2, alpha=0.1, seed=9)
+    params, meta, ws, out = _setup(wl)
+    cu = torch.from_numpy(wl.cu_seqlens).cuda()
+    q, k, v = wl.q.cuda(), wl.k.cuda(), wl.v.cuda()
+    fp2.estimate(params, q, k, v, cu, wl.max_seqlen, meta, ws)
+    fp2.sparse_prefill(params, q, k, v, cu, wl.max_seqlen, meta, out, ws)
+    assert fp2.get_error(ws) == 0
+    ref = out.clone()
+
+    monkeypatch.setenv("FP2_TEST_WAIT_TIMEOUT", "1")
+    out.zero_()
+    fp2.sparse_prefill(params, q, k, v, cu, wl.max_seqlen, meta, out, ws)
+    assert fp2.get_error(ws) == TIMEOUT
+    monkeypatch.delenv("FP2_TEST_WAIT_TIMEOUT")
+
+    out.zero_()
+    fp2.sparse_prefill(params, q, k, v, cu, wl.max_seqlen, meta, out, ws)
+    assert fp2.get_error(ws) == 0
+    assert torch.equal(out.view(torch.int16), ref.view(torch.int16))
