@@ -9,9 +9,10 @@
 //   pool_kernel    block means of Q, K, V (HBM-bound streaming pass, every input
 //                  byte read once, TMA into a ring of shared-memory stages)
 //   score_kernel   s = tau * qbar . kbar for the causal block pairs of a tile of
-//                  q-blocks (fp32 FMA from shared memory), per-head row max,
-//                  exp(s - m) >= alpha threshold, union over the G query heads of
-//                  a KV head, forced diagonal, ascending compaction
+//                  q-blocks (tcgen05 MMAs on bf16 hi/lo parts of the means, fp32
+//                  accumulation in TMEM), per-head row max, exp(s - m) >= alpha
+//                  threshold, union over the G query heads of a KV head, forced
+//                  diagonal, ascending compaction
 //   meanlp_kernel  block means -> bf16 / e4m3 operands of the correction MMA
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>

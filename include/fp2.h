@@ -43,6 +43,10 @@
  * by the caller, except the fp2_params / fp2_blockmeta structs themselves,
  * which are read on the host during the call.  The library allocates no memory
  * and keeps no global state; scratch memory is the caller's workspace.
+ * Alignment: q, k, v (or the pools), out, k_mean and v_mean start on 16-byte
+ * boundaries (TMA operands and 16-byte accesses), lse on 4 bytes, the workspace
+ * on 256 bytes; otherwise the call returns FP2_ERR_INVALID_ARG (FP2_ERR_WORKSPACE
+ * for the workspace) without enqueuing anything.
  *
  * Errors: argument errors are returned synchronously and nothing is enqueued.
  * A failed launch returns FP2_ERR_CUDA.  Errors found on the device (a bad
