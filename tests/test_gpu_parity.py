@@ -124,6 +124,28 @@ def test_paged_equals_contiguous_small():
     _check_outputs(wl, gp, True)
 
 
+def test_e4m3_paged_equals_contiguous():
+    """e4m3 page pools (the pooling kernel's byte-wide TMA boxes over pages) give the masks
+    and the output of the contiguous e4m3 path, which matches the oracle."""
+    wl = make_workload([900, 130, 2000, 1], 8, 2, alpha=0.1, seed=42, dtype="e4m3", paged=True)
+    gp = run_gpu(wl, paged=True)
+    gc = run_gpu(wl, paged=False)
+    assert (gp["kept_cnt"] == gc["kept_cnt"]).all() and (gp["kept_idx"] == gc["kept_idx"]).all()
+    assert np.array_equal(gp["o"], gc["o"], equal_nan=True), "paged output differs from contiguous"
+    _check_masks(wl, gp)
+    _check_outputs(wl, gp, True, max_abs=E4M3_MAX_ABS, mean_abs=1.0, lse_abs=E4M3_MAX_ABS)
+
+
+def test_partial_column_slabs_g5():
+    """Hq = 20: the query heads span three 8-head pooling slabs, the last one half outside
+    the tensor (zero-filled TMA box columns); G = 5 gives work items with one Q tile and a
+    score tile of 25 q-blocks whose G rows meet in shared memory."""
+    wl = make_workload([700, 300, 129], 20, 4, alpha=0.1, seed=13, n_retrieval=1)
+    g = run_gpu(wl)
+    _check_masks(wl, g)
+    _check_outputs(wl, g, True)
+
+
 def test_paged_ragged_batch_sampled():
     wl = make_config(4, seqlen=32768)
     g = run_gpu(wl, paged=True)
