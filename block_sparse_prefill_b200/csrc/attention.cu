@@ -136,11 +136,18 @@ __host__ __device__ inline size_t meta_bytes(int32_t nb_cap) {
     return (b + 15) & ~size_t(15);
 }
 
-// Descriptor of K-major operand step k (Q or K tile at `base`).
+// Byte offset of K-major operand step k inside a tile (Q or K).
 template <bool kE4M3>
-__device__ __forceinline__ uint64_t kmajor_desc(uint32_t base, int k) {
-    const uint32_t addr = kE4M3 ? base + k * 32 : base + (k >> 2) * 16384 + (k & 3) * 32;
-    return sdesc_sw128(addr, 16, 1024);
+__device__ __forceinline__ constexpr uint32_t kmajor_off(int k) {
+    return kE4M3 ? k * 32 : (k >> 2) * 16384 + (k & 3) * 32;
+}
+
+// The value itself, opaque to the compiler: keeps a descriptor from being
+// hoisted (with its per-step variants) out of the issuer's loops, which under
+// the issuer's register budget would spill.
+__device__ __forceinline__ uint64_t opaque64(uint64_t x) {
+    asm volatile("mov.b64 %0, %0;" : "+l"(x));
+    return x;
 }
 
 // Descriptor of the MN-major V tile, keys [k*K, (k+1)*K).
@@ -169,14 +176,17 @@ __device__ __forceinline__ void regs_dec() {
 template <bool kE4M3>
 __device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_addr, uint32_t k_addr) {
     using C = Cfg<kE4M3>;
+    // step k's descriptors = step 0's + (offset >> 4) in the start-address field
+    // (no carry out of it: shared-memory addresses are below 256 KB)
+    const uint64_t qa = opaque64(sdesc_sw128(q_addr, 16, 1024));
+    const uint64_t kb = sdesc_sw128(k_addr, 16, 1024);
 #pragma unroll
     for (int k = 0; k < C::kKSteps; ++k) {
+        const uint64_t off = kmajor_off<kE4M3>(k) >> 4;
         if (kE4M3)
-            mma_f8_ss(d_tmem, kmajor_desc<true>(q_addr, k), kmajor_desc<true>(k_addr, k), C::kIdescQK,
-                      k > 0);
+            mma_f8_ss(d_tmem, qa + off, kb + off, C::kIdescQK, k > 0);
         else
-            mma_bf16_ss(d_tmem, kmajor_desc<false>(q_addr, k), kmajor_desc<false>(k_addr, k),
-                        C::kIdescQK, k > 0);
+            mma_bf16_ss(d_tmem, qa + off, kb + off, C::kIdescQK, k > 0);
     }
 }
 
