@@ -150,13 +150,6 @@ __device__ __forceinline__ uint64_t opaque64(uint64_t x) {
     return x;
 }
 
-// Descriptor of the MN-major V tile, keys [k*K, (k+1)*K).
-template <bool kE4M3>
-__device__ __forceinline__ uint64_t vmajor_desc(uint32_t base, int k) {
-    const uint32_t addr = base + k * (kE4M3 ? 4096 : 2048);
-    return sdesc_sw128(addr, 16384, 1024);
-}
-
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, WsHeader* hdr,
                                           volatile int32_t* abort, int32_t where) {
     const bool ok = mbar_wait(bar, parity, hdr, abort, where);
@@ -195,13 +188,15 @@ template <bool kE4M3>
 __device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint32_t v_addr,
                                          bool first) {
     using C = Cfg<kE4M3>;
+    const uint64_t vb = sdesc_sw128(v_addr, 16384, 1024);
 #pragma unroll
     for (int k = 0; k < C::kKSteps; ++k) {
         const uint32_t acc = (!first || k > 0) ? 1u : 0u;
+        const uint64_t off = (k * (kE4M3 ? 4096u : 2048u)) >> 4;  // keys [k*K, (k+1)*K)
         if (kE4M3)
-            mma_f8_ts(o_tmem, p_tmem + 8 * k, vmajor_desc<true>(v_addr, k), C::kIdescPV, acc);
+            mma_f8_ts(o_tmem, p_tmem + 8 * k, vb + off, C::kIdescPV, acc);
         else
-            mma_bf16_ts(o_tmem, p_tmem + 8 * k, vmajor_desc<false>(v_addr, k), C::kIdescPV, acc);
+            mma_bf16_ts(o_tmem, p_tmem + 8 * k, vb + off, C::kIdescPV, acc);
     }
 }
 
@@ -568,11 +563,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 continue;
             }
             const int32_t cnt = m->cnt, ntot = m->cnt + m->ncorr, nwords = m->nwords;
-            const int32_t g = m->g, h = m->h0 + qt, nrows = m->nrows, qrow0 = m->qrow0;
-            const uint32_t* pruned = pruned_of(m);
-            const int32_t* ctiles = ctiles_of(m);
             float qk = a.scale_log2;
-            if (kE4M3) qk *= a.q_scale[h] * a.k_scale[g];
+            if (kE4M3) qk *= a.q_scale[m->h0 + qt] * a.k_scale[m->g];
             // correction tiles: +log2(128) after scaling == +7/qk before it
             const float corr_bias = 7.f / qk;
             float m_ref = -INFINITY;
@@ -596,7 +588,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int c = 0; c < 128; ++c)
                         if (c > r) sv[c] = __float_as_uint(-INFINITY);
                 } else if (n >= cnt) {
-                    const int32_t w0 = ctiles[n - cnt] * 4;
+                    // (lists re-read from the metadata buffer: fewer live registers)
+                    const uint32_t* pruned = pruned_of(m);
+                    const int32_t w0 = ctiles_of(m)[n - cnt] * 4;
 #pragma unroll
                     for (int wi = 0; wi < 4; ++wi) {
                         const uint32_t bits = (w0 + wi < nwords) ? pruned[w0 + wi] : 0u;
@@ -697,6 +691,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             // ---- epilogue: O / l -> bf16 ------------------------------------
             if (ok && ntot > 0 && (ok = warp_wait(&bars.o_done[qt], (items++) & 1, hdr, abort, 420000))) {
+                const int32_t g = m->g, h = m->h0 + qt, nrows = m->nrows, qrow0 = m->qrow0;
                 tc_fence_after();
                 float inv = 1.f / l;
                 if (kE4M3) inv *= a.v_scale[g];
