@@ -116,8 +116,9 @@ struct SmemMisc {
 };
 
 // One work item (a q-block x up to two query heads of one KV head), prepared
-// by the scheduler warp into one of two shared-memory buffers.  The kept list,
-// the pruned-block bitmask and the correction tile list follow the header.
+// by the scheduler warp into one of two shared-memory buffers.  The kept list
+// (as the first K/V row of each kept block, ascending), the pruned-block bitmask
+// and the correction tile list follow the header.
 struct ItemMeta {
     int32_t stop;     // 1: no work left
     int32_t t, b, i, g, h0, ntiles, nrows, qrow0, cb, cnt, ncorr, nwords;
@@ -338,6 +339,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                     nc += __popc(mask);
                 }
             }
+            // kept blocks -> the first K/V row of each (a page of the pool, or the
+            // request's rows), so the producer's per-tile work is one shared-memory read
+            for (int32_t e = lane; e < cnt; e += 32) {
+                const int32_t j = klist[e];
+                int32_t row;
+                if (a.block_table) {
+                    int32_t page = a.block_table[static_cast<int64_t>(b) * a.max_blocks_per_seq + j];
+                    if (page < 0 || page >= a.num_pages) {
+                        set_error(hdr, FP2_ERR_BAD_INDEX, t);
+                        page = 0;
+                    }
+                    row = page * kBlock;
+                } else {
+                    row = a.cu[b] + j * kBlock;
+                }
+                klist[e] = row;
+            }
+            __syncwarp();
             if (lane == 0) {
                 m->stop = 0;
                 m->t = t;
@@ -375,7 +394,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             ItemMeta* m = meta(buf);
             if (m->stop) break;
             const int32_t ntiles = m->ntiles, cnt = m->cnt, ntot = m->cnt + m->ncorr;
-            const int32_t nrows = m->nrows, g = m->g, b = m->b, t = m->t, cb = m->cb;
+            const int32_t nrows = m->nrows, g = m->g, cb = m->cb;
             const int32_t* klist = klist_of(m);
             const int32_t* ctiles = ctiles_of(m);
             bool ok = true;
@@ -401,19 +420,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const CUtensorMap* mv;
                 int32_t row = 0;
                 if (n < cnt) {
-                    const int32_t j = klist[cnt - 1 - n];
+                    row = klist[cnt - 1 - n];  // nearest kept block first (the diagonal)
                     mk = &tk;
                     mv = &tv;
-                    if (a.block_table) {
-                        int32_t page = a.block_table[static_cast<int64_t>(b) * a.max_blocks_per_seq + j];
-                        if (page < 0 || page >= a.num_pages) {
-                            if (leader) set_error(hdr, FP2_ERR_BAD_INDEX, t);
-                            page = 0;
-                        }
-                        row = page * kBlock;
-                    } else {
-                        row = a.cu[b] + j * kBlock;
-                    }
                 } else {
                     mk = &tkb;
                     mv = &tvb;
