@@ -100,7 +100,12 @@ struct Bars {
     uint64_t p_full[2];
     uint64_t o_done[2];   // the last PV of Q tile t in a work item has finished
     uint64_t kv_full[8];
-    uint64_t kv_empty[8];
+    uint64_t ev[8];       // slot-release events: the issuer commits one after the S MMAs
+                          // of an item's first step and one at the end of every step; a
+                          // commit tracks every earlier MMA, so event E + j of an item
+                          // whose first event is E frees its ring entries base .. base + 2j
+                          // (all of them for j = ntot).  A ring of kSlots barriers: no
+                          // event can run kSlots ahead of the producer's wait for it.
     uint64_t v_tail[2];   // per metadata buffer: V rows past the request end zeroed
                           // (partial diagonal block); per buffer so that a waiter can
                           // never be two phases behind
@@ -113,6 +118,7 @@ struct SmemMisc {
     Bars bars;
     uint32_t tmem_base;
     int32_t abort;
+    int32_t rel_ev[8];    // event that frees each ring slot's current entry (producer only)
 };
 
 // One work item (a q-block x up to two query heads of one KV head), prepared
@@ -226,8 +232,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int32_t tid = threadIdx.x;
     const int32_t warp = tid >> 5;
     const int32_t lane = tid & 31;
-    const int32_t per_blk = a.hkv * a.pairs;
-    const int32_t n_items = hdr->total_blocks * per_blk;
 
     auto meta = [&](int32_t buf) { return reinterpret_cast<ItemMeta*>(meta_base + buf * meta_stride); };
     auto klist_of = [](ItemMeta* m) { return reinterpret_cast<int32_t*>(m + 1); };
@@ -253,7 +257,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int s = 0; s < C::kSlots; ++s) {
             mbar_init(&bars.kv_full[s], 1);
-            mbar_init(&bars.kv_empty[s], 1);
+            mbar_init(&bars.ev[s], 1);
         }
         mbar_init(&bars.never, 1);
         mbar_init(&bars.v_tail[0], 1);
@@ -269,6 +273,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       regs_dec<kOtherRegs>();
       if (warp == kSchedWarp) {
         // ---- scheduler: next work item -> metadata buffer ----------------
+        const int32_t per_blk = a.hkv * a.pairs;
+        const int32_t n_items = hdr->total_blocks * per_blk;
         for (int32_t k = 0;; ++k) {
             const int32_t buf = k & 1;
             if (!warp_wait(&bars.meta_empty[buf], ((k >> 1) & 1) ^ 1, hdr, abort, 500000 + k)) break;
@@ -386,8 +392,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_prefetch_desc(&tk);
             tma_prefetch_desc(&tv);
         }
-        int32_t issued = 0;  // K/V ring entries issued so far
-        int32_t nq = 0;      // Q loads issued so far
+        int32_t issued = 0;   // K/V ring entries issued so far
+        int32_t nq = 0;       // Q loads issued so far
+        int32_t ev_item = 0;  // first release event of the current item
         for (int32_t k = 0; !*abort; ++k) {
             const int32_t buf = k & 1;
             if (!warp_wait(&bars.meta_full[buf], (k >> 1) & 1, hdr, abort, 510000 + k)) break;
@@ -397,6 +404,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int32_t nrows = m->nrows, g = m->g, cb = m->cb;
             const int32_t* klist = klist_of(m);
             const int32_t* ctiles = ctiles_of(m);
+            const int32_t item_base = issued;
             bool ok = true;
             for (int32_t n = 0; ok && n < ntot; ++n) {
                 if (n == 1 || (n == 0 && ntot == 1)) {
@@ -432,9 +440,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int32_t idx = issued;
                     const int32_t s = idx % C::kSlots;
                     if (leader) {
-                        ok = mbar_wait(&bars.kv_empty[s], ((idx / C::kSlots) & 1) ^ 1, hdr, abort,
-                                       100000 + n);
+                        if (idx >= C::kSlots) {
+                            const int32_t e = misc->rel_ev[s];
+                            ok = mbar_wait(&bars.ev[e % C::kSlots], static_cast<uint32_t>((e / C::kSlots) & 1),
+                                           hdr, abort, 100000 + n);
+                        }
                         if (ok) {
+                            // entry idx is freed by event ev_item + ceil((idx - base) / 2)
+                            misc->rel_ev[s] = ev_item + (idx - item_base + 1) / 2;
                             mbar_arrive_expect_tx(&bars.kv_full[s], C::kTileBytes);
                             for (int ch = 0; ch < C::kChunks; ++ch)
                                 tma_load_3d(kv_s + s * C::kTileBytes + ch * 16384, kv ? mv : mk,
@@ -462,15 +475,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
             if (leader) mbar_arrive(&bars.meta_empty[buf]);
             if (!ok) break;
+            ev_item += ntot + 1;
         }
-        // drain: every issued tile has been consumed and released; after an
-        // abort, at least every issued copy has landed
+        // drain: every issued tile has been consumed and released (the last item's
+        // last event); after an abort, at least every issued copy has landed
         if (leader) {
             bool drained = true;
-            for (int32_t idx = max(0, issued - C::kSlots); drained && idx < issued; ++idx) {
-                const int32_t s = idx % C::kSlots;
-                drained = mbar_wait(&bars.kv_empty[s], (idx / C::kSlots) & 1, hdr, abort, 200000 + idx);
-            }
+            if (ev_item > 0)
+                drained = mbar_wait(&bars.ev[(ev_item - 1) % C::kSlots],
+                                    static_cast<uint32_t>(((ev_item - 1) / C::kSlots) & 1), hdr, abort, 200000);
             if (!drained) {
                 for (int32_t idx = max(0, issued - C::kSlots); idx < issued; ++idx)
                     mbar_wait_drain(&bars.kv_full[idx % C::kSlots], (idx / C::kSlots) & 1);
@@ -485,6 +498,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             auto slot = [](int32_t idx) { return idx % C::kSlots; };
             auto phase = [](int32_t idx) { return static_cast<uint32_t>((idx / C::kSlots) & 1); };
             int32_t base = 0;          // ring entry of the current item's first K tile
+            int32_t ev_item = 0;       // first release event of the current item
             int32_t it[2] = {0, 0};    // PV iterations issued per Q tile
             int32_t vt[2] = {0, 0};    // partial items seen per metadata buffer
             bool ok = true;
@@ -507,7 +521,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                     kv_addr + slot(base) * C::kTileBytes);
                     mma_commit(&bars.s_full[qt]);
                 }
-                mma_commit(&bars.kv_empty[slot(base)]);
+                mma_commit(&bars.ev[ev_item % C::kSlots]);  // frees K_0
                 if (ntot == 1) mma_commit(&bars.q_empty);
                 for (int32_t n = 0; ok && n < ntot; ++n) {
                     const int32_t iv = base + 2 * n + 1, ik = base + 2 * n + 2;
@@ -542,10 +556,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     if (!ok) break;
                     if (n + 2 == ntot) mma_commit(&bars.q_empty);  // S_t(ntot-1) were the last
-                    if (next) mma_commit(&bars.kv_empty[slot(ik)]);
-                    mma_commit(&bars.kv_empty[slot(iv)]);
+                    mma_commit(&bars.ev[(ev_item + n + 1) % C::kSlots]);  // frees V_n, K_(n+1)
                 }
                 base += 2 * ntot;
+                ev_item += ntot + 1;
                 mbar_arrive(&bars.meta_empty[buf]);
             }
         }
