@@ -16,11 +16,13 @@
 //   warpgroup 0 (warps 0-3)  softmax of Q tile 0 (one thread per row = TMEM lane)
 //   warpgroup 1 (warps 4-7)  softmax of Q tile 1
 //   warpgroup 2: warp 8      TMA producer: Q tiles, then K/V (or mean-K/mean-V)
-//                            tiles into a ring of shared-memory slots, following
-//                            the kept list and, in paged mode, the block table
+//                            tiles into a ring of shared-memory slots, at the rows
+//                            the scheduler prepared
 //                warp 9      TMEM owner and MMA issuer
 //                warp 10     scheduler: takes work items from a global counter and
-//                            prepares their kept lists in shared memory
+//                            prepares them in shared memory: the kept list as K/V
+//                            rows (pages of the pool, through the block table, in
+//                            paged mode), the pruned blocks, the correction tiles
 //                warp 11     idle (it only donates registers)
 // The softmax warpgroups raise their register budget (setmaxnreg) so that a
 // whole 128-column row of S stays in registers; warpgroup 2 lowers its own.
@@ -31,7 +33,9 @@
 // order, so S_t(n+1) may be issued right after PV_t(n), which still reads P_t
 // from the same columns):
 //   PV_0(n), S_0(n+1), PV_1(n), S_1(n+1)
-// so the softmax of one tile overlaps the other tile's two MMAs.
+// so the softmax of one tile overlaps the other tile's two MMAs.  Three commits
+// per step (each costs tensor-pipe time): S_0 ready, S_1 ready, and one event
+// that frees the step's K/V ring entries.
 // The running max is only raised when a row max exceeds it by more than a
 // threshold (log2 units), so O is rarely rescaled.
 // Tile order: diagonal block first (it fixes the causal mask and usually the
