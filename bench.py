@@ -230,6 +230,48 @@ def time_layer(st, wl, steps, warmup, dist_ctx, clocks=None):
     return total, est, att, clk
 
 
+def approximation_error(st, wl, n_rows=256, seed=7):
+    """The method's approximation quality (not a parity check): the block-sparse output of the
+    layer against dense causal softmax attention, computed in fp64 on the GPU with torch, on
+    `n_rows` seeded rows of a single-request layer, all query heads.  Also for the same call
+    without the mean correction, which shows what the correction term buys."""
+    import torch
+    import block_sparse_prefill_b200 as fp2
+    assert wl.batch == 1
+    T, hq, hkv = wl.total_tokens, wl.num_q_heads, wl.num_kv_heads
+    G = hq // hkv
+    tau = 1.0 / math.sqrt(wl.head_dim)
+    rows = np.sort(np.random.default_rng(seed).choice(T, n_rows, replace=False))
+    rows_t = torch.from_numpy(rows).to(st["q"].device)
+    # the same layer without the correction term
+    p0 = fp2.Params(num_q_heads=hq, num_kv_heads=hkv, alpha=wl.alpha, correction=False,
+                    dtype=st["params"].dtype)
+    out0 = torch.empty_like(st["out"])
+    fp2.sparse_prefill(p0, st["q"], st["k"], st["v"], st["cu"], wl.max_seqlen, st["meta"], out0, st["ws"])
+    torch.cuda.synchronize()
+    q = st["q"][rows_t].double()
+    keys = torch.arange(T, device=q.device)
+    causal = keys[None, :] > rows_t[:, None]
+    err = {"with": [], "without": []}
+    ref_norm = 0.0
+    for g in range(hkv):
+        kg, vg = st["k"][:, g].double(), st["v"][:, g].double()
+        for h in range(g * G, (g + 1) * G):
+            logits = (q[:, h] @ kg.T) * tau
+            logits.masked_fill_(causal, float("-inf"))
+            ref = torch.softmax(logits, dim=1) @ vg
+            ref_norm += float((ref ** 2).sum())
+            for key, o in (("with", st["out"]), ("without", out0)):
+                err[key].append(o[rows_t, h].double() - ref)
+    res = {"rows": int(n_rows), "heads": hq, "reference": "dense causal softmax attention, fp64"}
+    for key in ("with", "without"):
+        e = torch.stack(err[key])
+        res[key + "_correction"] = {"max_abs": float(e.abs().max()), "mean_abs": float(e.abs().mean()),
+                                    "rel_l2": math.sqrt(float((e ** 2).sum()) / ref_norm)}
+    del out0
+    return res
+
+
 def time_e2e(st, wl, steps, dist_ctx):
     """Same layer through the C ABI with host buffers: every step copies its Q/K/V from pinned
     host memory and reads its output back, inside the timed region.  Steps are pipelined as
@@ -424,6 +466,8 @@ def ours(args):
     ms_att = statistics.mean(att)
     value = weak_scaling_value(ctx.world, flops, ms_step)
 
+    approx = approximation_error(st, wl) if wl.batch == 1 else None
+
     e2e = None
     if not args.no_e2e:
         e2e_ms, h2d, d2h = time_e2e(st, wl, max(2, min(6, args.steps)), ctx)
@@ -491,6 +535,8 @@ def ours(args):
         "ms_per_layer": ms_step,
         "ms_estimate": ms_est,
         "ms_attention": ms_att,
+        "ms_attention_median": statistics.median(att), "ms_attention_min": min(att),
+        "ms_estimate_median": statistics.median(est), "ms_estimate_min": min(est),
         "tflops_attention": ach_att,
         "roofline": {
             "bound": "tensor", "achieved": ach_att, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
@@ -513,6 +559,7 @@ def ours(args):
         "gpu_launches": args.steps * 6,
         "clocks": clk,
         "fp8": fp8,
+        "approximation_vs_dense": approx,
     }
     if ctx.rank == 0 and ctx.world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl)
