@@ -601,10 +601,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!(ok = warp_wait(&bars.s_full[qt], it & 1, hdr, abort, 400000 + n))) break;
                 tc_fence_after();
                 uint32_t sv[128];
-                tmem_ld32(s_addr + 0, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-                tmem_ld32(s_addr + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
-                tmem_ld32(s_addr + 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[64]));
-                tmem_ld32(s_addr + 96, *reinterpret_cast<uint32_t(*)[32]>(&sv[96]));
+                tmem_ld128(s_addr, sv);
                 tmem_wait_ld();
                 // masks (warp-uniform branch per tile kind):
                 //   diagonal block (n == 0): keys c <= r
@@ -664,52 +661,59 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 // P = exp2(s * qk - m + offset) in the MMA precision, written over S
                 const float neg = C::kPOffset - ((m_ref == -INFINITY) ? 0.f : m_ref);
-                // exp2 of packed pairs (MUFU; optionally some pairs on the FMA pipe)
+                // exp2 of packed pairs (MUFU; optionally some pairs on the FMA pipe), in
+                // two halves of 64 keys: the first half's P goes to TMEM (asynchronously)
+                // while the second half is computed
                 float2 rsp[4];
 #pragma unroll
                 for (int j = 0; j < 4; ++j) rsp[j] = make_float2(0.f, 0.f);
+                __half2 hs[4];  // e4m3: sums of the quantised weights
 #pragma unroll
-                for (int c = 0; c < 128; c += 2) {
-                    float2 x = ffma2(make_float2(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])),
-                                     make_float2(qk, qk), make_float2(neg, neg));
-                    if (C::kEmuEvery > 0 &&
-                        ((c >> 1) % (C::kEmuEvery > 0 ? C::kEmuEvery : 1)) == C::kEmuEvery - 1) {
-                        x = exp2_poly2(x);
-                    } else {
-                        x.x = ex2(x.x);
-                        x.y = ex2(x.y);
+                for (int j = 0; j < 4; ++j) hs[j] = __float2half2_rn(0.f);
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf) {
+#pragma unroll
+                    for (int c = 64 * hf; c < 64 * hf + 64; c += 2) {
+                        float2 x = ffma2(make_float2(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])),
+                                         make_float2(qk, qk), make_float2(neg, neg));
+                        if (C::kEmuEvery > 0 &&
+                            ((c >> 1) % (C::kEmuEvery > 0 ? C::kEmuEvery : 1)) == C::kEmuEvery - 1) {
+                            x = exp2_poly2(x);
+                        } else {
+                            x.x = ex2(x.x);
+                            x.y = ex2(x.y);
+                        }
+                        sv[c] = __float_as_uint(x.x);
+                        sv[c + 1] = __float_as_uint(x.y);
+                        rsp[(c >> 1) & 3] = fadd2(rsp[(c >> 1) & 3], x);
                     }
-                    sv[c] = __float_as_uint(x.x);
-                    sv[c + 1] = __float_as_uint(x.y);
-                    rsp[(c >> 1) & 3] = fadd2(rsp[(c >> 1) & 3], x);
+                    if (kE4M3) {
+                        // the O normaliser sums the quantised weights the PV MMA sees
+#pragma unroll
+                        for (int c = 16 * hf; c < 16 * hf + 16; ++c) {
+                            const uint32_t pk = pack_e4m3x4(
+                                __uint_as_float(sv[4 * c]), __uint_as_float(sv[4 * c + 1]),
+                                __uint_as_float(sv[4 * c + 2]), __uint_as_float(sv[4 * c + 3]));
+                            hs[c & 3] = __hadd2(hs[c & 3], e4m3x4_sum2(pk));
+                            sv[c] = pk;
+                        }
+                        tmem_st16(s_addr + 16 * hf, &sv[16 * hf]);
+                    } else {
+#pragma unroll
+                        for (int c = 32 * hf; c < 32 * hf + 32; ++c)
+                            sv[c] = pack_bf16(__uint_as_float(sv[2 * c]), __uint_as_float(sv[2 * c + 1]));
+                        tmem_st32(s_addr + 32 * hf, *reinterpret_cast<uint32_t(*)[32]>(&sv[32 * hf]));
+                    }
                 }
                 const float2 rs2 = fadd2(fadd2(rsp[0], rsp[1]), fadd2(rsp[2], rsp[3]));
                 const float rs = rs2.x + rs2.y;
                 l_lse += rs;
                 if (kE4M3) {
-                    // the O normaliser sums the quantised weights the PV MMA sees
-                    __half2 hs[4];
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) hs[j] = __float2half2_rn(0.f);
-#pragma unroll
-                    for (int c = 0; c < 32; ++c) {
-                        const uint32_t pk = pack_e4m3x4(
-                            __uint_as_float(sv[4 * c]), __uint_as_float(sv[4 * c + 1]),
-                            __uint_as_float(sv[4 * c + 2]), __uint_as_float(sv[4 * c + 3]));
-                        hs[c & 3] = __hadd2(hs[c & 3], e4m3x4_sum2(pk));
-                        sv[c] = pk;
-                    }
                     const float2 h01 = __half22float2(hs[0]), h23 = __half22float2(hs[1]);
                     const float2 h45 = __half22float2(hs[2]), h67 = __half22float2(hs[3]);
                     l += ((h01.x + h01.y) + (h23.x + h23.y)) + ((h45.x + h45.y) + (h67.x + h67.y));
-                    tmem_st32(s_addr, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
                 } else {
                     l += rs;
-#pragma unroll
-                    for (int c = 0; c < 64; ++c)
-                        sv[c] = pack_bf16(__uint_as_float(sv[2 * c]), __uint_as_float(sv[2 * c + 1]));
-                    tmem_st32(s_addr, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-                    tmem_st32(s_addr + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
                 }
                 tmem_wait_st();
                 tc_fence_before();
