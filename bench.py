@@ -35,6 +35,11 @@ METRIC = "ms/layer & effective TFLOP/s at 128K prefill (BF16/FP8); % of tensor-c
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 E4M3_OVER_BF16 = 2.0  # nominal dense ratio (4.5 / 2.25 PFLOP/s)
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch of the 128K bf16 layer's
+# kernels, from one single-pass ncu capture each of the kernels as they stand (attention:
+# 6.26 GB read + 1.06 GB written; pooling: 1.61 GB + 0.03 GB).  Reported only for that
+# workload; to be captured again whenever these kernels change.
+TRAFFIC_128K = {"attention": 7.32e9, "pool": 1.64e9}
 
 
 def load_peaks():
@@ -540,7 +545,8 @@ def ours(args):
         "tflops_attention": ach_att,
         "roofline": {
             "bound": "tensor", "achieved": ach_att, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-            "frac": ach_att / peaks["bf16_tflops"], "traffic": None,
+            "frac": ach_att / peaks["bf16_tflops"],
+            "traffic": TRAFFIC_128K["attention"] if wl.max_seqlen == 131072 else None,
             "kernel": "attention_kernel<bf16> (fp2_sparse_prefill call)",
             "work": "4*d flops per kept causal query-key pair + 4*d per (row, pruned block) correction term",
             "peak_kind": f"{peaks_kind} bf16 burst",
@@ -553,6 +559,7 @@ def ours(args):
         "estimator_roofline": {
             "bound": "hbm", "achieved": est_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
             "frac": est_gbs / peaks["hbm_gbs"], "bytes": est_bytes,
+            "traffic_pool_kernel": TRAFFIC_128K["pool"] if wl.max_seqlen == 131072 else None,
             "kernel": "fp2_estimate call (pool + score kernels)",
         },
         "e2e": e2e,
