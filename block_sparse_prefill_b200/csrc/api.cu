@@ -392,6 +392,8 @@ fp2_status fp2_estimate(const fp2_params* params, const void* q, const void* k, 
     if (st != FP2_OK) return st;
     if ((st = check_meta(meta, params, pr, false)) != FP2_OK) return st;
     if (block_table && (max_blocks_per_seq < 1 || num_pages < 1)) return FP2_ERR_INVALID_ARG;
+    // page rows are int32 inside the kernels (TMA coordinates)
+    if (block_table && int64_t(num_pages) * kBlock > (int64_t(1) << 31) - 1) return FP2_ERR_UNSUPPORTED;
     return run_estimate(params, q, k, v, cu_seqlens, pr, block_table, max_blocks_per_seq, num_pages,
                         meta, workspace, static_cast<cudaStream_t>(stream));
 }
@@ -422,6 +424,8 @@ fp2_status fp2_prefill_paged(const fp2_params* params, const void* q, const void
     if (st != FP2_OK) return st;
     if ((st = check_meta(meta, params, pr, true)) != FP2_OK) return st;
     if (batch > 0 && (!block_table || max_blocks_per_seq < 1 || num_pages < 1)) return FP2_ERR_INVALID_ARG;
+    // page rows are int32 inside the kernels (TMA coordinates)
+    if (int64_t(num_pages) * kBlock > (int64_t(1) << 31) - 1) return FP2_ERR_UNSUPPORTED;
     if (total_tokens > 0 && (!out || !aligned(out, 16))) return FP2_ERR_INVALID_ARG;
     if (lse && !aligned(lse, 4)) return FP2_ERR_INVALID_ARG;
     const cudaStream_t s = static_cast<cudaStream_t>(stream);

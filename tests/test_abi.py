@@ -97,6 +97,8 @@ def test_bad_problem_rejected(lib):
     small = _lib.fp2_blockmeta(4096, 4096, 4096, 4096, None, 4, 9)     # nb_max < ceil(1024/128)
     assert _estimate(lib, p, meta=small) == 1
     assert _estimate(lib, p, bt=ctypes.c_void_p(4096), mbps=0, npages=4) == 1
+    # page rows (page x 128) must fit the kernels' int32 coordinates
+    assert _estimate(lib, p, bt=ctypes.c_void_p(4096), mbps=8, npages=(1 << 24) + 1) == 2
 
 
 def test_workspace_init_checks(lib):
