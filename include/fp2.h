@@ -134,7 +134,8 @@ fp2_status fp2_workspace_init(void* workspace, size_t ws_bytes, void* stream);
  *   k, v         contiguous [total_tokens, Hkv, d] when block_table == NULL,
  *                else page pools [num_pages * block_size, Hkv, d]
  *   block_table  NULL (contiguous) or [batch, max_blocks_per_seq] page indices
- *   num_pages    pages in the pools (paged mode; ignored otherwise) */
+ *   num_pages    pages in the pools (paged mode; ignored otherwise); num_pages *
+ *                block_size < 2^31, else FP2_ERR_UNSUPPORTED */
 fp2_status fp2_estimate(const fp2_params* params, const void* q, const void* k, const void* v,
                         const int32_t* cu_seqlens, int32_t batch, int64_t total_tokens,
                         int32_t max_seqlen, const int32_t* block_table,
