@@ -118,7 +118,8 @@ __global__ void meanlp_kernel(MeanLpArgs a);
 
 // Shared-memory bytes of the attention kernel for a kept-list capacity.
 size_t attn_smem_bytes(bool e4m3, int32_t nb_cap);
-// Launches the attention kernel (one CTA per (q-block, KV head, query-head pair)).
+// Launches the persistent attention kernel: one CTA per SM, taking work items
+// (q-block, KV head, query-head pair) from a counter in the workspace.
 cudaError_t launch_attention(bool e4m3, const AttnArgs& a, const CUtensorMap& tq,
                              const CUtensorMap& tk, const CUtensorMap& tv,
                              const CUtensorMap& tkb, const CUtensorMap& tvb, int64_t max_blocks,
