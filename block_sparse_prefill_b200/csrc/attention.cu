@@ -11,8 +11,9 @@
 //       / [sum_{kept c <= r} e^{l_c}     + sum_{pruned j<i} 128 e^{lbar_j}]
 // with l_c = tau q_r . k_c and lbar_j = tau q_r . kbar_j (pruned blocks are full).
 //
-// Structure (one CTA = one q-block x two query heads of one KV head, so every
-// K/V tile fetched into shared memory serves both heads):
+// Structure: persistent, one CTA per SM.  A work item is one q-block x two query
+// heads of one KV head, so every K/V tile fetched into shared memory serves both
+// heads; the CTA takes items from a counter in the workspace, longest first.
 //   warpgroup 0 (warps 0-3)  softmax of Q tile 0 (one thread per row = TMEM lane)
 //   warpgroup 1 (warps 4-7)  softmax of Q tile 1
 //   warpgroup 2: warp 8      TMA producer: Q tiles, then K/V (or mean-K/mean-V)
