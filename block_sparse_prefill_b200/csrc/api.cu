@@ -1,6 +1,8 @@
 // api.cu -- the C ABI (include/fp2.h): argument checks, workspace layout,
-// TMA descriptors and kernel launches.  No allocation, no global state besides
-// the cached driver entry point of cuTensorMapEncodeTiled.
+// TMA descriptors and kernel launches.  No allocation; the only global state is
+// the cached driver entry point of cuTensorMapEncodeTiled and, for the
+// allocation-free entry point, its static device scratch array and the cached
+// addresses of that array per device.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -54,7 +56,6 @@ bool make_map(CUtensorMap* m, const void* base, bool e4m3, int64_t heads, int64_
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// 2-D bf16 map over [rows, 128] with 128-byte-swizzled boxes of 128 rows x 64 columns.
 // [rows, heads, d] without swizzle, box of 32 rows x hb heads x d (the pooling stages).
 bool make_map_pool(CUtensorMap* m, const void* base, bool e4m3, int64_t heads, int64_t rows,
                    int32_t hb) {
@@ -72,6 +73,7 @@ bool make_map_pool(CUtensorMap* m, const void* base, bool e4m3, int64_t heads, i
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 2-D bf16 map over [rows, 128] with 128-byte-swizzled boxes of 128 rows x 64 columns.
 bool make_map_2d(CUtensorMap* m, const void* base, int64_t rows) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return false;
