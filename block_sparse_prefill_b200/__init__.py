@@ -51,6 +51,73 @@ def _check(code: int, where: str):
         raise FP2Error(code, where)
 
 
+_E4M3_DTYPES = (torch.float8_e4m3fn, torch.uint8)
+
+
+def _arg(t, name: str, dtypes, shape, where: str):
+    """Checks one array argument before its pointer goes to the C ABI, which
+    sees only the address: a dense (contiguous) tensor of one of ``dtypes``
+    whose shape matches ``shape`` (None entries match any size).  ``None``
+    passes for optional arguments.  The device is checked by ``_same_cuda``
+    once every argument's layout has passed."""
+    if t is None:
+        return
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{where}: {name} must be a torch.Tensor, got {type(t).__name__}")
+    if t.dtype not in dtypes:
+        raise TypeError(f"{where}: {name} has dtype {t.dtype}, expected one of {list(dtypes)}")
+    if t.dim() != len(shape) or any(s is not None and s != n for s, n in zip(shape, t.shape)):
+        want = "[" + ", ".join("*" if s is None else str(s) for s in shape) + "]"
+        raise ValueError(f"{where}: {name} has shape {list(t.shape)}, expected {want}")
+    if not t.is_contiguous():
+        raise ValueError(f"{where}: {name} must be contiguous (row-major); pass .contiguous()")
+
+
+def _same_cuda(where: str, **arrays) -> None:
+    """Every array given must sit on one CUDA device (an array on another GPU
+    would reach the kernels as a peer address)."""
+    dev = None
+    for name, t in arrays.items():
+        if t is None:
+            continue
+        if t.device.type != "cuda":
+            raise ValueError(f"{where}: {name} must be on a CUDA device, got {t.device}")
+        if dev is None:
+            dev = t.device
+        elif t.device != dev:
+            raise ValueError(f"{where}: {name} is on {t.device}, the other arrays on {dev}")
+
+
+def _qkv_args(params: "Params", q, k, v, cu_seqlens, out, lse, where: str, kv_rows=None):
+    """Checks the arrays shared by the compute calls: q [T, Hq, d] and k, v
+    [kv_rows, Hkv, d] in the input type, cu_seqlens [batch + 1] int32,
+    out [T, Hq, d] bf16, lse [T, Hq] fp32."""
+    for name, t in (("q", q), ("k", k), ("v", v), ("cu_seqlens", cu_seqlens)):
+        if t is None:
+            raise TypeError(f"{where}: {name} is required")
+    io = (torch.bfloat16,) if params.dtype == FP2_BF16 else _E4M3_DTYPES
+    d, hq, hkv = params.head_dim, params.num_q_heads, params.num_kv_heads
+    _arg(q, "q", io, (None, hq, d), where)
+    T = int(q.shape[0])
+    _arg(k, "k", io, (T if kv_rows is None else kv_rows, hkv, d), where)
+    _arg(v, "v", io, (T if kv_rows is None else kv_rows, hkv, d), where)
+    _arg(cu_seqlens, "cu_seqlens", (torch.int32,), (None,), where)
+    if cu_seqlens.numel() < 1:
+        raise ValueError(f"{where}: cu_seqlens needs batch + 1 >= 1 entries")
+    _arg(out, "out", (torch.bfloat16,), (T, hq, d), where)
+    _arg(lse, "lse", (torch.float32,), (T, hq), where)
+
+
+def _check_args(params: "Params", where: str, q, k, v, cu_seqlens, out=None, lse=None, kv_rows=None,
+                **more) -> None:
+    """Layout of every array argument of a compute call, then their device.
+    ``more`` holds extra arrays already layout-checked by the caller."""
+    params.check(where)
+    _qkv_args(params, q, k, v, cu_seqlens, out, lse, where, kv_rows=kv_rows)
+    _same_cuda(where, q=q, k=k, v=v, cu_seqlens=cu_seqlens, out=out, lse=lse,
+               q_scale=params.q_scale, k_scale=params.k_scale, v_scale=params.v_scale, **more)
+
+
 @dataclasses.dataclass
 class Params:
     """Mirror of ``fp2_params``.  Scales are device tensors (e4m3 only)."""
@@ -66,6 +133,17 @@ class Params:
     v_scale: Optional[torch.Tensor] = None
     head_dim: int = HEAD_DIM
     block_size: int = BLOCK
+
+    def check(self, where: str) -> None:
+        """Checks the e4m3 scale arrays: fp32 device vectors [Hq], [Hkv], [Hkv]."""
+        if self.dtype != FP2_E4M3:
+            return
+        for name, t, n in (("q_scale", self.q_scale, self.num_q_heads),
+                           ("k_scale", self.k_scale, self.num_kv_heads),
+                           ("v_scale", self.v_scale, self.num_kv_heads)):
+            if t is None:
+                raise ValueError(f"{where}: e4m3 inputs need params.{name}")
+            _arg(t, name, (torch.float32,), (n,), where)
 
     def c(self) -> _lib.fp2_params:
         return _lib.fp2_params(self.num_q_heads, self.num_kv_heads, self.head_dim, self.block_size,
@@ -143,6 +221,11 @@ def _bt_args(block_table: Optional[torch.Tensor], num_pages: int):
 def estimate(params: Params, q, k, v, cu_seqlens, max_seqlen: int, meta: BlockMeta, ws: Workspace,
              block_table: Optional[torch.Tensor] = None, num_pages: int = 0, stream=None) -> None:
     """``fp2_estimate``: kept-block lists and block means into ``meta``."""
+    where = "fp2_estimate"
+    if cu_seqlens is not None:
+        _arg(block_table, "block_table", (torch.int32,), (int(cu_seqlens.numel()) - 1, None), where)
+    kv_rows = None if block_table is None else int(num_pages) * params.block_size
+    _check_args(params, where, q, k, v, cu_seqlens, kv_rows=kv_rows, block_table=block_table)
     p, m = params.c(), meta.c()
     bt, mbps, npg = _bt_args(block_table, num_pages)
     _check(_lib.load().fp2_estimate(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens),
@@ -154,6 +237,7 @@ def estimate(params: Params, q, k, v, cu_seqlens, max_seqlen: int, meta: BlockMe
 def sparse_prefill(params: Params, q, k, v, cu_seqlens, max_seqlen: int, meta: BlockMeta, out,
                    ws: Workspace, lse=None, stream=None) -> None:
     """``fp2_sparse_prefill``: attention over the kept blocks (+ mean correction)."""
+    _check_args(params, "fp2_sparse_prefill", q, k, v, cu_seqlens, out, lse)
     p, m = params.c(), meta.c()
     _check(_lib.load().fp2_sparse_prefill(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens),
                                           int(cu_seqlens.numel()) - 1, int(q.shape[0]), int(max_seqlen),
@@ -165,6 +249,13 @@ def sparse_prefill(params: Params, q, k, v, cu_seqlens, max_seqlen: int, meta: B
 def prefill_paged(params: Params, q, k_pool, v_pool, cu_seqlens, max_seqlen: int, block_table,
                   num_pages: int, meta: BlockMeta, out, ws: Workspace, lse=None, stream=None) -> None:
     """``fp2_prefill_paged``: estimator + attention on a paged KV cache."""
+    where = "fp2_prefill_paged"
+    if block_table is None:
+        raise TypeError(f"{where}: block_table is required")
+    if cu_seqlens is not None:
+        _arg(block_table, "block_table", (torch.int32,), (int(cu_seqlens.numel()) - 1, None), where)
+    _check_args(params, where, q, k_pool, v_pool, cu_seqlens, out, lse,
+                kv_rows=int(num_pages) * params.block_size, block_table=block_table)
     p, m = params.c(), meta.c()
     _check(_lib.load().fp2_prefill_paged(ctypes.byref(p), _ptr(q), _ptr(k_pool), _ptr(v_pool),
                                          _ptr(cu_seqlens), int(cu_seqlens.numel()) - 1, int(q.shape[0]),
@@ -181,6 +272,9 @@ def sparse_prefill_noalloc(params: Params, q, k, v, cu_seqlens, max_seqlen: int,
     (the library's own fixed device array serves as scratch).  The first call
     on a device must come before any stream capture on it, and calls that
     overlap on the GPU race on the shared array."""
+    where = "fp2_sparse_prefill_noalloc"
+    _arg(device_status, "device_status", (torch.int32,), (None,), where)
+    _check_args(params, where, q, k, v, cu_seqlens, out, lse, device_status=device_status)
     p, m = params.c(), meta.c()
     _check(_lib.load().fp2_sparse_prefill_noalloc(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens),
                                                   int(cu_seqlens.numel()) - 1, int(q.shape[0]),
