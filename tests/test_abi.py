@@ -105,3 +105,77 @@ def test_workspace_init_checks(lib):
     assert lib.fp2_workspace_init(None, 1024, None) == 3
     assert lib.fp2_workspace_init(ctypes.c_void_p(4100), 1024, None) == 3
     assert lib.fp2_get_error(None, None) == 3
+
+
+def _c_probe(tmp_path, body: str) -> str:
+    """Compiles and runs a small C program against include/fp2.h (gcc, host only)."""
+    import subprocess
+    src = tmp_path / "probe.c"
+    exe = tmp_path / "probe"
+    src.write_text('#include <stdio.h>\n#include <stddef.h>\n#include "fp2.h"\n'
+                   "int main(void) {\n" + body + "return 0;\n}\n")
+    subprocess.run(["gcc", "-std=c11", "-Wall", "-Werror", "-I", os.path.dirname(HEADER), str(src),
+                    "-o", str(exe)], check=True)
+    return subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout
+
+
+@pytest.mark.parametrize("struct", ["fp2_params", "fp2_blockmeta"])
+def test_struct_mirrors_match_the_header(tmp_path, struct):
+    """Every field of the ctypes mirror sits at the C offset with the C size."""
+    mirror = getattr(_lib, struct)
+    body = f'printf("sizeof %zu\\n", sizeof({struct}));\n'
+    for name, _ in mirror._fields_:
+        body += (f'printf("{name} %zu %zu\\n", offsetof({struct}, {name}), '
+                 f'sizeof((({struct}*)0)->{name}));\n')
+    rows = dict((ln.split()[0], ln.split()[1:]) for ln in _c_probe(tmp_path, body).splitlines())
+    assert int(rows.pop("sizeof")[0]) == ctypes.sizeof(mirror)
+    for name, _ in mirror._fields_:
+        off, size = (int(x) for x in rows[name])
+        field = getattr(mirror, name)
+        assert (field.offset, field.size) == (off, size), name
+    # the C struct has no field the mirror lacks: the last field ends the struct
+    last = getattr(mirror, mirror._fields_[-1][0])
+    assert last.offset + last.size == ctypes.sizeof(mirror)
+
+
+def test_enum_values_match_the_header(tmp_path):
+    names = list(_lib.STATUS.values()) + ["FP2_BF16", "FP2_E4M3"]
+    body = "".join(f'printf("{n} %d\\n", (int){n});\n' for n in names)
+    vals = {ln.split()[0]: int(ln.split()[1]) for ln in _c_probe(tmp_path, body).splitlines()}
+    assert {v: k for k, v in _lib.STATUS.items()} == {n: vals[n] for n in _lib.STATUS.values()}
+    assert (vals["FP2_BF16"], vals["FP2_E4M3"]) == (_lib.FP2_BF16, _lib.FP2_E4M3)
+
+
+def _c_width(decl: str):
+    """('ptr', 8) for pointers, else (C type name, byte width) of a declaration."""
+    decl = re.sub(r"\bconst\b", "", decl).strip()
+    if "*" in decl:
+        return ("ptr", 8)
+    base = decl.split()[0]
+    widths = {"int32_t": 4, "int64_t": 8, "size_t": 8, "int": 4, "fp2_status": 4}
+    return (base, widths[base])
+
+
+def test_prototypes_match_the_ctypes_declarations(lib):
+    """Each header prototype: ctypes declares as many arguments, each pointer as a
+    pointer and each integer with the C width, and the matching result type."""
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    protos = re.findall(r"([A-Za-z_][\w\s\*]*?)\b(fp2_[a-z_]+)\s*\(([^)]*)\)\s*;", text)
+    assert {name for _, name, _ in protos} == set(_lib.EXPORTS)
+    for ret, name, args in protos:
+        fn = getattr(lib, name)
+        params = [a.strip() for a in args.split(",") if a.strip() and a.strip() != "void"]
+        assert len(fn.argtypes) == len(params), name
+        for decl, ct in zip(params, fn.argtypes):
+            kind, width = _c_width(decl)
+            if kind == "ptr":
+                assert ct is ctypes.c_void_p or ct is ctypes.c_char_p or issubclass(ct, ctypes._Pointer), \
+                    (name, decl)
+            else:
+                assert ctypes.sizeof(ct) == width, (name, decl)
+                assert (ct(-1).value < 0) == (kind != "size_t"), (name, decl)
+        rkind, rwidth = _c_width(ret)
+        if rkind == "ptr":
+            assert fn.restype is ctypes.c_char_p, name
+        else:
+            assert ctypes.sizeof(fn.restype) == rwidth, name
