@@ -197,7 +197,9 @@ fp2_status run_estimate(const fp2_params* p, const void* q, const void* k, const
     int32_t qt;
     if (!score_tiling(G, &qt)) return FP2_ERR_UNSUPPORTED;
     fp2_status st = run_setup(pr, ws, cu, qt, block_table != nullptr, mbps, meta->max_blocks, s);
-    if (st != FP2_OK || pr.batch == 0 || pr.max_blocks == 0) return st;
+    // an empty batch (no requests, or only empty ones) ends after the setup
+    // kernel has checked cu_seqlens: there is no block to pool or score
+    if (st != FP2_OK || pr.batch == 0 || pr.total_tokens == 0) return st;
 
     const bool e4m3 = p->dtype == FP2_E4M3;
     WsHeader* hdr = at<WsHeader>(ws, 0);
@@ -305,7 +307,7 @@ fp2_status run_attention(const fp2_params* p, const void* q, const void* k, cons
         st = run_setup(pr, ws, cu, 1, block_table != nullptr, mbps, meta->max_blocks, s);
         if (st != FP2_OK) return st;
     }
-    if (pr.batch == 0 || pr.max_blocks == 0) return FP2_OK;
+    if (pr.batch == 0 || pr.total_tokens == 0) return FP2_OK;  // no rows to attend
     WsHeader* hdr = at<WsHeader>(ws, 0);
     void* kb_lp = at<void>(ws, pr.ws.kbar_lp);
     void* vb_lp = at<void>(ws, pr.ws.vbar_lp);

@@ -33,7 +33,9 @@
  *   lse      [total_tokens, Hq]                    fp32 natural-log sum-exp
  *   cu_seqlens [batch + 1] int32, cu_seqlens[0] = 0, non-decreasing,
  *            cu_seqlens[batch] = total_tokens; request b is rows
- *            cu_seqlens[b] .. cu_seqlens[b+1]-1 of q (and of k/v when contiguous)
+ *            cu_seqlens[b] .. cu_seqlens[b+1]-1 of q (and of k/v when contiguous);
+ *            a request may be empty.  With total_tokens == 0 a call only
+ *            checks cu_seqlens (q, k, v and out may then be NULL).
  *   block_table [batch, max_blocks_per_seq] int32: page of logical block j of
  *            request b (paged mode).
  *   Blocks of all requests are numbered globally in request order:

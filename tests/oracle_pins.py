@@ -16,7 +16,7 @@ What pins what (definitions D0-D4 in the oracle header):
   weights_sum       D3 normalised weights (with correction) sum to one
   exact_correction  D3 correction is exact when K/V rows are constant per block
   gqa_packing       D2/D3 head -> group map: packed heads = each head alone
-  ragged            D0 ragged batch = each request alone
+  ragged            D0 ragged batch (an empty request included) = each request alone
   e4m3_scales       D4 dequantisation: codes x power-of-two scale = scaled values
 """
 from __future__ import annotations
@@ -254,7 +254,7 @@ def pin_gqa_packing(orc):
 
 
 def pin_ragged(orc):
-    lens = [300, 1, 520]
+    lens = [300, 0, 1, 520]                          # an empty request among them
     wl = _structured(lens, seed=51)
     q, k, v = wl.float_inputs()
     cu = wl.cu_seqlens
@@ -268,11 +268,14 @@ def pin_ragged(orc):
         qb1, kb1, vb1 = _means(orc, q[s:e], k[s:e], v[s:e], cu1)
         e1 = orc.estimate(qb1, kb1, cu1, 128, alpha=0.2, tau=TAU, nb_max=est["nb_max"])
         nb = (L + 127) // 128
+        assert e1["kept_cnt"].shape[0] == nb
         assert (e1["kept_cnt"] == est["kept_cnt"][t0:t0 + nb]).all()
         r1 = orc.attend(q[s:e], k[s:e], v[s:e], cu1, 128, TAU, e1["kept_cnt"], e1["kept_idx"], correction=True,
                         kbar=kb1, vbar=vb1)
-        assert np.abs(r1["o"] - full["o"][s:e]).max() == 0.0, "request in a batch differs from request alone"
+        assert r1["o"].shape[0] == L
+        assert np.array_equal(r1["o"], full["o"][s:e]), "request in a batch differs from request alone"
         t0 += nb
+    assert t0 == est["kept_cnt"].shape[0]
 
 
 def pin_e4m3_scales(orc):
