@@ -107,27 +107,38 @@ def test_workspace_init_checks(lib):
     assert lib.fp2_get_error(None, None) == 3
 
 
-def _c_probe(tmp_path, body: str) -> str:
-    """Compiles and runs a small C program against include/fp2.h (gcc, host only)."""
+PROBE_DIR = os.path.join(ROOT, "tests", "_build")
+
+
+def _c_probe(name: str, body: str) -> str:
+    """Compiles and runs a small C program against include/fp2.h (gcc, host only),
+    built in the git-ignored tests/_build folder."""
     import subprocess
-    src = tmp_path / "probe.c"
-    exe = tmp_path / "probe"
-    src.write_text('#include <stdio.h>\n#include <stddef.h>\n#include "fp2.h"\n'
-                   "int main(void) {\n" + body + "return 0;\n}\n")
-    subprocess.run(["gcc", "-std=c11", "-Wall", "-Werror", "-I", os.path.dirname(HEADER), str(src),
-                    "-o", str(exe)], check=True)
-    return subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout
+    os.makedirs(PROBE_DIR, exist_ok=True)
+    src = os.path.join(PROBE_DIR, f"{name}_{os.getpid()}.c")
+    exe = src[:-2]
+    with open(src, "w") as f:
+        f.write('#include <stdio.h>\n#include <stddef.h>\n#include "fp2.h"\n'
+                "int main(void) {\n" + body + "return 0;\n}\n")
+    try:
+        subprocess.run(["gcc", "-std=c11", "-Wall", "-Werror", "-I", os.path.dirname(HEADER), src, "-o", exe],
+                       check=True)
+        return subprocess.run([exe], check=True, capture_output=True, text=True).stdout
+    finally:
+        for f in (src, exe):
+            if os.path.exists(f):
+                os.remove(f)
 
 
 @pytest.mark.parametrize("struct", ["fp2_params", "fp2_blockmeta"])
-def test_struct_mirrors_match_the_header(tmp_path, struct):
+def test_struct_mirrors_match_the_header(struct):
     """Every field of the ctypes mirror sits at the C offset with the C size."""
     mirror = getattr(_lib, struct)
     body = f'printf("sizeof %zu\\n", sizeof({struct}));\n'
     for name, _ in mirror._fields_:
         body += (f'printf("{name} %zu %zu\\n", offsetof({struct}, {name}), '
                  f'sizeof((({struct}*)0)->{name}));\n')
-    rows = dict((ln.split()[0], ln.split()[1:]) for ln in _c_probe(tmp_path, body).splitlines())
+    rows = dict((ln.split()[0], ln.split()[1:]) for ln in _c_probe(struct, body).splitlines())
     assert int(rows.pop("sizeof")[0]) == ctypes.sizeof(mirror)
     for name, _ in mirror._fields_:
         off, size = (int(x) for x in rows[name])
@@ -138,10 +149,10 @@ def test_struct_mirrors_match_the_header(tmp_path, struct):
     assert last.offset + last.size == ctypes.sizeof(mirror)
 
 
-def test_enum_values_match_the_header(tmp_path):
+def test_enum_values_match_the_header():
     names = list(_lib.STATUS.values()) + ["FP2_BF16", "FP2_E4M3"]
     body = "".join(f'printf("{n} %d\\n", (int){n});\n' for n in names)
-    vals = {ln.split()[0]: int(ln.split()[1]) for ln in _c_probe(tmp_path, body).splitlines()}
+    vals = {ln.split()[0]: int(ln.split()[1]) for ln in _c_probe("enums", body).splitlines()}
     assert {v: k for k, v in _lib.STATUS.items()} == {n: vals[n] for n in _lib.STATUS.values()}
     assert (vals["FP2_BF16"], vals["FP2_E4M3"]) == (_lib.FP2_BF16, _lib.FP2_E4M3)
 
