@@ -19,6 +19,14 @@
  *               section "Why block-sparse attention for prefill?"; stuffinsider
  *               page, "Technical Details").  n_j = rows of block j.  Token r sees
  *               tokens c <= r of the same request (causal prefill).
+ *               Chunked form (prefill of the last Lq_b of Lk_b tokens, the first
+ *               P_b = Lk_b - Lq_b already in the KV cache; the pages name paged KV
+ *               and continuous batching but not this case, so the plainest
+ *               extension is taken): key blocks as above over Lk_b; query row t
+ *               is position P_b + t; query blocks keep the same absolute grid, so
+ *               q-block i holds the positions of [i Bs, i Bs + Bs) that are in
+ *               [P_b, Lk_b) and the first one may be partial.  Position p sees
+ *               keys c <= p.  With P_b = 0 this is the plain definition.
  *   D1 estimate xbar_j = (1/n_j) sum_{r in j} x_r for x in {q, k, v}
  *               (reading of "computes a small sample of attention scores" /
  *               "estimating scores at the block level": block means), and
@@ -55,40 +63,67 @@
 /* D0: number of blocks of a request of length L. */
 static int64_t nblocks(int64_t L, int64_t Bs) { return (L + Bs - 1) / Bs; }
 
-/* D0: first global block id of every request (cb[B] = total blocks). */
-static void block_offsets(const int32_t* cu, int B, int Bs, int64_t* cb) {
-    cb[0] = 0;
-    for (int b = 0; b < B; ++b) cb[b + 1] = cb[b] + nblocks(cu[b + 1] - cu[b], Bs);
+/* D0 (chunked form): rows at request positions pos0 .. pos0 + L - 1 lie in the
+ * blocks floor(pos0 / Bs) .. ceil((pos0 + L) / Bs) - 1. */
+static int64_t first_block(int64_t pos0, int64_t Bs) { return pos0 / Bs; }
+static int64_t blocks_at(int64_t pos0, int64_t L, int64_t Bs) {
+    return L > 0 ? nblocks(pos0 + L, Bs) - first_block(pos0, Bs) : 0;
 }
 
-/* Total blocks of a batch. */
-int64_t orc_total_blocks(const int32_t* cu, int B, int Bs) {
+/* D0: first global block id of every request (cb[B] = total blocks); the rows
+ * of request b start at position pos0[b] (pos0 NULL: at 0). */
+static void block_offsets(const int32_t* cu, const int64_t* pos0, int B, int Bs, int64_t* cb) {
+    cb[0] = 0;
+    for (int b = 0; b < B; ++b) cb[b + 1] = cb[b] + blocks_at(pos0 ? pos0[b] : 0, cu[b + 1] - cu[b], Bs);
+}
+
+/* D0 (chunked form): P_b = Lk_b - Lq_b, the position of the first query row.
+ * NULL when a request has Lq_b < 0 or Lq_b > Lk_b.  The caller frees it. */
+static int64_t* chunk_starts(const int32_t* cu_q, const int32_t* cu_k, int B) {
+    int64_t* P = (int64_t*)malloc(sizeof(int64_t) * (B + 1));
+    for (int b = 0; b < B; ++b) {
+        int64_t Lq = cu_q[b + 1] - cu_q[b], Lk = cu_k[b + 1] - cu_k[b];
+        if (Lq < 0 || Lq > Lk) { free(P); return NULL; }
+        P[b] = Lk - Lq;
+    }
+    return P;
+}
+
+/* Total blocks of a batch whose request b starts at position pos0[b] (NULL: 0). */
+int64_t orc_total_blocks(const int32_t* cu, const int64_t* pos0, int B, int Bs) {
     int64_t t = 0;
-    for (int b = 0; b < B; ++b) t += nblocks(cu[b + 1] - cu[b], Bs);
+    for (int b = 0; b < B; ++b) t += blocks_at(pos0 ? pos0[b] : 0, cu[b + 1] - cu[b], Bs);
     return t;
 }
 
-/* D1: block means of a dequantised input x[T, H, d] (value * scale[h]).
- * out: [total_blocks, H, d]. */
-void orc_block_means(const float* x, const double* scale, const int32_t* cu, int B, int H, int d,
-                     int Bs, double* out) {
+/* D1: block means of a dequantised input x[T, H, d] (value * scale[h]).  Row
+ * t of request b is at position pos0[b] + t (pos0 NULL: 0); the mean of a
+ * block runs over its positions that hold rows.  out: [total_blocks, H, d]. */
+void orc_block_means(const float* x, const double* scale, const int32_t* cu, const int64_t* pos0,
+                     int B, int H, int d, int Bs, double* out) {
     int64_t* cb = (int64_t*)malloc(sizeof(int64_t) * (B + 1));
-    block_offsets(cu, B, Bs, cb);
+    block_offsets(cu, pos0, B, Bs, cb);
     for (int b = 0; b < B; ++b) {
         int64_t L = cu[b + 1] - cu[b];
-        int64_t nb = nblocks(L, Bs);
+        int64_t p0 = pos0 ? pos0[b] : 0;
+        int64_t i0 = first_block(p0, Bs);
+        int64_t nb = blocks_at(p0, L, Bs);
 #pragma omp parallel for schedule(static)
-        for (int64_t j = 0; j < nb; ++j) {
-            int64_t n = L - j * Bs < Bs ? L - j * Bs : Bs;
-            double denom = MUT(5) ? (double)Bs : (double)n;
+        for (int64_t t = 0; t < nb; ++t) {
+            int64_t i = i0 + t;
+            int64_t lo = i * Bs > p0 ? i * Bs : p0;                       /* first position */
+            int64_t hi = (i + 1) * Bs < p0 + L ? (i + 1) * Bs : p0 + L;   /* one past the last */
+            double denom = MUT(5) ? (double)Bs
+                         : MUT(13) ? (double)(hi - i * Bs)              /* mutant: counts P's rows */
+                         : (double)(hi - lo);
             for (int h = 0; h < H; ++h) {
                 for (int c = 0; c < d; ++c) {
                     double s = 0.0;
-                    for (int64_t r = 0; r < n; ++r) {
-                        int64_t row = cu[b] + j * Bs + r;
+                    for (int64_t p = lo; p < hi; ++p) {
+                        int64_t row = cu[b] + (p - p0);
                         s += (double)x[(row * H + h) * (int64_t)d + c] * scale[h];
                     }
-                    out[((cb[b] + j) * H + h) * (int64_t)d + c] = s / denom;
+                    out[((cb[b] + t) * H + h) * (int64_t)d + c] = s / denom;
                 }
             }
         }
@@ -106,24 +141,35 @@ static double block_score(const double* qbar, const double* kbar, int64_t qb, in
 }
 
 /* D1 + D2: kept-block lists.
- *   kept_cnt [total_blocks, Hkv], kept_idx [total_blocks, Hkv, nb_max] (ascending);
- *   s_out    [total_blocks, Hq, nb_max] raw scores s (NULL to skip), entries j > i untouched;
- *   m_out    [total_blocks, Hq] row maxima (NULL to skip).
- * Returns 0, or -1 when a request has more than nb_max blocks. */
-int orc_estimate(const double* qbar, const double* kbar, const int32_t* cu, int B, int Hq, int Hkv,
-                 int d, int Bs, double tau, double alpha, int nb_max, int32_t* kept_cnt,
-                 int32_t* kept_idx, double* s_out, double* m_out) {
+ *   qbar [total q-blocks, Hq, d] (rows at positions P_b + t, see D0), kbar
+ *   [total k-blocks, Hkv, d]; request b has cu_q[b+1] - cu_q[b] query rows
+ *   and cu_k[b+1] - cu_k[b] keys (cu_q == cu_k: plain prefill).
+ *   kept_cnt [total q-blocks, Hkv], kept_idx [total q-blocks, Hkv, nb_max]:
+ *            the request's key blocks j <= i kept by q-block i, ascending;
+ *   s_out    [total q-blocks, Hq, nb_max] raw scores s (NULL to skip), entries j > i untouched;
+ *   m_out    [total q-blocks, Hq] row maxima (NULL to skip).
+ * Returns 0, -1 when a request has more than nb_max key blocks, -3 when one
+ * has more queries than keys. */
+int orc_estimate(const double* qbar, const double* kbar, const int32_t* cu_q, const int32_t* cu_k,
+                 int B, int Hq, int Hkv, int d, int Bs, double tau, double alpha, int nb_max,
+                 int32_t* kept_cnt, int32_t* kept_idx, double* s_out, double* m_out) {
     int G = Hq / Hkv;
     double ln_alpha = alpha > 0 ? log(alpha) : -INFINITY;
-    int64_t* cb = (int64_t*)malloc(sizeof(int64_t) * (B + 1));
-    block_offsets(cu, B, Bs, cb);
+    int64_t* P = chunk_starts(cu_q, cu_k, B);
+    if (!P) return -3;
     for (int b = 0; b < B; ++b)
-        if (nblocks(cu[b + 1] - cu[b], Bs) > nb_max) { free(cb); return -1; }
+        if (nblocks(cu_k[b + 1] - cu_k[b], Bs) > nb_max) { free(P); return -1; }
+    int64_t* cbq = (int64_t*)malloc(sizeof(int64_t) * (B + 1));
+    int64_t* cbk = (int64_t*)malloc(sizeof(int64_t) * (B + 1));
+    block_offsets(cu_q, P, B, Bs, cbq);
+    block_offsets(cu_k, NULL, B, Bs, cbk);
     for (int b = 0; b < B; ++b) {
-        int64_t nb = nblocks(cu[b + 1] - cu[b], Bs);
+        int64_t i0 = first_block(P[b], Bs);
+        int64_t nbq = blocks_at(P[b], cu_q[b + 1] - cu_q[b], Bs);
 #pragma omp parallel for schedule(dynamic, 1)
-        for (int64_t i = 0; i < nb; ++i) {
-            int64_t qb = cb[b] + i;
+        for (int64_t t = 0; t < nbq; ++t) {
+            int64_t i = i0 + t;                       /* block index in the request */
+            int64_t qb = cbq[b] + t;                  /* global q-block id */
             double* s = (double*)malloc(sizeof(double) * (i + 1));
             unsigned char* keep = (unsigned char*)malloc(i + 1);
             for (int g = 0; g < Hkv; ++g) {
@@ -133,7 +179,7 @@ int orc_estimate(const double* qbar, const double* kbar, const int32_t* cu, int 
                     int gk = MUT(3) ? h % Hkv : g;  /* mutant: wrong head -> group map */
                     double m = -INFINITY;
                     for (int64_t j = 0; j <= i; ++j) {
-                        s[j] = block_score(qbar, kbar, qb, cb[b] + j, h, gk, Hq, Hkv, d, tau);
+                        s[j] = block_score(qbar, kbar, qb, cbk[b] + j, h, gk, Hq, Hkv, d, tau);
                         if (s[j] > m) m = s[j];
                     }
                     for (int64_t j = 0; j <= i; ++j) {
@@ -158,7 +204,9 @@ int orc_estimate(const double* qbar, const double* kbar, const int32_t* cu, int 
             free(keep);
         }
     }
-    free(cb);
+    free(P);
+    free(cbq);
+    free(cbk);
     return 0;
 }
 
@@ -174,44 +222,53 @@ static int list_ok(const int32_t* idx, int32_t cnt, int64_t i) {
 
 /* D3: attention over the kept blocks plus (correction != 0) the mean-corrected
  * pruned blocks.
- *   q [T, Hq, d], k/v [T, Hkv, d] stored values; qs/ks/vs per-head scales;
- *   kbar/vbar [total_blocks, Hkv, d] block means (needed when correction != 0);
+ *   q [Tq, Hq, d], k/v [Tk, Hkv, d] stored values; qs/ks/vs per-head scales;
+ *   cu_q / cu_k: query rows and keys of every request (D0 chunked form;
+ *   cu_q == cu_k: plain prefill);
+ *   kbar/vbar [total k-blocks, Hkv, d] block means (needed when correction != 0);
  *   sel: global q-block ids to compute (NULL = all), nsel entries;
- *   o [T, Hq, d], lse [T, Hq], wsum [T, Hq] (sum of normalised weights; NULL ok).
- * Returns 0, -1 on an invalid kept list, -2 on a bad q-block id. */
+ *   o [Tq, Hq, d], lse [Tq, Hq], wsum [Tq, Hq] (sum of normalised weights; NULL ok).
+ * Returns 0, -1 on an invalid kept list, -2 on a bad q-block id, -3 when a
+ * request has more queries than keys. */
 int orc_attend(const float* q, const float* k, const float* v, const double* qs, const double* ks,
-               const double* vs, const int32_t* cu, int B, int Hq, int Hkv, int d, int Bs,
-               double tau, const int32_t* kept_cnt, const int32_t* kept_idx, int nb_max,
-               int correction, const double* kbar, const double* vbar, const int64_t* sel,
-               int64_t nsel, double* o, double* lse, double* wsum) {
+               const double* vs, const int32_t* cu_q, const int32_t* cu_k, int B, int Hq, int Hkv,
+               int d, int Bs, double tau, const int32_t* kept_cnt, const int32_t* kept_idx,
+               int nb_max, int correction, const double* kbar, const double* vbar,
+               const int64_t* sel, int64_t nsel, double* o, double* lse, double* wsum) {
     int G = Hq / Hkv;
-    int64_t* cb = (int64_t*)malloc(sizeof(int64_t) * (B + 1));
-    block_offsets(cu, B, Bs, cb);
-    int64_t total = cb[B];
+    int64_t* P = chunk_starts(cu_q, cu_k, B);
+    if (!P) return -3;
+    int64_t* cbq = (int64_t*)malloc(sizeof(int64_t) * (B + 1));
+    int64_t* cbk = (int64_t*)malloc(sizeof(int64_t) * (B + 1));
+    block_offsets(cu_q, P, B, Bs, cbq);
+    block_offsets(cu_k, NULL, B, Bs, cbk);
+    int64_t total = cbq[B];
     int64_t nwork = sel ? nsel : total;
-    /* request of every block */
+    /* request of every q-block */
     int32_t* req = (int32_t*)malloc(sizeof(int32_t) * (total > 0 ? total : 1));
     for (int b = 0; b < B; ++b)
-        for (int64_t t = cb[b]; t < cb[b + 1]; ++t) req[t] = b;
+        for (int64_t t = cbq[b]; t < cbq[b + 1]; ++t) req[t] = b;
     int status = 0;
     for (int64_t w = 0; w < nwork; ++w) {
         int64_t qb = sel ? sel[w] : w;
         if (qb < 0 || qb >= total) { status = -2; break; }
         int b = req[qb];
-        int64_t i = qb - cb[b];
+        int64_t i = first_block(P[b], Bs) + (qb - cbq[b]);
         for (int g = 0; g < Hkv; ++g)
             if (!list_ok(kept_idx + (qb * Hkv + g) * (int64_t)nb_max, kept_cnt[qb * Hkv + g], i))
                 status = -1;
     }
-    if (status != 0) { free(cb); free(req); return status; }
+    if (status != 0) { free(P); free(cbq); free(cbk); free(req); return status; }
 
 #pragma omp parallel for schedule(dynamic, 1) collapse(2)
     for (int64_t w = 0; w < nwork; ++w) {
         for (int h = 0; h < Hq; ++h) {
             int64_t qb = sel ? sel[w] : w;
             int b = req[qb];
-            int64_t i = qb - cb[b];
-            int64_t L = cu[b + 1] - cu[b];
+            int64_t p0 = P[b];                         /* position of the first query row */
+            int64_t i0 = first_block(p0, Bs);
+            int64_t i = i0 + (qb - cbq[b]);            /* block index in the request */
+            int64_t L = cu_k[b + 1] - cu_k[b];         /* keys of the request */
             int g = MUT(3) ? h % Hkv : h / G;
             const int32_t* idx = kept_idx + (qb * Hkv + g) * (int64_t)nb_max;
             int32_t cnt = kept_cnt[qb * Hkv + g];
@@ -224,10 +281,10 @@ int orc_attend(const float* q, const float* k, const float* v, const double* qs,
             double* vbuf = (double*)malloc(sizeof(double) * (size_t)cnt * Bs * d);
             double* qd = (double*)malloc(sizeof(double) * d);
             double* acc = (double*)malloc(sizeof(double) * d);
-            int64_t nrows = (L - i * Bs) < Bs ? (L - i * Bs) : Bs;
-            for (int64_t rr = 0; rr < nrows; ++rr) {
-                int64_t p = i * Bs + rr;                 /* request-local position */
-                int64_t grow = cu[b] + p;
+            int64_t lo = i * Bs > p0 ? i * Bs : p0;                   /* positions of the block's rows */
+            int64_t hi = (i + 1) * Bs < L ? (i + 1) * Bs : L;
+            for (int64_t p = lo; p < hi; ++p) {
+                int64_t grow = cu_q[b] + (p - p0);
                 for (int c = 0; c < d; ++c) qd[c] = (double)q[(grow * Hq + h) * (int64_t)d + c] * qs[h];
                 int64_t n = 0;
                 int64_t nv = 0;
@@ -235,9 +292,11 @@ int orc_attend(const float* q, const float* k, const float* v, const double* qs,
                     int64_t j = idx[t];
                     for (int64_t cc = 0; cc < Bs; ++cc) {
                         int64_t kp = j * Bs + cc;
-                        int visible = MUT(6) ? (kp < p) : (kp <= p);
+                        int visible = MUT(6) ? (kp < p)
+                                    : MUT(12) ? (kp <= p - p0)         /* mutant: chunk-relative mask */
+                                    : (kp <= p);
                         if (kp >= L || !visible) continue;
-                        int64_t krow = cu[b] + kp;
+                        int64_t krow = cu_k[b] + kp;
                         double dot = 0.0;
                         for (int c = 0; c < d; ++c)
                             dot += qd[c] * ((double)k[(krow * Hkv + g) * (int64_t)d + c] * ks[g]);
@@ -251,9 +310,10 @@ int orc_attend(const float* q, const float* k, const float* v, const double* qs,
                     }
                 }
                 if (correction) {
-                    for (int64_t j = 0; j < i; ++j) {
+                    /* mutant 14: the cached prefix's pruned blocks left out */
+                    for (int64_t j = MUT(14) ? i0 : 0; j < i; ++j) {
                         if (kept[j]) continue;
-                        int64_t kb = cb[b] + j;
+                        int64_t kb = cbk[b] + j;
                         int64_t nj = (L - j * Bs) < Bs ? (L - j * Bs) : Bs;
                         double dot = 0.0;
                         for (int c = 0; c < d; ++c) dot += qd[c] * kbar[(kb * Hkv + g) * (int64_t)d + c];
@@ -282,7 +342,9 @@ int orc_attend(const float* q, const float* k, const float* v, const double* qs,
             free(kept); free(lg); free(vrow); free(vbuf); free(qd); free(acc);
         }
     }
-    free(cb);
+    free(P);
+    free(cbq);
+    free(cbk);
     free(req);
     return 0;
 }

@@ -53,13 +53,13 @@ def _load(mutant: int = 0):
         if mutant in _cache:
             return _cache[mutant]
         lib = ctypes.CDLL(build(mutant))
-        lib.orc_total_blocks.argtypes = [_P, _I, _I]
+        lib.orc_total_blocks.argtypes = [_P, _P, _I, _I]
         lib.orc_total_blocks.restype = _L
-        lib.orc_block_means.argtypes = [_P, _P, _P, _I, _I, _I, _I, _P]
+        lib.orc_block_means.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _P]
         lib.orc_block_means.restype = None
-        lib.orc_estimate.argtypes = [_P, _P, _P, _I, _I, _I, _I, _I, _D, _D, _I, _P, _P, _P, _P]
+        lib.orc_estimate.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _I, _D, _D, _I, _P, _P, _P, _P]
         lib.orc_estimate.restype = _I
-        lib.orc_attend.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _D, _P, _P, _I,
+        lib.orc_attend.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _D, _P, _P, _I,
                                    _I, _P, _P, _P, _L, _P, _P, _P]
         lib.orc_attend.restype = _I
         lib.orc_mutant_id.restype = _I
@@ -83,6 +83,18 @@ def _i32(a):
     return np.ascontiguousarray(a, dtype=np.int32)
 
 
+def _i64(a):
+    return None if a is None else np.ascontiguousarray(a, dtype=np.int64)
+
+
+def chunk_starts(cu_seqlens_q, cu_seqlens_k) -> np.ndarray:
+    """D0 chunked form: position P_b = Lk_b - Lq_b of every request's first query row."""
+    lq, lk = np.diff(_i32(cu_seqlens_q)).astype(np.int64), np.diff(_i32(cu_seqlens_k)).astype(np.int64)
+    if lq.shape != lk.shape or (lq < 0).any() or (lq > lk).any():
+        raise ValueError("every request needs 0 <= query rows <= keys")
+    return lk - lq
+
+
 class Oracle:
     """fp64 CPU reference of the estimator (D1, D2) and the attention (D3)."""
 
@@ -91,36 +103,43 @@ class Oracle:
         self.mutant = mutant
 
     # D0
-    def total_blocks(self, cu_seqlens, block_size: int) -> int:
-        cu = _i32(cu_seqlens)
-        return int(self.lib.orc_total_blocks(_ptr(cu), len(cu) - 1, block_size))
+    def total_blocks(self, cu_seqlens, block_size: int, pos0=None) -> int:
+        """Blocks of a batch; request b's rows start at position pos0[b] (None: 0)."""
+        cu, p0 = _i32(cu_seqlens), _i64(pos0)
+        return int(self.lib.orc_total_blocks(_ptr(cu), _ptr(p0), len(cu) - 1, block_size))
 
     # D1
-    def block_means(self, x, cu_seqlens, block_size: int, scale=None) -> np.ndarray:
-        """x: [T, H, d] stored values; scale: [H] dequantisation scales."""
+    def block_means(self, x, cu_seqlens, block_size: int, scale=None, pos0=None) -> np.ndarray:
+        """x: [T, H, d] stored values; scale: [H] dequantisation scales; pos0: [B]
+        position of every request's first row (None: 0; query rows of a chunk:
+        ``chunk_starts(cu_q, cu_k)``)."""
         x = _f32(x)
         T, H, d = x.shape
-        cu = _i32(cu_seqlens)
+        cu, p0 = _i32(cu_seqlens), _i64(pos0)
         sc = _f64(np.ones(H) if scale is None else scale)
-        out = np.zeros((self.total_blocks(cu, block_size), H, d), np.float64)
-        self.lib.orc_block_means(_ptr(x), _ptr(sc), _ptr(cu), len(cu) - 1, H, d, block_size, _ptr(out))
+        out = np.zeros((self.total_blocks(cu, block_size, p0), H, d), np.float64)
+        self.lib.orc_block_means(_ptr(x), _ptr(sc), _ptr(cu), _ptr(p0), len(cu) - 1, H, d, block_size,
+                                 _ptr(out))
         return out
 
     # D1 + D2
     def estimate(self, qbar, kbar, cu_seqlens, block_size: int, alpha: float, tau: float,
-                 nb_max: Optional[int] = None, want_scores: bool = False):
-        """Returns dict(kept_cnt [nb, Hkv], kept_idx [nb, Hkv, nb_max], s, m)."""
+                 nb_max: Optional[int] = None, want_scores: bool = False, cu_seqlens_k=None):
+        """Returns dict(kept_cnt [nb, Hkv], kept_idx [nb, Hkv, nb_max], s, m).
+        ``cu_seqlens`` counts query rows, ``cu_seqlens_k`` keys (None: the same,
+        plain prefill); nb counts q-blocks."""
         qbar, kbar, cu = _f64(qbar), _f64(kbar), _i32(cu_seqlens)
+        cuk = cu if cu_seqlens_k is None else _i32(cu_seqlens_k)
         nblk, Hq, d = qbar.shape
         Hkv = kbar.shape[1]
-        lens = np.diff(cu)
+        lens = np.diff(cuk)
         if nb_max is None:
             nb_max = max(1, int(max([(int(L) + block_size - 1) // block_size for L in lens] or [1])))
         cnt = np.zeros((nblk, Hkv), np.int32)
         idx = np.full((nblk, Hkv, nb_max), -1, np.int32)
         s = np.full((nblk, Hq, nb_max), np.nan) if want_scores else None
         m = np.full((nblk, Hq), np.nan) if want_scores else None
-        rc = self.lib.orc_estimate(_ptr(qbar), _ptr(kbar), _ptr(cu), len(cu) - 1, Hq, Hkv, d,
+        rc = self.lib.orc_estimate(_ptr(qbar), _ptr(kbar), _ptr(cu), _ptr(cuk), len(cu) - 1, Hq, Hkv, d,
                                    block_size, tau, alpha, nb_max, _ptr(cnt), _ptr(idx), _ptr(s), _ptr(m))
         if rc != 0:
             raise ValueError(f"orc_estimate failed: {rc}")
@@ -129,9 +148,12 @@ class Oracle:
     # D3
     def attend(self, q, k, v, cu_seqlens, block_size: int, tau: float, kept_cnt, kept_idx,
                correction: bool = False, kbar=None, vbar=None, q_scale=None, k_scale=None,
-               v_scale=None, sel=None, want_wsum: bool = False):
-        """Returns dict(o [T, Hq, d], lse [T, Hq], wsum). Rows outside ``sel`` stay NaN."""
+               v_scale=None, sel=None, want_wsum: bool = False, cu_seqlens_k=None):
+        """Returns dict(o [T, Hq, d], lse [T, Hq], wsum). Rows outside ``sel`` stay NaN.
+        ``cu_seqlens_k`` (None: ``cu_seqlens``) gives the keys of every request
+        when only its last query rows are computed (D0 chunked form)."""
         q, k, v, cu = _f32(q), _f32(k), _f32(v), _i32(cu_seqlens)
+        cuk = cu if cu_seqlens_k is None else _i32(cu_seqlens_k)
         T, Hq, d = q.shape
         Hkv = k.shape[1]
         kept_cnt, kept_idx = _i32(kept_cnt), _i32(kept_idx)
@@ -146,7 +168,7 @@ class Oracle:
         ws = np.full((T, Hq), np.nan) if want_wsum else None
         selv = None if sel is None else np.ascontiguousarray(sel, dtype=np.int64)
         rc = self.lib.orc_attend(_ptr(q), _ptr(k), _ptr(v), _ptr(qs), _ptr(ks), _ptr(vs), _ptr(cu),
-                                 len(cu) - 1, Hq, Hkv, d, block_size, tau, _ptr(kept_cnt),
+                                 _ptr(cuk), len(cu) - 1, Hq, Hkv, d, block_size, tau, _ptr(kept_cnt),
                                  _ptr(kept_idx), nb_max, 1 if correction else 0,
                                  _ptr(kbar) if correction else None, _ptr(vbar) if correction else None,
                                  _ptr(selv), 0 if selv is None else len(selv), _ptr(o), _ptr(lse), _ptr(ws))

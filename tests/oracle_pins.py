@@ -18,6 +18,11 @@ What pins what (definitions D0-D4 in the oracle header):
   gqa_packing       D2/D3 head -> group map: packed heads = each head alone
   ragged            D0 ragged batch (an empty request included) = each request alone
   e4m3_scales       D4 dequantisation: codes x power-of-two scale = scaled values
+  chunk_dense_sdpa  D0 chunked form (the last Lq of Lk tokens), alpha <= 0: torch SDPA
+                    with an explicit bottom-right causal mask
+  chunk_equals_full D0 chunked form: a block-aligned chunk = the full prefill's rows
+  chunk_bilinearity D0/D1 chunked form: a partial first q-block's score = mean logit
+  chunk_exact_correction  D3 on chunks, the cached prefix's pruned blocks included
 """
 from __future__ import annotations
 
@@ -305,5 +310,176 @@ def pin_e4m3_scales(orc):
     assert np.abs(a["o"] - b["o"]).max() < 1e-12, "e4m3 dequantisation differs from scaled values"
 
 
+# ---------------------------------------------------------------------------
+# chunked prefill (D0 chunked form): the last Lq_b of Lk_b tokens are the
+# queries, at positions P_b = Lk_b - Lq_b onwards; q-blocks keep the absolute
+# grid of the request
+# ---------------------------------------------------------------------------
+def _chunk_of(q_full, cu_k, lq):
+    """The query rows of a chunk: the last lq[b] rows of every request."""
+    parts = [q_full[int(cu_k[b + 1]) - n:int(cu_k[b + 1])] for b, n in enumerate(lq)]
+    cu_q = np.concatenate([[0], np.cumsum(lq)]).astype(np.int32)
+    return np.ascontiguousarray(np.concatenate(parts)), cu_q
+
+
+def _chunk_means(orc, q, k, v, cu_q, cu_k):
+    from oracle.oracle import chunk_starts
+    p0 = chunk_starts(cu_q, cu_k)
+    return (orc.block_means(q, cu_q, 128, pos0=p0), orc.block_means(k, cu_k, 128),
+            orc.block_means(v, cu_k, 128), p0)
+
+
+def _sdpa_chunk(q, k, v, cu_q, cu_k, hq, hkv):
+    """Dense attention of the chunk rows with torch (fp64), GQA expanded: query t
+    of request b sits at position P_b + t and sees keys c <= P_b + t (an
+    explicit boolean mask, since torch's is_causal aligns the mask top-left)."""
+    g = hq // hkv
+    outs, lses = [], []
+    for b in range(len(cu_q) - 1):
+        qs_, qe, ks_, ke = int(cu_q[b]), int(cu_q[b + 1]), int(cu_k[b]), int(cu_k[b + 1])
+        lq, lk = qe - qs_, ke - ks_
+        if lq == 0:
+            continue
+        mask = torch.arange(lk)[None, :] <= (lk - lq + torch.arange(lq))[:, None]
+        qt = torch.from_numpy(q[qs_:qe]).double().permute(1, 0, 2)
+        kt = torch.from_numpy(k[ks_:ke]).double().repeat_interleave(g, dim=1).permute(1, 0, 2)
+        vt = torch.from_numpy(v[ks_:ke]).double().repeat_interleave(g, dim=1).permute(1, 0, 2)
+        o = torch.nn.functional.scaled_dot_product_attention(qt[None], kt[None], vt[None], attn_mask=mask,
+                                                             scale=TAU)[0]
+        logits = (qt @ kt.transpose(1, 2)) * TAU
+        lse = torch.logsumexp(logits.masked_fill(~mask, -math.inf), dim=-1)
+        outs.append(o.permute(1, 0, 2).numpy())
+        lses.append(lse.permute(1, 0).numpy())
+    return np.concatenate(outs), np.concatenate(lses)
+
+
+def _prefix_pruned(est, p0, lq, lk, hkv):
+    """True when some q-block of a chunk drops a key block of the cached prefix."""
+    t = 0
+    for b in range(len(lq)):
+        if lq[b] == 0:
+            continue
+        i0 = int(p0[b]) // 128
+        for i in range(i0, (lk[b] + 127) // 128):
+            for g in range(hkv):
+                kept = set(est["kept_idx"][t, g, :est["kept_cnt"][t, g]].tolist())
+                if any(j not in kept for j in range(i0)):
+                    return True
+            t += 1
+    return False
+
+
+def pin_chunk_dense_sdpa(orc):
+    lk = [700, 700, 129, 256, 383, 300, 700]
+    lq = [700, 572, 1, 0, 255, 299, 500]      # P = 0, 128, 128, -, 128, 1, 200
+    hq, hkv = 4, 2
+    q_full, k, v, cu_k = _rand_inputs(lk, hq, hkv, seed=71)
+    q, cu_q = _chunk_of(q_full, cu_k, lq)
+    qb, kb, vb, p0 = _chunk_means(orc, q, k, v, cu_q, cu_k)
+    est = orc.estimate(qb, kb, cu_q, 128, alpha=0.0, tau=TAU, cu_seqlens_k=cu_k)
+    ref_o, ref_lse = _sdpa_chunk(q, k, v, cu_q, cu_k, hq, hkv)
+    for corr in (False, True):
+        r = orc.attend(q, k, v, cu_q, 128, TAU, est["kept_cnt"], est["kept_idx"], correction=corr,
+                       kbar=kb, vbar=vb, cu_seqlens_k=cu_k)
+        assert np.abs(r["o"] - ref_o).max() < 1e-12, "chunk output differs from dense masked SDPA"
+        assert np.abs(r["lse"] - ref_lse).max() < 1e-12, "chunk LSE differs from torch.logsumexp"
+
+
+def pin_chunk_equals_full(orc):
+    """A chunk that starts on a block boundary has the full prefill's q-blocks, so
+    its block means, kept lists, outputs and LSE are the full prefill's rows."""
+    lk = [1000, 640, 385]
+    lq = [744, 256, 385]                      # P = 256, 384, 0
+    wl = _structured(lk, seed=81)
+    q_full, k, v = wl.float_inputs()
+    cu_k = wl.cu_seqlens
+    q, cu_q = _chunk_of(q_full, cu_k, lq)
+    qb, kb, vb, p0 = _chunk_means(orc, q, k, v, cu_q, cu_k)
+    assert (p0 % 128 == 0).all()
+    qb_full = orc.block_means(q_full, cu_k, 128)
+    ef = orc.estimate(qb_full, kb, cu_k, 128, alpha=0.2, tau=TAU)
+    ec = orc.estimate(qb, kb, cu_q, 128, alpha=0.2, tau=TAU, cu_seqlens_k=cu_k, nb_max=ef["nb_max"])
+    assert _prefix_pruned(ec, p0, lq, lk, 2), "case prunes no prefix block"
+    full = orc.attend(q_full, k, v, cu_k, 128, TAU, ef["kept_cnt"], ef["kept_idx"], correction=True,
+                      kbar=kb, vbar=vb)
+    ch = orc.attend(q, k, v, cu_q, 128, TAU, ec["kept_cnt"], ec["kept_idx"], correction=True, kbar=kb,
+                    vbar=vb, cu_seqlens_k=cu_k)
+    tf = tc = 0
+    for b in range(len(lk)):
+        nbk, i0 = (lk[b] + 127) // 128, int(p0[b]) // 128
+        n = nbk - i0
+        for key, a, c in (("qbar", qb_full, qb), ("kept_cnt", ef["kept_cnt"], ec["kept_cnt"]),
+                          ("kept_idx", ef["kept_idx"], ec["kept_idx"])):
+            assert np.array_equal(c[tc:tc + n], a[tf + i0:tf + nbk]), f"chunk {key} differs from full prefill"
+        rows_f = slice(int(cu_k[b]) + int(p0[b]), int(cu_k[b + 1]))
+        rows_c = slice(int(cu_q[b]), int(cu_q[b + 1]))
+        assert np.array_equal(ch["o"][rows_c], full["o"][rows_f]), "chunk rows differ from full prefill"
+        assert np.array_equal(ch["lse"][rows_c], full["lse"][rows_f])
+        tf += nbk
+        tc += n
+
+
+def pin_chunk_bilinearity(orc):
+    """Chunks whose first q-block is partial: the block score is the mean token
+    logit over the query rows that block holds and every key of block j."""
+    lk = [700, 300]
+    lq = [500, 45]                            # P = 200 (56 rows in block 1), 255 (1 row in block 1)
+    hq, hkv = 4, 2
+    q_full, k, v, cu_k = _rand_inputs(lk, hq, hkv, seed=91)
+    q, cu_q = _chunk_of(q_full, cu_k, lq)
+    qb, kb, vb, p0 = _chunk_means(orc, q, k, v, cu_q, cu_k)
+    est = orc.estimate(qb, kb, cu_q, 128, alpha=0.1, tau=TAU, cu_seqlens_k=cu_k, want_scores=True)
+    s = est["s"]
+    t = 0
+    for b in range(len(lk)):
+        P, L = int(p0[b]), lk[b]
+        qq = torch.from_numpy(q[cu_q[b]:cu_q[b + 1]]).double()
+        kk = torch.from_numpy(k[cu_k[b]:cu_k[b + 1]]).double()
+        for i in range(P // 128, (L + 127) // 128):
+            lo, hi = max(P, i * 128), min(L, (i + 1) * 128)
+            for h in range(hq):
+                g = h // (hq // hkv)
+                logits = (qq[lo - P:hi - P, h, :] @ kk[:, g, :].T * TAU).numpy()
+                for j in range(i + 1):
+                    blk = logits[:, j * 128:min(L, (j + 1) * 128)]
+                    assert abs(s[t, h, j] - blk.mean()) < 1e-12, "chunk score is not the mean block logit"
+            t += 1
+    assert t == s.shape[0]
+
+
+def pin_chunk_exact_correction(orc):
+    """Block-constant K and V under chunks: the corrected output equals dense
+    attention with the bottom-right causal mask for any alpha, the pruned
+    blocks of the cached prefix included."""
+    lk = [1024, 700]
+    lq = [600, 572]                           # P = 424 (unaligned), 128
+    hq, hkv = 4, 2
+    rng = np.random.default_rng(101)
+    T = sum(lk)
+    q_full = (rng.standard_normal((T, hq, 128)) + rng.standard_normal((1, hq, 128))).astype(np.float32)
+    k = np.zeros((T, hkv, 128), np.float32)
+    v = np.zeros((T, hkv, 128), np.float32)
+    cu_k = np.array([0, lk[0], T], np.int32)
+    for b, L in enumerate(lk):
+        for j in range((L + 127) // 128):
+            s0, e0 = cu_k[b] + j * 128, cu_k[b] + min(L, (j + 1) * 128)
+            k[s0:e0] = (rng.standard_normal((hkv, 128)) * 1.5).astype(np.float32)
+            v[s0:e0] = rng.standard_normal((hkv, 128)).astype(np.float32)
+    q, cu_q = _chunk_of(q_full, cu_k, lq)
+    qb, kb, vb, p0 = _chunk_means(orc, q, k, v, cu_q, cu_k)
+    ref_o, ref_lse = _sdpa_chunk(q, k, v, cu_q, cu_k, hq, hkv)
+    for a in (0.3, 0.9):
+        est = orc.estimate(qb, kb, cu_q, 128, alpha=a, tau=TAU, cu_seqlens_k=cu_k)
+        assert _prefix_pruned(est, p0, lq, lk, hkv), "case prunes no prefix block"
+        r = orc.attend(q, k, v, cu_q, 128, TAU, est["kept_cnt"], est["kept_idx"], correction=True, kbar=kb,
+                       vbar=vb, cu_seqlens_k=cu_k)
+        assert np.abs(r["o"] - ref_o).max() < 1e-11, "chunk mean correction is not exact on block-constant K/V"
+        assert np.abs(r["lse"] - ref_lse).max() < 1e-11
+        r0 = orc.attend(q, k, v, cu_q, 128, TAU, est["kept_cnt"], est["kept_idx"], correction=False,
+                        cu_seqlens_k=cu_k)
+        assert np.abs(r0["o"] - ref_o).max() > 1e-3, "pruning had no effect"
+
+
 ALL_PINS = [pin_dense_sdpa, pin_means_numpy, pin_bilinearity, pin_threshold_golden, pin_diagonal_kept,
-            pin_nesting, pin_weights_sum, pin_exact_correction, pin_gqa_packing, pin_ragged, pin_e4m3_scales]
+            pin_nesting, pin_weights_sum, pin_exact_correction, pin_gqa_packing, pin_ragged, pin_e4m3_scales,
+            pin_chunk_dense_sdpa, pin_chunk_equals_full, pin_chunk_bilinearity, pin_chunk_exact_correction]

@@ -17,6 +17,9 @@ MUTANTS = {
     9: "mean key used as the correction value",
     10: "value scale ignored",
     11: "LSE without the row max",
+    12: "chunk: causal mask relative to the chunk start, not the position",
+    13: "chunk: partial first q-block mean divided by rows before the chunk too",
+    14: "chunk: pruned blocks of the cached prefix get no correction",
 }
 
 
