@@ -162,6 +162,23 @@ bool score_tiling(int32_t G, int32_t* qt) {
     return true;
 }
 
+// Size limits of the kernels, checked before anything is enqueued: the setup
+// kernel's per-index histogram and the attention kernel's per-item kept-list
+// staging live in shared memory, and the score kernel's grid has at most 65535
+// tiles in y.
+fp2_status check_limits(const fp2_params* p, const Problem& pr, bool estimate, bool attention) {
+    const int32_t nb_cap = pr.nb_need > 0 ? pr.nb_need : 1;
+    if (sizeof(int32_t) * (nb_cap + 1) > kMaxSmem) return FP2_ERR_UNSUPPORTED;
+    if (estimate) {
+        int32_t qt;
+        if (!score_tiling(p->num_q_heads / p->num_kv_heads, &qt)) return FP2_ERR_UNSUPPORTED;
+        if ((pr.max_blocks + qt - 1) / qt + pr.batch > 65535) return FP2_ERR_UNSUPPORTED;
+    }
+    if (attention && attn_smem_bytes(p->dtype == FP2_E4M3, pr.nb_need) > kMaxSmem)
+        return FP2_ERR_UNSUPPORTED;
+    return FP2_OK;
+}
+
 fp2_status run_setup(const Problem& pr, void* ws, const int32_t* cu, int32_t qt, bool paged,
                      int32_t mbps, int64_t meta_blocks, cudaStream_t s) {
     SetupArgs sa;
@@ -194,9 +211,11 @@ fp2_status run_estimate(const fp2_params* p, const void* q, const void* k, const
                         int32_t mbps, int32_t num_pages, fp2_blockmeta* meta, void* ws,
                         cudaStream_t s) {
     const int32_t G = p->num_q_heads / p->num_kv_heads;
+    fp2_status st = check_limits(p, pr, true, false);
+    if (st != FP2_OK) return st;
     int32_t qt;
-    if (!score_tiling(G, &qt)) return FP2_ERR_UNSUPPORTED;
-    fp2_status st = run_setup(pr, ws, cu, qt, block_table != nullptr, mbps, meta->max_blocks, s);
+    score_tiling(G, &qt);
+    st = run_setup(pr, ws, cu, qt, block_table != nullptr, mbps, meta->max_blocks, s);
     // an empty batch (no requests, or only empty ones) ends after the setup
     // kernel has checked cu_seqlens: there is no block to pool or score
     if (st != FP2_OK || pr.batch == 0 || pr.total_tokens == 0) return st;
@@ -289,8 +308,7 @@ fp2_status run_estimate(const fp2_params* p, const void* q, const void* k, const
     if (cudaFuncSetAttribute(score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess)
         return FP2_ERR_CUDA;
-    const int64_t tiles = (pr.max_blocks + qt - 1) / qt + pr.batch;
-    if (tiles > 65535) return FP2_ERR_UNSUPPORTED;
+    const int64_t tiles = (pr.max_blocks + qt - 1) / qt + pr.batch;  // <= 65535 (check_limits)
     score_kernel<<<dim3(static_cast<unsigned>(p->num_kv_heads), static_cast<unsigned>(tiles)),
                    kScoreThreads, smem, s>>>(sa, tqh, tql, tkh, tkl);
     return launched(cudaGetLastError());
@@ -301,8 +319,8 @@ fp2_status run_attention(const fp2_params* p, const void* q, const void* k, cons
                          int32_t mbps, int32_t num_pages, const fp2_blockmeta* meta, void* out,
                          float* lse, void* ws, cudaStream_t s, bool need_setup) {
     const bool e4m3 = p->dtype == FP2_E4M3;
-    if (attn_smem_bytes(e4m3, pr.nb_need) > kMaxSmem) return FP2_ERR_UNSUPPORTED;
-    fp2_status st = FP2_OK;
+    fp2_status st = check_limits(p, pr, false, true);
+    if (st != FP2_OK) return st;
     if (need_setup) {
         st = run_setup(pr, ws, cu, 1, block_table != nullptr, mbps, meta->max_blocks, s);
         if (st != FP2_OK) return st;
@@ -432,6 +450,8 @@ fp2_status fp2_prefill_paged(const fp2_params* params, const void* q, const void
     if (int64_t(num_pages) * kBlock > (int64_t(1) << 31) - 1) return FP2_ERR_UNSUPPORTED;
     if (total_tokens > 0 && (!out || !aligned(out, 16))) return FP2_ERR_INVALID_ARG;
     if (lse && !aligned(lse, 4)) return FP2_ERR_INVALID_ARG;
+    // the attention's limits too, before the estimator is enqueued
+    if ((st = check_limits(params, pr, true, true)) != FP2_OK) return st;
     const cudaStream_t s = static_cast<cudaStream_t>(stream);
     if ((st = run_estimate(params, q, k_pool, v_pool, cu_seqlens, pr, block_table, max_blocks_per_seq,
                            num_pages, meta, workspace, s)) != FP2_OK)

@@ -146,7 +146,14 @@ fp2_status fp2_estimate(const fp2_params* params, const void* q, const void* k, 
 
 /* Sparse attention over the kept blocks of `meta` (from fp2_estimate on the
  * same inputs) with contiguous K/V, plus the mean correction when
- * params->correction != 0.  Writes out (bf16) and, when non-NULL, lse. */
+ * params->correction != 0.  Writes out (bf16) and, when non-NULL, lse.
+ * Length limit of the attention calls (this one, fp2_prefill_paged and
+ * fp2_sparse_prefill_noalloc): a work item keeps its kept-block list in shared
+ * memory, so ceil(max_seqlen / block_size) may be at most FP2_MAX_SEQ_BLOCKS_BF16
+ * (4133 blocks, 529024 tokens) for bf16 and FP2_MAX_SEQ_BLOCKS_E4M3 (8075
+ * blocks, 1033600 tokens) for e4m3; longer returns FP2_ERR_UNSUPPORTED. */
+#define FP2_MAX_SEQ_BLOCKS_BF16 4133
+#define FP2_MAX_SEQ_BLOCKS_E4M3 8075
 fp2_status fp2_sparse_prefill(const fp2_params* params, const void* q, const void* k,
                               const void* v, const int32_t* cu_seqlens, int32_t batch,
                               int64_t total_tokens, int32_t max_seqlen,

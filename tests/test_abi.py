@@ -171,6 +171,7 @@ def test_prototypes_match_the_ctypes_declarations(lib):
     """Each header prototype: ctypes declares as many arguments, each pointer as a
     pointer and each integer with the C width, and the matching result type."""
     text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    text = re.sub(r"^\s*#.*$", "", text, flags=re.M)          # preprocessor lines
     protos = re.findall(r"([A-Za-z_][\w\s\*]*?)\b(fp2_[a-z_]+)\s*\(([^)]*)\)\s*;", text)
     assert {name for _, name, _ in protos} == set(_lib.EXPORTS)
     for ret, name, args in protos:
@@ -190,3 +191,42 @@ def test_prototypes_match_the_ctypes_declarations(lib):
             assert fn.restype is ctypes.c_char_p, name
         else:
             assert ctypes.sizeof(fn.restype) == rwidth, name
+
+
+def _max_seq_blocks():
+    text = open(HEADER).read()
+    return {name: int(re.search(rf"#define FP2_MAX_SEQ_BLOCKS_{name}\s+(\d+)", text).group(1))
+            for name in ("BF16", "E4M3")}
+
+
+def _attention_call(lib, fn, dtype, max_seqlen):
+    """An attention call with fake (never dereferenced) device addresses."""
+    sc = 4096 if dtype else None
+    p = _lib.fp2_params(32, 8, 128, 128, 0.05, 0.0, 1, dtype, sc, sc, sc)
+    nb = (max_seqlen + 127) // 128
+    m = _lib.fp2_blockmeta(4096, 4096, 4096, 4096, None, nb, nb + 1)
+    a = ctypes.c_void_p(4096)
+    if fn == "fp2_prefill_paged":
+        return lib.fp2_prefill_paged(ctypes.byref(p), a, a, a, a, 1, max_seqlen, max_seqlen, a, nb, nb,
+                                     ctypes.byref(m), a, None, ctypes.c_void_p(1 << 20), 1 << 40, None)
+    return lib.fp2_sparse_prefill(ctypes.byref(p), a, a, a, a, 1, max_seqlen, max_seqlen, ctypes.byref(m),
+                                  a, None, ctypes.c_void_p(1 << 20), 1 << 40, None)
+
+
+@pytest.mark.parametrize("fn", ["fp2_sparse_prefill", "fp2_prefill_paged"])
+@pytest.mark.parametrize("dtype,name", [(0, "BF16"), (1, "E4M3")])
+def test_length_limit_rejected_before_any_launch(lib, fn, dtype, name):
+    """One block past the documented limit returns FP2_ERR_UNSUPPORTED, and the
+    paged call returns it before enqueueing its estimator."""
+    limit = _max_seq_blocks()[name]
+    assert _attention_call(lib, fn, dtype, limit * 128 + 1) == 2
+
+
+@pytest.mark.skipif(__import__("torch").cuda.is_available(),
+                    reason="the accepted call would launch kernels on fake addresses")
+@pytest.mark.parametrize("dtype,name", [(0, "BF16"), (1, "E4M3")])
+def test_length_limit_is_tight(lib, dtype, name):
+    """At the documented limit every host check passes: without a GPU the call
+    gets as far as the first CUDA call and returns FP2_ERR_CUDA."""
+    limit = _max_seq_blocks()[name]
+    assert _attention_call(lib, "fp2_sparse_prefill", dtype, limit * 128) == 4
