@@ -235,6 +235,108 @@ def time_layer(st, wl, steps, warmup, dist_ctx, clocks=None):
     return total, est, att, clk
 
 
+def dense_causal_flops(seqlens, hq, d=128):
+    """4*d flops per causal query-key pair, summed over the requests and query heads."""
+    return 4.0 * d * hq * sum(L * (L + 1) / 2 for L in seqlens)
+
+
+def comparators(wl, dev, ms_layer, reps=5):
+    """Context for the pages' speedup ratios on this GPU and this layer: dense causal
+    attention by this library (alpha = 0 keeps every causal block, so both calls run with
+    nothing pruned), by torch's scaled_dot_product_attention for each backend that accepts
+    the layer, and by flash_attn where it runs here.  Each is timed with CUDA events (3
+    warm-up calls, then `reps`); `speedup` = its time over the sparse layer's.  A comparator
+    that fails reports its error and does not stop the others."""
+    import dataclasses
+    import torch
+    import torch.nn.functional as F
+    import block_sparse_prefill_b200 as fp2
+    T, hq, hkv, d = wl.total_tokens, wl.num_q_heads, wl.num_kv_heads, 128
+    flops = dense_causal_flops(wl.seqlens, hq, d)
+    stream = torch.cuda.current_stream()
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / reps
+
+    def entry(ms, note):
+        return {"ms": ms, "tflops_dense_work": flops / (ms * 1e-3) / 1e12, "speedup_of_sparse_layer": ms / ms_layer,
+                "note": note}
+
+    def failed(e):
+        return {"error": f"{type(e).__name__}: {e}"[:300]}
+
+    res = {"work": "dense causal attention of the same layer, 4*d flops per causal query-key pair",
+           "dense_tflop": flops / 1e12, "sparse_layer_ms": ms_layer, "reps": reps}
+    st = setup_layer(wl, dev)
+    try:
+        p0 = dataclasses.replace(st["params"], alpha=0.0)
+        meta0 = fp2.BlockMeta.empty(p0, wl.batch, T, wl.max_seqlen, dev)
+
+        def ours_dense():
+            fp2.estimate(p0, st["q"], st["k"], st["v"], st["cu"], wl.max_seqlen, meta0, st["ws"], stream=stream)
+            fp2.sparse_prefill(p0, st["q"], st["k"], st["v"], st["cu"], wl.max_seqlen, meta0, st["out"], st["ws"],
+                               lse=st["lse"], stream=stream)
+        ms = timed(ours_dense)
+        err = fp2.get_error(st["ws"])
+        res["ours_alpha0"] = (entry(ms, "this library at alpha = 0 (estimator + attention, every causal block)")
+                              if err == 0 else {"error": fp2.status_string(err)})
+        del meta0
+    except Exception as e:  # noqa: BLE001 - context only: report and go on
+        res["ours_alpha0"] = failed(e)
+    if wl.batch == 1:
+        try:
+            from torch.nn.attention import SDPBackend, sdpa_kernel
+            qt = st["q"].permute(1, 0, 2).unsqueeze(0).contiguous()      # [1, Hq, T, d]
+            kt = st["k"].permute(1, 0, 2).unsqueeze(0).contiguous()      # [1, Hkv, T, d]
+            vt = st["v"].permute(1, 0, 2).unsqueeze(0).contiguous()
+            kx = vx = None
+            for name in ("CUDNN_ATTENTION", "FLASH_ATTENTION", "EFFICIENT_ATTENTION"):
+                backend = getattr(SDPBackend, name, None)
+                if backend is None:
+                    continue
+                key = "torch_sdpa_" + name.split("_")[0].lower()
+                try:
+                    with sdpa_kernel([backend]):
+                        try:
+                            F.scaled_dot_product_attention(qt[:, :, :128], kt[:, :, :128], vt[:, :, :128],
+                                                           is_causal=True, enable_gqa=True)
+                            ms = timed(lambda: F.scaled_dot_product_attention(qt, kt, vt, is_causal=True,
+                                                                              enable_gqa=True))
+                            res[key] = entry(ms, f"torch {torch.__version__} SDPA {name}, is_causal, enable_gqa")
+                        except RuntimeError:
+                            if kx is None:
+                                kx = kt.repeat_interleave(hq // hkv, dim=1)
+                                vx = vt.repeat_interleave(hq // hkv, dim=1)
+                            ms = timed(lambda: F.scaled_dot_product_attention(qt, kx, vx, is_causal=True))
+                            res[key] = entry(ms, f"torch {torch.__version__} SDPA {name}, is_causal, K/V "
+                                                 "expanded to the query heads")
+                except Exception as e:  # noqa: BLE001
+                    res[key] = failed(e)
+            del qt, kt, vt, kx, vx
+        except Exception as e:  # noqa: BLE001
+            res["torch_sdpa"] = failed(e)
+    try:
+        import flash_attn
+        from flash_attn import flash_attn_varlen_func
+        ms = timed(lambda: flash_attn_varlen_func(st["q"], st["k"], st["v"], st["cu"], st["cu"], wl.max_seqlen,
+                                                  wl.max_seqlen, causal=True))
+        res["flash_attn"] = entry(ms, f"flash_attn {flash_attn.__version__} varlen, causal, native GQA")
+    except Exception as e:  # noqa: BLE001
+        res["flash_attn"] = failed(e)
+    del st
+    torch.cuda.empty_cache()
+    return res
+
+
 def approximation_error(st, wl, n_rows=256, seed=7):
     """The method's approximation quality (not a parity check): the block-sparse output of the
     layer against dense causal softmax attention, computed in fp64 on the GPU with torch, on
@@ -512,6 +614,12 @@ def ours(args):
         }
         del st8
 
+    # dense comparators (context only), after every timed measurement above
+    comp = None
+    if args.comparators and ctx.world == 1:
+        torch.cuda.empty_cache()
+        comp = comparators(wl, dev, ms_step)
+
     # roofline of the dominant kernel (the attention call: attention kernel +
     # two small set-up launches) and the estimator (HBM)
     ach_att = (flops + corr_flops) / (ms_att * 1e-3) / 1e12
@@ -568,6 +676,8 @@ def ours(args):
         "fp8": fp8,
         "approximation_vs_dense": approx,
     }
+    if comp is not None:
+        line["comparators"] = comp
     if ctx.rank == 0 and ctx.world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl)
     if ctx.rank == 0:
@@ -615,6 +725,9 @@ def main():
     ap.add_argument("--no-fp8", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--comparators", action="store_true",
+                    help="also time dense attention of the same layer (this library at alpha = 0, torch SDPA, "
+                         "flash_attn) as context for the speedup")
     ap.add_argument("--seqlen", type=int, default=None,
                     help="shorter sequence for profiling runs (default: the 128K workload)")
     args = ap.parse_args()

@@ -92,3 +92,24 @@ def test_layer_work_matches_brute_force():
                 kept_idx[t, g, :len(js)] = js
             t += 1
     assert bench.layer_work(seqlens, kept_cnt, kept_idx, hq, hkv) == _brute_work(seqlens, kept_cnt, kept_idx, hq, hkv)
+
+
+def test_dense_flops_equal_layer_work_with_every_block_kept():
+    """The comparators' dense work and the layer's kept-pair work agree when
+    nothing is pruned (the diagonal block counted causally)."""
+    seqlens = [1, 127, 128, 129, 700, 1000]
+    hq, hkv = 8, 2
+    nbs = [(L + 127) // 128 for L in seqlens]
+    nb_max = max(nbs)
+    rows = sum(nbs)
+    cnt = np.zeros((rows, hkv), np.int32)
+    idx = np.full((rows, hkv, nb_max), -1, np.int32)
+    t = 0
+    for nb in nbs:
+        for i in range(nb):
+            cnt[t] = i + 1
+            idx[t, :, :i + 1] = np.arange(i + 1)
+            t += 1
+    flops, corr = bench.layer_work(seqlens, cnt, idx, hq, hkv)
+    assert corr == 0.0
+    assert flops == bench.dense_causal_flops(seqlens, hq)
