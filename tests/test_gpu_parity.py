@@ -52,6 +52,23 @@ def test_tiny_config(correction):
     _check_outputs(wl, g, correction)
 
 
+@pytest.mark.parametrize("paged", [False, True])
+def test_empty_requests_in_a_batch(paged):
+    """Empty requests first, in the middle and last get no blocks; the others
+    match the oracle as in any ragged batch."""
+    wl = make_workload([0, 300, 0, 200, 129, 0], 8, 2, alpha=0.1, seed=17, n_retrieval=1, paged=paged)
+    g = run_gpu(wl, paged=paged)
+    _check_masks(wl, g)
+    _check_outputs(wl, g, True)
+
+
+def test_all_requests_empty():
+    """total_tokens == 0: the call checks cu_seqlens, writes nothing and reports no error."""
+    wl = make_workload([0, 0], 4, 2, alpha=0.1, seed=18)
+    g = run_gpu(wl)
+    assert g["o"].shape[0] == 0 and g["kept_cnt"].shape[0] == 0
+
+
 def test_dense_alpha_zero():
     wl = make_workload([1000, 300], 4, 2, alpha=0.0, seed=3)
     g = run_gpu(wl, alpha=0.0)
