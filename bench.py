@@ -243,8 +243,8 @@ def dense_causal_flops(seqlens, hq, d=128):
 def comparators(wl, dev, ms_layer, reps=5):
     """Context for the pages' speedup ratios on this GPU and this layer: dense causal
     attention by this library (alpha = 0 keeps every causal block, so both calls run with
-    nothing pruned), by torch's scaled_dot_product_attention for each backend that accepts
-    the layer, and by flash_attn where it runs here.  Each is timed with CUDA events (3
+    nothing pruned), by torch's scaled_dot_product_attention with its cuDNN and flash
+    backends, and by flash_attn where it runs here.  Each is timed with CUDA events (3
     warm-up calls, then `reps`); `speedup` = its time over the sparse layer's.  A comparator
     that fails reports its error and does not stop the others."""
     import dataclasses
@@ -299,7 +299,7 @@ def comparators(wl, dev, ms_layer, reps=5):
             kt = st["k"].permute(1, 0, 2).unsqueeze(0).contiguous()      # [1, Hkv, T, d]
             vt = st["v"].permute(1, 0, 2).unsqueeze(0).contiguous()
             kx = vx = None
-            for name in ("CUDNN_ATTENTION", "FLASH_ATTENTION", "EFFICIENT_ATTENTION"):
+            for name in ("CUDNN_ATTENTION", "FLASH_ATTENTION"):
                 backend = getattr(SDPBackend, name, None)
                 if backend is None:
                     continue
@@ -616,7 +616,7 @@ def ours(args):
 
     # dense comparators (context only), after every timed measurement above
     comp = None
-    if args.comparators and ctx.world == 1:
+    if not args.no_comparators and ctx.world == 1:
         torch.cuda.empty_cache()
         comp = comparators(wl, dev, ms_step)
 
@@ -725,9 +725,9 @@ def main():
     ap.add_argument("--no-fp8", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--comparators", action="store_true",
-                    help="also time dense attention of the same layer (this library at alpha = 0, torch SDPA, "
-                         "flash_attn) as context for the speedup")
+    ap.add_argument("--no-comparators", action="store_true",
+                    help="skip the dense attention of the same layer (this library at alpha = 0, torch SDPA, "
+                         "flash_attn), timed as context for the speedup at 1 GPU")
     ap.add_argument("--seqlen", type=int, default=None,
                     help="shorter sequence for profiling runs (default: the 128K workload)")
     args = ap.parse_args()
