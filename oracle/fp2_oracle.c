@@ -46,6 +46,15 @@
  *               key and mean value).  LSE = ln(denominator).
  *   D4 e4m3     inputs are codes times a per-(tensor, head) scale; the oracle
  *               dequantises them exactly in double.
+ *   D3 variants (not the method as the pages give it; compared on approximation
+ *               error only): correction mode 2 adds the Gaussian second-order
+ *               term to every pruned block's logit, lbar_j + (tau^2 / 2)
+ *               sum_c q_c^2 var_j[c], with var_j the per-dimension key variance
+ *               inside block j (the logit variance when the dimensions are
+ *               uncorrelated inside the block; by Jensen the plain form
+ *               undercounts a block's mass by about e^{var / 2}).  Mode 3 uses the
+ *               block-pooled logit tau qbar_i . kbar_j, shared by all rows of
+ *               q-block i, instead of the row's own.
  *
  * Build with -DORC_MUTANT=n to plant one deliberate mistake (see the MUT()
  * sites); the oracle self-tests check that every such mistake is caught.
@@ -124,6 +133,40 @@ void orc_block_means(const float* x, const double* scale, const int32_t* cu, con
                         s += (double)x[(row * H + h) * (int64_t)d + c] * scale[h];
                     }
                     out[((cb[b] + t) * H + h) * (int64_t)d + c] = s / denom;
+                }
+            }
+        }
+    }
+    free(cb);
+}
+
+/* Per-dimension variance of the dequantised rows inside every block, around the
+ * block means `mean` (from orc_block_means with the same arguments):
+ * out[t, h, c] = (1/n) sum_{r in t} (x[r, h, c] * scale[h] - mean[t, h, c])^2. */
+void orc_block_vars(const float* x, const double* scale, const int32_t* cu, const int64_t* pos0,
+                    int B, int H, int d, int Bs, const double* mean, double* out) {
+    int64_t* cb = (int64_t*)malloc(sizeof(int64_t) * (B + 1));
+    block_offsets(cu, pos0, B, Bs, cb);
+    for (int b = 0; b < B; ++b) {
+        int64_t L = cu[b + 1] - cu[b];
+        int64_t p0 = pos0 ? pos0[b] : 0;
+        int64_t i0 = first_block(p0, Bs);
+        int64_t nb = blocks_at(p0, L, Bs);
+#pragma omp parallel for schedule(static)
+        for (int64_t t = 0; t < nb; ++t) {
+            int64_t i = i0 + t;
+            int64_t lo = i * Bs > p0 ? i * Bs : p0;
+            int64_t hi = (i + 1) * Bs < p0 + L ? (i + 1) * Bs : p0 + L;
+            for (int h = 0; h < H; ++h) {
+                for (int c = 0; c < d; ++c) {
+                    int64_t at = ((cb[b] + t) * H + h) * (int64_t)d + c;
+                    double s = 0.0;
+                    for (int64_t p = lo; p < hi; ++p) {
+                        int64_t row = cu[b] + (p - p0);
+                        double e = (double)x[(row * H + h) * (int64_t)d + c] * scale[h] - mean[at];
+                        s += e * e;
+                    }
+                    out[at] = s / (double)(hi - lo);
                 }
             }
         }
@@ -225,16 +268,22 @@ static int list_ok(const int32_t* idx, int32_t cnt, int64_t i) {
  *   q [Tq, Hq, d], k/v [Tk, Hkv, d] stored values; qs/ks/vs per-head scales;
  *   cu_q / cu_k: query rows and keys of every request (D0 chunked form;
  *   cu_q == cu_k: plain prefill);
+ *   correction: 0 none, 1 mean correction (D3), 2 with the variance term, 3
+ *   block-pooled (D3 variants);
  *   kbar/vbar [total k-blocks, Hkv, d] block means (needed when correction != 0);
+ *   kvar [total k-blocks, Hkv, d] key variances (correction 2), qbar [total
+ *   q-blocks, Hq, d] query block means (correction 3);
  *   sel: global q-block ids to compute (NULL = all), nsel entries;
  *   o [Tq, Hq, d], lse [Tq, Hq], wsum [Tq, Hq] (sum of normalised weights; NULL ok).
  * Returns 0, -1 on an invalid kept list, -2 on a bad q-block id, -3 when a
- * request has more queries than keys. */
+ * request has more queries than keys, -4 on a bad correction mode or a missing
+ * array it needs. */
 int orc_attend(const float* q, const float* k, const float* v, const double* qs, const double* ks,
                const double* vs, const int32_t* cu_q, const int32_t* cu_k, int B, int Hq, int Hkv,
                int d, int Bs, double tau, const int32_t* kept_cnt, const int32_t* kept_idx,
                int nb_max, int correction, const double* kbar, const double* vbar,
-               const int64_t* sel, int64_t nsel, double* o, double* lse, double* wsum) {
+               const double* kvar, const double* qbar, const int64_t* sel, int64_t nsel,
+               double* o, double* lse, double* wsum) {
     int G = Hq / Hkv;
     int64_t* P = chunk_starts(cu_q, cu_k, B);
     if (!P) return -3;
@@ -258,6 +307,8 @@ int orc_attend(const float* q, const float* k, const float* v, const double* qs,
             if (!list_ok(kept_idx + (qb * Hkv + g) * (int64_t)nb_max, kept_cnt[qb * Hkv + g], i))
                 status = -1;
     }
+    if ((correction == 2 && !kvar) || (correction == 3 && !qbar) || correction < 0 || correction > 3)
+        status = -4;
     if (status != 0) { free(P); free(cbq); free(cbk); free(req); return status; }
 
 #pragma omp parallel for schedule(dynamic, 1) collapse(2)
@@ -315,9 +366,21 @@ int orc_attend(const float* q, const float* k, const float* v, const double* qs,
                         if (kept[j]) continue;
                         int64_t kb = cbk[b] + j;
                         int64_t nj = (L - j * Bs) < Bs ? (L - j * Bs) : Bs;
+                        const double* kj = kbar + (kb * Hkv + g) * (int64_t)d;
                         double dot = 0.0;
-                        for (int c = 0; c < d; ++c) dot += qd[c] * kbar[(kb * Hkv + g) * (int64_t)d + c];
+                        if (correction == 3) {        /* block-pooled: qbar of q-block i */
+                            const double* qi = qbar + (qb * Hq + h) * (int64_t)d;
+                            for (int c = 0; c < d; ++c) dot += qi[c] * kj[c];
+                        } else {
+                            for (int c = 0; c < d; ++c) dot += qd[c] * kj[c];
+                        }
                         lg[n] = tau * dot + (MUT(1) ? 0.0 : log((double)nj));
+                        if (correction == 2) {        /* second-order (variance) term */
+                            const double* vj = kvar + (kb * Hkv + g) * (int64_t)d;
+                            double q2v = 0.0;
+                            for (int c = 0; c < d; ++c) q2v += qd[c] * qd[c] * vj[c];
+                            lg[n] += (MUT(15) ? 1.0 : 0.5) * tau * tau * q2v;
+                        }
                         vrow[n] = (MUT(9) ? kbar : vbar) + (kb * Hkv + g) * (int64_t)d;
                         ++n;
                     }

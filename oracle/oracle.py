@@ -59,8 +59,10 @@ def _load(mutant: int = 0):
         lib.orc_block_means.restype = None
         lib.orc_estimate.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _I, _D, _D, _I, _P, _P, _P, _P]
         lib.orc_estimate.restype = _I
+        lib.orc_block_vars.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _P, _P]
+        lib.orc_block_vars.restype = None
         lib.orc_attend.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _D, _P, _P, _I,
-                                   _I, _P, _P, _P, _L, _P, _P, _P]
+                                   _I, _P, _P, _P, _P, _P, _L, _P, _P, _P]
         lib.orc_attend.restype = _I
         lib.orc_mutant_id.restype = _I
         _cache[mutant] = lib
@@ -122,6 +124,18 @@ class Oracle:
                                  _ptr(out))
         return out
 
+    def block_vars(self, x, cu_seqlens, block_size: int, mean, scale=None, pos0=None) -> np.ndarray:
+        """Per-dimension variance of the dequantised rows inside every block around
+        ``mean`` (``block_means`` of the same arguments); the D3 variance variant."""
+        x = _f32(x)
+        T, H, d = x.shape
+        cu, p0, mean = _i32(cu_seqlens), _i64(pos0), _f64(mean)
+        sc = _f64(np.ones(H) if scale is None else scale)
+        out = np.zeros_like(mean)
+        self.lib.orc_block_vars(_ptr(x), _ptr(sc), _ptr(cu), _ptr(p0), len(cu) - 1, H, d, block_size,
+                                _ptr(mean), _ptr(out))
+        return out
+
     # D1 + D2
     def estimate(self, qbar, kbar, cu_seqlens, block_size: int, alpha: float, tau: float,
                  nb_max: Optional[int] = None, want_scores: bool = False, cu_seqlens_k=None):
@@ -148,10 +162,13 @@ class Oracle:
     # D3
     def attend(self, q, k, v, cu_seqlens, block_size: int, tau: float, kept_cnt, kept_idx,
                correction: bool = False, kbar=None, vbar=None, q_scale=None, k_scale=None,
-               v_scale=None, sel=None, want_wsum: bool = False, cu_seqlens_k=None):
+               v_scale=None, sel=None, want_wsum: bool = False, cu_seqlens_k=None, kvar=None, qbar=None):
         """Returns dict(o [T, Hq, d], lse [T, Hq], wsum). Rows outside ``sel`` stay NaN.
         ``cu_seqlens_k`` (None: ``cu_seqlens``) gives the keys of every request
-        when only its last query rows are computed (D0 chunked form)."""
+        when only its last query rows are computed (D0 chunked form).
+        ``correction``: False/0 none, True/1 the mean correction (D3); the D3
+        variants 2 (with the variance term, needs ``kvar``) and 3 (block-pooled,
+        needs ``qbar``) are for approximation studies."""
         q, k, v, cu = _f32(q), _f32(k), _f32(v), _i32(cu_seqlens)
         cuk = cu if cu_seqlens_k is None else _i32(cu_seqlens_k)
         T, Hq, d = q.shape
@@ -161,17 +178,20 @@ class Oracle:
         qs = _f64(np.ones(Hq) if q_scale is None else q_scale)
         ks = _f64(np.ones(Hkv) if k_scale is None else k_scale)
         vs = _f64(np.ones(Hkv) if v_scale is None else v_scale)
-        if correction:
+        mode = int(correction)
+        if mode:
             kbar, vbar = _f64(kbar), _f64(vbar)
+        kvar = None if mode != 2 else _f64(kvar)
+        qbar = None if mode != 3 else _f64(qbar)
         o = np.full((T, Hq, d), np.nan)
         lse = np.full((T, Hq), np.nan)
         ws = np.full((T, Hq), np.nan) if want_wsum else None
         selv = None if sel is None else np.ascontiguousarray(sel, dtype=np.int64)
         rc = self.lib.orc_attend(_ptr(q), _ptr(k), _ptr(v), _ptr(qs), _ptr(ks), _ptr(vs), _ptr(cu),
                                  _ptr(cuk), len(cu) - 1, Hq, Hkv, d, block_size, tau, _ptr(kept_cnt),
-                                 _ptr(kept_idx), nb_max, 1 if correction else 0,
-                                 _ptr(kbar) if correction else None, _ptr(vbar) if correction else None,
-                                 _ptr(selv), 0 if selv is None else len(selv), _ptr(o), _ptr(lse), _ptr(ws))
+                                 _ptr(kept_idx), nb_max, mode,
+                                 _ptr(kbar) if mode else None, _ptr(vbar) if mode else None,
+                                 _ptr(kvar), _ptr(qbar), _ptr(selv), 0 if selv is None else len(selv), _ptr(o), _ptr(lse), _ptr(ws))
         if rc != 0:
             raise ValueError(f"orc_attend failed: {rc}")
         return {"o": o, "lse": lse, "wsum": ws}

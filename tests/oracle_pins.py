@@ -23,6 +23,9 @@ What pins what (definitions D0-D4 in the oracle header):
   chunk_equals_full D0 chunked form: a block-aligned chunk = the full prefill's rows
   chunk_bilinearity D0/D1 chunked form: a partial first q-block's score = mean logit
   chunk_exact_correction  D3 on chunks, the cached prefix's pruned blocks included
+  variance_term     D3 variant 2: half the within-block logit variance (numpy) on
+                    blocks with an exactly diagonal key covariance; block variances
+  pooled_reduces_to_rows  D3 variant 3 = row-wise correction for block-constant q
 """
 from __future__ import annotations
 
@@ -480,6 +483,69 @@ def pin_chunk_exact_correction(orc):
         assert np.abs(r0["o"] - ref_o).max() > 1e-3, "pruning had no effect"
 
 
+# ---------------------------------------------------------------------------
+# D3 variants (approximation studies): variance term and block-pooled logits
+# ---------------------------------------------------------------------------
+def pin_variance_term(orc):
+    """Correction mode 2 adds half the within-block logit variance to each pruned
+    block's logit.  Key blocks built as the block mean plus axis-aligned +/- pairs
+    have an exactly diagonal covariance, so the per-dimension formula must equal
+    the variance of the actual token logits (numpy); the check goes through the
+    LSE of rows whose only kept block is the diagonal.  Block variances are also
+    checked against numpy.var."""
+    L, hq, hkv, d = 640, 2, 1, 128
+    rng = np.random.default_rng(111)
+    q = (rng.integers(-16, 17, (L, hq, d)) / 16.0).astype(np.float32)
+    k = np.zeros((L, hkv, d), np.float32)
+    v = rng.standard_normal((L, hkv, d)).astype(np.float32)
+    for j in range(L // 128):
+        mean = rng.integers(-8, 9, (hkv, d)) / 16.0
+        blk = np.repeat(mean[None], 128, axis=0)
+        if j != 2:                                   # block 2 stays constant: zero variance
+            for t in range(64):
+                axis, amp = rng.integers(0, d), rng.integers(1, 17) / 16.0
+                blk[2 * t, :, axis] += amp
+                blk[2 * t + 1, :, axis] -= amp
+        k[j * 128:(j + 1) * 128] = blk.astype(np.float32)
+    cu = np.array([0, L], np.int32)
+    qb, kb, vb = _means(orc, q, k, v, cu)
+    kv = orc.block_vars(k, cu, 128, kb)
+    for j in range(L // 128):
+        assert np.abs(kv[j] - k[j * 128:(j + 1) * 128].astype(np.float64).var(axis=0)).max() < 1e-14
+    nb = L // 128
+    cnt = np.ones((nb, hkv), np.int32)
+    idx = np.full((nb, hkv, nb), -1, np.int32)
+    idx[np.arange(nb), 0, 0] = np.arange(nb)           # only the diagonal block kept
+    r = orc.attend(q, k, v, cu, 128, TAU, cnt, idx, correction=2, kbar=kb, vbar=vb, kvar=kv)
+    kk = k.astype(np.float64)
+    for row in (130, 300, 511, 639):
+        i = row // 128
+        for h in range(hq):
+            qr = q[row, h].astype(np.float64)
+            logits = TAU * (kk[:, 0] @ qr)
+            den = np.exp(logits[i * 128:row + 1]).sum()
+            for j in range(i):
+                lj = logits[j * 128:(j + 1) * 128]
+                den += 128 * math.exp(lj.mean() + 0.5 * lj.var())
+            assert abs(r["lse"][row, h] - math.log(den)) < 1e-12, "variance term differs from the logit variance"
+
+
+def pin_pooled_reduces_to_rows(orc):
+    """Correction mode 3 (block-pooled logits) equals the row-wise correction when
+    every row of a q-block equals the block's mean query."""
+    wl = _structured([700], seed=121)
+    q, k, v = wl.float_inputs()
+    q = np.repeat(q[::128], 128, axis=0)[:700]       # rows constant inside each q-block
+    cu = wl.cu_seqlens
+    qb, kb, vb = _means(orc, q, k, v, cu)
+    est = orc.estimate(qb, kb, cu, 128, alpha=0.3, tau=TAU)
+    a = orc.attend(q, k, v, cu, 128, TAU, est["kept_cnt"], est["kept_idx"], correction=1, kbar=kb, vbar=vb)
+    b = orc.attend(q, k, v, cu, 128, TAU, est["kept_cnt"], est["kept_idx"], correction=3, kbar=kb, vbar=vb,
+                   qbar=qb)
+    assert np.array_equal(a["o"], b["o"]) and np.array_equal(a["lse"], b["lse"]), "pooled != row-wise"
+
+
 ALL_PINS = [pin_dense_sdpa, pin_means_numpy, pin_bilinearity, pin_threshold_golden, pin_diagonal_kept,
             pin_nesting, pin_weights_sum, pin_exact_correction, pin_gqa_packing, pin_ragged, pin_e4m3_scales,
-            pin_chunk_dense_sdpa, pin_chunk_equals_full, pin_chunk_bilinearity, pin_chunk_exact_correction]
+            pin_chunk_dense_sdpa, pin_chunk_equals_full, pin_chunk_bilinearity, pin_chunk_exact_correction,
+            pin_variance_term, pin_pooled_reduces_to_rows]

@@ -1,0 +1,72 @@
+"""Approximation quality of the mean correction and two variants of it (CPU, oracle).
+
+Not a parity test.  The method approximates dense causal attention, and this
+measures how far its output lands from dense attention.  The input is the seeded
+Llama-3-8B-shaped workload of the 128K benchmark, generated at 8192 tokens
+(alpha = 0.05).  The error is taken over every row of six seeded q-blocks and
+all 32 query heads.  Corrections:
+  none      pruned blocks dropped;
+  mean      the mean correction, which the GPU kernels implement;
+  variance  the mean correction plus half the within-block logit variance,
+            taken per dimension of the keys (oracle correction mode 2);
+  pooled    the mean correction with the q-block's mean query (mode 3).
+By Jensen's inequality the mean correction undercounts a pruned block's mass by
+about exp(var / 2), which the variance term restores.  The test requires
+variance < mean < none and prints the errors (run with -s).  Set
+FP2_APPROX_SEQLEN=32768 to run the same study at 32K.
+"""
+import math
+import os
+
+import numpy as np
+import torch
+
+from oracle.oracle import Oracle
+from workloads import make_config
+
+SEQLEN = int(os.environ.get("FP2_APPROX_SEQLEN", "8192"))
+
+
+def _dense_rows(q, k, v, rows, hq, hkv, tau):
+    """Dense causal attention (torch fp64) of the given rows of a single request,
+    128 rows at a time."""
+    g = hq // hkv
+    out = []
+    for s in range(0, len(rows), 128):
+        rr = rows[s:s + 128]
+        end = int(rr.max()) + 1
+        qt = torch.from_numpy(q[rr]).double().transpose(0, 1)                           # [Hq, R, d]
+        kt = torch.from_numpy(k[:end]).double().repeat_interleave(g, dim=1).transpose(0, 1)  # [Hq, end, d]
+        vt = torch.from_numpy(v[:end]).double().repeat_interleave(g, dim=1).transpose(0, 1)
+        logits = (qt @ kt.transpose(1, 2)) * tau
+        mask = torch.arange(end)[None, :] <= torch.from_numpy(rr)[:, None]
+        w = torch.softmax(logits.masked_fill(~mask[None], -math.inf), dim=-1)
+        out.append((w @ vt).transpose(0, 1).numpy())
+    return np.concatenate(out)
+
+
+def test_correction_variants_against_dense():
+    wl = make_config(2, seqlen=SEQLEN)
+    orc = Oracle()
+    q, k, v = wl.float_inputs()
+    cu = wl.cu_seqlens
+    tau = 1.0 / math.sqrt(wl.head_dim)
+    qb = orc.block_means(q, cu, 128)
+    kb = orc.block_means(k, cu, 128)
+    vb = orc.block_means(v, cu, 128)
+    kv = orc.block_vars(k, cu, 128, kb)
+    est = orc.estimate(qb, kb, cu, 128, alpha=wl.alpha, tau=tau)
+    nb = qb.shape[0]
+    sel = np.sort(np.random.default_rng(5).choice(np.arange(8, nb), 6, replace=False))
+    rows = np.concatenate([np.arange(i * 128, min(wl.total_tokens, (i + 1) * 128)) for i in sel])
+    ref = _dense_rows(q, k, v, rows, wl.num_q_heads, wl.num_kv_heads, tau)
+    ref_norm = np.linalg.norm(ref)
+    err = {}
+    for name, mode in (("none", 0), ("mean", 1), ("variance", 2), ("pooled", 3)):
+        r = orc.attend(q, k, v, cu, 128, tau, est["kept_cnt"], est["kept_idx"], correction=mode, kbar=kb,
+                       vbar=vb, kvar=kv, qbar=qb, sel=sel)
+        err[name] = float(np.linalg.norm(r["o"][rows] - ref) / ref_norm)
+    density = est["kept_cnt"].sum() / (wl.num_kv_heads * nb * (nb + 1) / 2)
+    print(f"\n{SEQLEN} tokens, alpha {wl.alpha}, kept density {density:.4f}, q-blocks {sel.tolist()}: "
+          + ", ".join(f"{k_} rel-L2 {v_:.4f}" for k_, v_ in err.items()))
+    assert err["variance"] < err["mean"] < err["none"], err

@@ -20,6 +20,7 @@ MUTANTS = {
     12: "chunk: causal mask relative to the chunk start, not the position",
     13: "chunk: partial first q-block mean divided by rows before the chunk too",
     14: "chunk: pruned blocks of the cached prefix get no correction",
+    15: "variance variant: the full logit variance added instead of half of it",
 }
 
 
