@@ -9,7 +9,10 @@ all 32 query heads.  Corrections:
   mean      the mean correction, which the GPU kernels implement;
   variance  the mean correction plus half the within-block logit variance,
             taken per dimension of the keys (oracle correction mode 2);
-  pooled    the mean correction with the q-block's mean query (mode 3).
+  pooled    the mean correction with the q-block's mean query (mode 3);
+  strided   the mean correction, with kept lists estimated from every 8th
+            query row of each block instead of all 128 (the estimator would
+            read an eighth of Q).
 By Jensen's inequality the mean correction undercounts a pruned block's mass by
 about exp(var / 2), which the variance term restores.  The test requires
 variance < mean < none and prints the errors (run with -s).  Set
@@ -66,7 +69,23 @@ def test_correction_variants_against_dense():
         r = orc.attend(q, k, v, cu, 128, tau, est["kept_cnt"], est["kept_idx"], correction=mode, kbar=kb,
                        vbar=vb, kvar=kv, qbar=qb, sel=sel)
         err[name] = float(np.linalg.norm(r["o"][rows] - ref) / ref_norm)
+    # strided estimate: query means over rows 0, 8, 16, ... of each block; in the
+    # subsampled sequence a block is 128 / 8 rows
+    stride = 8
+    q_sub = np.ascontiguousarray(q[::stride])
+    qb_sub = orc.block_means(q_sub, np.array([0, q_sub.shape[0]], np.int32), 128 // stride)
+    assert qb_sub.shape == qb.shape
+    est_s = orc.estimate(qb_sub, kb, cu, 128, alpha=wl.alpha, tau=tau, nb_max=est["nb_max"])
+    r = orc.attend(q, k, v, cu, 128, tau, est_s["kept_cnt"], est_s["kept_idx"], correction=1, kbar=kb, vbar=vb,
+                   sel=sel)
+    err["strided"] = float(np.linalg.norm(r["o"][rows] - ref) / ref_norm)
+    same = np.mean([set(est["kept_idx"][t, g, :est["kept_cnt"][t, g]].tolist())
+                    == set(est_s["kept_idx"][t, g, :est_s["kept_cnt"][t, g]].tolist())
+                    for t in range(nb) for g in range(wl.num_kv_heads)])
     density = est["kept_cnt"].sum() / (wl.num_kv_heads * nb * (nb + 1) / 2)
     print(f"\n{SEQLEN} tokens, alpha {wl.alpha}, kept density {density:.4f}, q-blocks {sel.tolist()}: "
-          + ", ".join(f"{k_} rel-L2 {v_:.4f}" for k_, v_ in err.items()))
+          + ", ".join(f"{k_} rel-L2 {v_:.4f}" for k_, v_ in err.items())
+          + f"; strided: kept lists equal to the full estimate's {same:.3f}, kept density "
+          f"{est_s['kept_cnt'].sum() / (wl.num_kv_heads * nb * (nb + 1) / 2):.4f}")
     assert err["variance"] < err["mean"] < err["none"], err
+    assert err["strided"] < err["none"], err
