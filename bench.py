@@ -235,6 +235,13 @@ def time_layer(st, wl, steps, warmup, dist_ctx, clocks=None):
     return total, est, att, clk
 
 
+def mufu_bound_tflops(sms, mhz, d=128, exp_per_clk_per_sm=16):
+    """Ceiling of an attention kernel set by the exponential unit: one exp2 per
+    (query, key) pair, which carries 4*d flops, at the nominal 16 exp2 per clock
+    per SM (MUFU).  Binding for e4m3, whose MMAs outrun it."""
+    return exp_per_clk_per_sm * 4.0 * d * sms * mhz * 1e6 / 1e12
+
+
 def dense_causal_flops(seqlens, hq, d=128):
     """4*d flops per causal query-key pair, summed over the requests and query heads."""
     return 4.0 * d * hq * sum(L * (L + 1) / 2 for L in seqlens)
@@ -612,6 +619,14 @@ def ours(args):
             "peak_note": note8,
             "frac_attention_of_2x_bf16": (f8 + c8) / (a8 * 1e-3) / 1e12 / (peaks["bf16_tflops"] * E4M3_OVER_BF16),
         }
+        # the exponential unit bounds e4m3 attention below the e4m3 GEMM peak
+        max_mhz = (clk or {}).get("sm_max_mhz") or 1965.0
+        mufu = mufu_bound_tflops(torch.cuda.get_device_properties(dev).multi_processor_count, max_mhz)
+        fp8["mufu_bound_tflops"] = mufu
+        fp8["frac_attention_of_mufu_bound"] = fp8["tflops_attention"] / mufu
+        fp8["mufu_note"] = ("one exp2 per query-key pair (4*d flops) at 16 exp2/clk/SM, all SMs, "
+                            f"{max_mhz:.0f} MHz; a ceiling (masked diagonal and correction columns also "
+                            "take exponentials)")
         del st8
 
     # dense comparators (context only), after every timed measurement above

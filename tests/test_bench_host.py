@@ -113,3 +113,8 @@ def test_dense_flops_equal_layer_work_with_every_block_kept():
     flops, corr = bench.layer_work(seqlens, cnt, idx, hq, hkv)
     assert corr == 0.0
     assert flops == bench.dense_causal_flops(seqlens, hq)
+
+
+def test_mufu_bound():
+    """16 exp2/clk/SM x 148 SMs x 1965 MHz, 512 flops per exp2 (d = 128)."""
+    assert abs(bench.mufu_bound_tflops(148, 1965.0) - 2382.40) < 0.01
