@@ -666,6 +666,13 @@ def ours(args):
         "ms_attention_median": statistics.median(att), "ms_attention_min": min(att),
         "ms_estimate_median": statistics.median(est), "ms_estimate_min": min(est),
         "tflops_attention": ach_att,
+        "work": {
+            "kept_pairs_tflop": flops / 1e12, "correction_tflop": corr_flops / 1e12,
+            "total_tflop": (flops + corr_flops) / 1e12,
+            "tflops_attention_kept_pairs_only": flops / (ms_att * 1e-3) / 1e12,
+            "note": "4*d flops per kept causal query-key pair (diagonal block counted causally) and per "
+                    "(row, pruned block) correction term; tflops_attention counts both",
+        },
         "roofline": {
             "bound": "tensor", "achieved": ach_att, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
             "frac": ach_att / peaks["bf16_tflops"],
