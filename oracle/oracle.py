@@ -199,19 +199,24 @@ class Oracle:
     # whole path for a workload
     def run(self, wl, alpha: Optional[float] = None, correction: bool = True, sel=None,
             want_scores: bool = False, tau: Optional[float] = None, kept=None):
-        """Estimate (unless ``kept`` is given) then attend, on a ``workloads.Workload``."""
+        """Estimate (unless ``kept`` is given) then attend, on a ``workloads.Workload``
+        (chunked workloads: queries are the last ``query_lens[b]`` tokens of each request)."""
         q, k, v = wl.float_inputs()
-        cu = wl.cu_seqlens
+        cu = wl.cu_seqlens                              # keys
+        chunked = getattr(wl, "query_lens", None) is not None
+        cu_q = wl.cu_seqlens_q if chunked else cu      # query rows
+        pos0 = chunk_starts(cu_q, cu) if chunked else None
         bs = wl.block_size
         tau = 1.0 / math.sqrt(wl.head_dim) if tau is None else tau
         a = wl.alpha if alpha is None else alpha
-        qbar = self.block_means(q, cu, bs, wl.q_scale)
+        qbar = self.block_means(q, cu_q, bs, wl.q_scale, pos0=pos0)
         kbar = self.block_means(k, cu, bs, wl.k_scale)
         vbar = self.block_means(v, cu, bs, wl.v_scale)
-        est = kept if kept is not None else self.estimate(qbar, kbar, cu, bs, a, tau, want_scores=want_scores)
-        att = self.attend(q, k, v, cu, bs, tau, est["kept_cnt"], est["kept_idx"], correction=correction,
+        est = kept if kept is not None else self.estimate(qbar, kbar, cu_q, bs, a, tau, want_scores=want_scores,
+                                                          cu_seqlens_k=cu)
+        att = self.attend(q, k, v, cu_q, bs, tau, est["kept_cnt"], est["kept_idx"], correction=correction,
                           kbar=kbar, vbar=vbar, q_scale=wl.q_scale, k_scale=wl.k_scale,
-                          v_scale=wl.v_scale, sel=sel)
+                          v_scale=wl.v_scale, sel=sel, cu_seqlens_k=cu)
         return {**est, **att, "qbar": qbar, "kbar": kbar, "vbar": vbar}
 
 

@@ -52,3 +52,48 @@ def test_config_shapes():
     # config 3 is config 2 encoded in e4m3
     x = w3.q.float() * torch.from_numpy(w3.q_scale)[None, :, None]
     assert ((x - w2.q.float()).abs() <= w2.q.float().abs() * 2 ** -4 + 1e-2).all()
+
+
+def test_chunked_workload_rows_and_scales():
+    """The queries of a chunked workload are the last rows of the plain workload's
+    requests (same seed); e4m3 query scales come from the chunk's rows."""
+    from workloads import make_chunked_workload
+    lens, lq = [700, 300, 129], [500, 45, 129]
+    full = make_workload(lens, 8, 2, alpha=0.1, seed=3)
+    ch = make_chunked_workload(lens, lq, 8, 2, alpha=0.1, seed=3)
+    cu, cuq = full.cu_seqlens, ch.cu_seqlens_q
+    assert list(cuq) == [0, 500, 545, 674] and ch.total_queries == 674 and ch.total_tokens == 1129
+    for b, n in enumerate(lq):
+        assert torch.equal(ch.q[cuq[b]:cuq[b + 1]], full.q[cu[b + 1] - n:cu[b + 1]])
+    assert torch.equal(ch.k, full.k) and torch.equal(ch.v, full.v)
+    e = make_chunked_workload(lens, lq, 8, 2, alpha=0.1, seed=3, dtype="e4m3")
+    amax = ch.q.float().abs().amax(dim=(0, 2)).numpy()
+    assert np.allclose(e.q_scale, amax / 448.0, rtol=1e-6)
+    amax_k = full.k.float().abs().amax(dim=(0, 2)).numpy()
+    assert np.allclose(e.k_scale, amax_k / 448.0, rtol=1e-6)
+
+
+def test_chunked_paged_pool_matches_contiguous():
+    from workloads import make_chunked_workload
+    wl = make_chunked_workload([700, 300], [500, 45], 4, 2, alpha=0.1, seed=4, paged=True)
+    cu = wl.cu_seqlens
+    for b, L in enumerate(wl.seqlens):
+        for j in range((L + 127) // 128):
+            page = int(wl.block_table[b, j])
+            n = min(128, L - j * 128)
+            assert torch.equal(wl.k_pool[page * 128:page * 128 + n], wl.k[cu[b] + j * 128:cu[b] + j * 128 + n])
+
+
+def test_oracle_run_on_a_block_aligned_chunk_equals_full_rows():
+    """Oracle.run on a chunked workload: a chunk starting on a block boundary gives
+    the full prefill's rows (the D0 chunked form reduces to the plain one there)."""
+    from oracle.oracle import Oracle
+    from workloads import make_chunked_workload
+    lens, lq = [1000, 640], [744, 256]              # chunks start at 256 and 384
+    orc = Oracle()
+    full = orc.run(make_workload(lens, 4, 2, alpha=0.2, seed=9))
+    ch = orc.run(make_chunked_workload(lens, lq, 4, 2, alpha=0.2, seed=9))
+    cu, cuq = np.array([0, 1000, 1640]), np.array([0, 744, 1000])
+    for b, n in enumerate(lq):
+        assert np.array_equal(ch["o"][cuq[b]:cuq[b + 1]], full["o"][cu[b + 1] - n:cu[b + 1]])
+        assert np.array_equal(ch["lse"][cuq[b]:cuq[b + 1]], full["lse"][cu[b + 1] - n:cu[b + 1]])

@@ -1,6 +1,6 @@
 """Seeded synthetic workloads shared by the tests, the benchmark and the oracle."""
-from .synthetic import (Workload, make_workload, make_config, ragged_lengths, quantize_e4m3,
-                        page_kv, CONFIG_NAMES)
+from .synthetic import (Workload, make_workload, make_chunked_workload, make_config, ragged_lengths,
+                        quantize_e4m3, page_kv, CONFIG_NAMES)
 
-__all__ = ["Workload", "make_workload", "make_config", "ragged_lengths", "quantize_e4m3",
+__all__ = ["Workload", "make_workload", "make_chunked_workload", "make_config", "ragged_lengths", "quantize_e4m3",
            "page_kv", "CONFIG_NAMES"]

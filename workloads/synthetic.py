@@ -62,7 +62,7 @@ class Workload:
     block_size: int
     alpha: float
     dtype: str                      # "bf16" or "e4m3"
-    q: torch.Tensor                 # [T, Hq, d] bf16 or float8_e4m3fn
+    q: torch.Tensor                 # [T, Hq, d] bf16 or float8_e4m3fn ([total_queries, ...] if chunked)
     k: torch.Tensor                 # [T, Hkv, d]
     v: torch.Tensor                 # [T, Hkv, d]
     q_scale: np.ndarray             # [Hq] float32 (all ones for bf16)
@@ -73,6 +73,9 @@ class Workload:
     k_pool: Optional[torch.Tensor] = None      # [num_pages * Bs, Hkv, d]
     v_pool: Optional[torch.Tensor] = None
     seed: int = 0
+    # chunked prefill: request b's queries are its last query_lens[b] tokens (q holds
+    # only those rows); None = every token is a query (plain prefill)
+    query_lens: Optional[list] = None
 
     @property
     def batch(self) -> int:
@@ -80,6 +83,7 @@ class Workload:
 
     @property
     def total_tokens(self) -> int:
+        """Keys of the batch (= query rows unless chunked; see total_queries)."""
         return int(sum(self.seqlens))
 
     @property
@@ -89,6 +93,17 @@ class Workload:
     @property
     def cu_seqlens(self) -> np.ndarray:
         return np.concatenate([[0], np.cumsum(self.seqlens)]).astype(np.int32)
+
+    @property
+    def cu_seqlens_q(self) -> np.ndarray:
+        """Query rows of every request (= cu_seqlens for plain prefill)."""
+        if self.query_lens is None:
+            return self.cu_seqlens
+        return np.concatenate([[0], np.cumsum(self.query_lens)]).astype(np.int32)
+
+    @property
+    def total_queries(self) -> int:
+        return int(self.cu_seqlens_q[-1])
 
     @property
     def num_pages(self) -> int:
@@ -244,6 +259,36 @@ def make_workload(seqlens, num_q_heads=32, num_kv_heads=8, head_dim=128, block_s
         prng = np.random.default_rng(seed + 7919)
         wl.block_table, wl.k_pool, wl.v_pool = page_kv(k, v, wl.seqlens, block_size, prng)
     return wl
+
+
+def make_chunked_workload(seqlens, query_lens, num_q_heads=32, num_kv_heads=8, head_dim=128,
+                          block_size=128, alpha=0.05, dtype="bf16", seed=0, n_retrieval=3,
+                          lam=LOCAL_LAMBDA, paged=False, name="chunked") -> Workload:
+    """Chunked prefill: request b has seqlens[b] keys, and its queries are its last
+    query_lens[b] tokens (the first seqlens[b] - query_lens[b] are already in the KV
+    cache).  The tokens are those of make_workload(seqlens, ...) with the same seed, so
+    the query rows are the last rows of that workload's requests; in e4m3 the query
+    scales come from the chunk's rows, the K/V scales from all keys."""
+    assert len(query_lens) == len(seqlens)
+    assert all(0 <= int(n) <= int(L) for n, L in zip(query_lens, seqlens))
+    full = make_workload(seqlens, num_q_heads, num_kv_heads, head_dim, block_size, alpha, "bf16", seed,
+                         n_retrieval, lam, paged=False, name=name)
+    cu = full.cu_seqlens
+    parts = [full.q[int(cu[b + 1]) - int(n):int(cu[b + 1])] for b, n in enumerate(query_lens)]
+    q = torch.cat(parts, dim=0) if parts else full.q[:0]
+    k, v = full.k, full.v
+    if dtype == "e4m3":
+        q, full.q_scale = quantize_e4m3(q)
+        k, full.k_scale = quantize_e4m3(k)
+        v, full.v_scale = quantize_e4m3(v)
+    elif dtype != "bf16":
+        raise ValueError(dtype)
+    full.q, full.k, full.v, full.dtype = q.contiguous(), k, v, dtype
+    full.query_lens = [int(n) for n in query_lens]
+    if paged:
+        prng = np.random.default_rng(seed + 7919)
+        full.block_table, full.k_pool, full.v_pool = page_kv(k, v, full.seqlens, block_size, prng)
+    return full
 
 
 def ragged_lengths(seed: int, n: int = 8, lo: int = 4096, hi: int = 131072):
