@@ -56,6 +56,21 @@
  *               block-pooled logit tau qbar_i . kbar_j, shared by all rows of
  *               q-block i, instead of the row's own.
  *
+ * Pins (tests/oracle_pins.py), each against a fact outside this file:
+ *   D0, D3 core   torch scaled_dot_product_attention in fp64 at alpha <= 0
+ *                 (plain and chunked, ragged lengths, an empty request);
+ *   D1            numpy means; the score equals the brute-force mean token logit;
+ *   D2            hand-derived golden cases; forced diagonal; nesting in alpha;
+ *                 packed heads equal each head alone;
+ *   D3 correction exact on block-constant K/V (plain and chunked); weights sum to 1;
+ *   D4            power-of-two scaled inputs;
+ *   D3 variants   numpy variance of the token logits; the pooled form reduces to
+ *                 the row-wise one.
+ * The pages print no worked example or value, so the readings named above
+ * (mean pooling, the threshold in the exp domain, the form of the correction,
+ * the chunked block grid) are parity unpinned by the pages themselves: the pins
+ * fix the arithmetic given each reading.
+ *
  * Build with -DORC_MUTANT=n to plant one deliberate mistake (see the MUT()
  * sites); the oracle self-tests check that every such mistake is caught.
  */
