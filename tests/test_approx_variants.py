@@ -34,17 +34,18 @@ def _dense_rows(q, k, v, rows, hq, hkv, tau):
     """Dense causal attention (torch fp64) of the given rows of a single request,
     128 rows at a time."""
     g = hq // hkv
+    end_all = int(rows.max()) + 1
+    kt_all = torch.from_numpy(k[:end_all]).double().repeat_interleave(g, dim=1).transpose(0, 1)  # [Hq, end, d]
+    vt_all = torch.from_numpy(v[:end_all]).double().repeat_interleave(g, dim=1).transpose(0, 1)
     out = []
     for s in range(0, len(rows), 128):
         rr = rows[s:s + 128]
         end = int(rr.max()) + 1
-        qt = torch.from_numpy(q[rr]).double().transpose(0, 1)                           # [Hq, R, d]
-        kt = torch.from_numpy(k[:end]).double().repeat_interleave(g, dim=1).transpose(0, 1)  # [Hq, end, d]
-        vt = torch.from_numpy(v[:end]).double().repeat_interleave(g, dim=1).transpose(0, 1)
-        logits = (qt @ kt.transpose(1, 2)) * tau
+        qt = torch.from_numpy(q[rr]).double().transpose(0, 1)                                    # [Hq, R, d]
+        logits = (qt @ kt_all[:, :end].transpose(1, 2)) * tau
         mask = torch.arange(end)[None, :] <= torch.from_numpy(rr)[:, None]
         w = torch.softmax(logits.masked_fill(~mask[None], -math.inf), dim=-1)
-        out.append((w @ vt).transpose(0, 1).numpy())
+        out.append((w @ vt_all[:, :end]).transpose(0, 1).numpy())
     return np.concatenate(out)
 
 
