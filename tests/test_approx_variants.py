@@ -16,7 +16,8 @@ all 32 query heads.  Corrections:
 By Jensen's inequality the mean correction undercounts a pruned block's mass by
 about exp(var / 2), which the variance term restores.  The test requires
 variance < mean < none and prints the errors (run with -s).  Set
-FP2_APPROX_SEQLEN=32768 to run the same study at 32K.
+FP2_APPROX_SEQLEN=32768 to run the same study at 32K, and FP2_APPROX_ALPHA to change
+alpha.
 """
 import math
 import os
@@ -28,6 +29,7 @@ from oracle.oracle import Oracle
 from workloads import make_config
 
 SEQLEN = int(os.environ.get("FP2_APPROX_SEQLEN", "8192"))
+ALPHA = float(os.environ.get("FP2_APPROX_ALPHA", "0.05"))
 
 
 def _dense_rows(q, k, v, rows, hq, hkv, tau):
@@ -50,7 +52,7 @@ def _dense_rows(q, k, v, rows, hq, hkv, tau):
 
 
 def test_correction_variants_against_dense():
-    wl = make_config(2, seqlen=SEQLEN)
+    wl = make_config(2, seqlen=SEQLEN, alpha=ALPHA)
     orc = Oracle()
     q, k, v = wl.float_inputs()
     cu = wl.cu_seqlens
