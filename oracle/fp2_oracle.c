@@ -54,7 +54,9 @@
  *               uncorrelated inside the block; by Jensen the plain form
  *               undercounts a block's mass by about e^{var / 2}).  Mode 3 uses the
  *               block-pooled logit tau qbar_i . kbar_j, shared by all rows of
- *               q-block i, instead of the row's own.
+ *               q-block i, instead of the row's own.  Mode 4 is mode 2 with the
+ *               key variance averaged over the dimensions, (tau^2 / 2) |q|^2
+ *               mean_c var_j[c]: one scalar per row times one per block.
  *
  * Pins (tests/oracle_pins.py), each against a fact outside this file:
  *   D0, D3 core   torch scaled_dot_product_attention in fp64 at alpha <= 0
@@ -284,9 +286,9 @@ static int list_ok(const int32_t* idx, int32_t cnt, int64_t i) {
  *   cu_q / cu_k: query rows and keys of every request (D0 chunked form;
  *   cu_q == cu_k: plain prefill);
  *   correction: 0 none, 1 mean correction (D3), 2 with the variance term, 3
- *   block-pooled (D3 variants);
+ *   block-pooled, 4 with the dimension-averaged variance term (D3 variants);
  *   kbar/vbar [total k-blocks, Hkv, d] block means (needed when correction != 0);
- *   kvar [total k-blocks, Hkv, d] key variances (correction 2), qbar [total
+ *   kvar [total k-blocks, Hkv, d] key variances (corrections 2, 4), qbar [total
  *   q-blocks, Hq, d] query block means (correction 3);
  *   sel: global q-block ids to compute (NULL = all), nsel entries;
  *   o [Tq, Hq, d], lse [Tq, Hq], wsum [Tq, Hq] (sum of normalised weights; NULL ok).
@@ -322,7 +324,8 @@ int orc_attend(const float* q, const float* k, const float* v, const double* qs,
             if (!list_ok(kept_idx + (qb * Hkv + g) * (int64_t)nb_max, kept_cnt[qb * Hkv + g], i))
                 status = -1;
     }
-    if ((correction == 2 && !kvar) || (correction == 3 && !qbar) || correction < 0 || correction > 3)
+    if (((correction == 2 || correction == 4) && !kvar) || (correction == 3 && !qbar) || correction < 0 ||
+        correction > 4)
         status = -4;
     if (status != 0) { free(P); free(cbq); free(cbk); free(req); return status; }
 
@@ -390,10 +393,16 @@ int orc_attend(const float* q, const float* k, const float* v, const double* qs,
                             for (int c = 0; c < d; ++c) dot += qd[c] * kj[c];
                         }
                         lg[n] = tau * dot + (MUT(1) ? 0.0 : log((double)nj));
-                        if (correction == 2) {        /* second-order (variance) term */
+                        if (correction == 2 || correction == 4) {   /* second-order (variance) term */
                             const double* vj = kvar + (kb * Hkv + g) * (int64_t)d;
                             double q2v = 0.0;
-                            for (int c = 0; c < d; ++c) q2v += qd[c] * qd[c] * vj[c];
+                            if (correction == 2) {
+                                for (int c = 0; c < d; ++c) q2v += qd[c] * qd[c] * vj[c];
+                            } else {                  /* |q|^2 times the mean variance */
+                                double q2 = 0.0, vm = 0.0;
+                                for (int c = 0; c < d; ++c) { q2 += qd[c] * qd[c]; vm += vj[c]; }
+                                q2v = q2 * (MUT(16) ? vm : vm / d);
+                            }
                             lg[n] += (MUT(15) ? 1.0 : 0.5) * tau * tau * q2v;
                         }
                         vrow[n] = (MUT(9) ? kbar : vbar) + (kb * Hkv + g) * (int64_t)d;

@@ -167,8 +167,9 @@ class Oracle:
         ``cu_seqlens_k`` (None: ``cu_seqlens``) gives the keys of every request
         when only its last query rows are computed (D0 chunked form).
         ``correction``: False/0 none, True/1 the mean correction (D3); the D3
-        variants 2 (with the variance term, needs ``kvar``) and 3 (block-pooled,
-        needs ``qbar``) are for approximation studies."""
+        variants 2 (with the variance term, needs ``kvar``), 3 (block-pooled,
+        needs ``qbar``) and 4 (the variance averaged over the dimensions, needs
+        ``kvar``) are for approximation studies."""
         q, k, v, cu = _f32(q), _f32(k), _f32(v), _i32(cu_seqlens)
         cuk = cu if cu_seqlens_k is None else _i32(cu_seqlens_k)
         T, Hq, d = q.shape
@@ -181,7 +182,7 @@ class Oracle:
         mode = int(correction)
         if mode:
             kbar, vbar = _f64(kbar), _f64(vbar)
-        kvar = None if mode != 2 else _f64(kvar)
+        kvar = None if mode not in (2, 4) else _f64(kvar)
         qbar = None if mode != 3 else _f64(qbar)
         o = np.full((T, Hq, d), np.nan)
         lse = np.full((T, Hq), np.nan)

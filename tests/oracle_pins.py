@@ -25,6 +25,7 @@ What pins what (definitions D0-D4 in the oracle header):
   chunk_exact_correction  D3 on chunks, the cached prefix's pruned blocks included
   variance_term     D3 variant 2: half the within-block logit variance (numpy) on
                     blocks with an exactly diagonal key covariance; block variances
+  isotropic_variance_term  D3 variant 4 on Hadamard blocks (isotropic covariance)
   pooled_reduces_to_rows  D3 variant 3 = row-wise correction for block-constant q
 """
 from __future__ import annotations
@@ -530,6 +531,48 @@ def pin_variance_term(orc):
             assert abs(r["lse"][row, h] - math.log(den)) < 1e-12, "variance term differs from the logit variance"
 
 
+def pin_isotropic_variance_term(orc):
+    """Correction mode 4 (the variance averaged over the key dimensions) on key
+    blocks with an exactly isotropic covariance: block mean plus a_j times
+    columns 1..64 of a 128x128 Hadamard matrix (zero column sums, orthogonal
+    columns; d = 64).  It must equal half the numpy variance of the token logits,
+    and mode 2 on the same blocks."""
+    L, hq, hkv, d = 640, 2, 1, 64
+    rng = np.random.default_rng(131)
+    h = np.array([[1.0]])
+    while h.shape[0] < 128:
+        h = np.block([[h, h], [h, -h]])
+    dev = h[:, 1:d + 1]                               # [128, 64], columns sum to 0
+    q = (rng.integers(-16, 17, (L, hq, d)) / 16.0).astype(np.float32)
+    k = np.zeros((L, hkv, d), np.float32)
+    v = rng.standard_normal((L, hkv, d)).astype(np.float32)
+    for j in range(L // 128):
+        mean = rng.integers(-8, 9, (hkv, d)) / 16.0
+        amp = 0.0 if j == 1 else rng.integers(1, 17) / 16.0
+        k[j * 128:(j + 1) * 128] = (mean[None] + amp * dev[:, None, :]).astype(np.float32)
+    cu = np.array([0, L], np.int32)
+    qb, kb, vb = _means(orc, q, k, v, cu)
+    kv = orc.block_vars(k, cu, 128, kb)
+    nb = L // 128
+    cnt = np.ones((nb, hkv), np.int32)
+    idx = np.full((nb, hkv, nb), -1, np.int32)
+    idx[np.arange(nb), 0, 0] = np.arange(nb)           # only the diagonal block kept
+    r4 = orc.attend(q, k, v, cu, 128, TAU, cnt, idx, correction=4, kbar=kb, vbar=vb, kvar=kv)
+    r2 = orc.attend(q, k, v, cu, 128, TAU, cnt, idx, correction=2, kbar=kb, vbar=vb, kvar=kv)
+    assert np.isfinite(r4["lse"]).all() and np.isfinite(r2["lse"]).all(), "non-finite LSE"
+    assert np.abs(r4["lse"] - r2["lse"]).max() < 1e-12, "isotropic blocks: mode 4 != mode 2"
+    kk = k.astype(np.float64)
+    for row in (130, 300, 511, 639):
+        i = row // 128
+        for hh in range(hq):
+            logits = TAU * (kk[:, 0] @ q[row, hh].astype(np.float64))
+            den = np.exp(logits[i * 128:row + 1]).sum()
+            for j in range(i):
+                lj = logits[j * 128:(j + 1) * 128]
+                den += 128 * math.exp(lj.mean() + 0.5 * lj.var())
+            assert abs(r4["lse"][row, hh] - math.log(den)) < 1e-12, "mode 4 differs from the logit variance"
+
+
 def pin_pooled_reduces_to_rows(orc):
     """Correction mode 3 (block-pooled logits) equals the row-wise correction when
     every row of a q-block equals the block's mean query."""
@@ -548,4 +591,4 @@ def pin_pooled_reduces_to_rows(orc):
 ALL_PINS = [pin_dense_sdpa, pin_means_numpy, pin_bilinearity, pin_threshold_golden, pin_diagonal_kept,
             pin_nesting, pin_weights_sum, pin_exact_correction, pin_gqa_packing, pin_ragged, pin_e4m3_scales,
             pin_chunk_dense_sdpa, pin_chunk_equals_full, pin_chunk_bilinearity, pin_chunk_exact_correction,
-            pin_variance_term, pin_pooled_reduces_to_rows]
+            pin_variance_term, pin_isotropic_variance_term, pin_pooled_reduces_to_rows]

@@ -10,6 +10,8 @@ all 32 query heads.  Corrections:
   variance  the mean correction plus half the within-block logit variance,
             taken per dimension of the keys (oracle correction mode 2);
   pooled    the mean correction with the q-block's mean query (mode 3);
+  isotropic the variance term with the key variance averaged over the
+            dimensions (mode 4): one scalar per row times one per block;
   strided   the mean correction, with kept lists estimated from every 8th
             query row of each block instead of all 128 (the estimator would
             read an eighth of Q).
@@ -68,7 +70,7 @@ def test_correction_variants_against_dense():
     ref = _dense_rows(q, k, v, rows, wl.num_q_heads, wl.num_kv_heads, tau)
     ref_norm = np.linalg.norm(ref)
     err = {}
-    for name, mode in (("none", 0), ("mean", 1), ("variance", 2), ("pooled", 3)):
+    for name, mode in (("none", 0), ("mean", 1), ("variance", 2), ("pooled", 3), ("isotropic", 4)):
         r = orc.attend(q, k, v, cu, 128, tau, est["kept_cnt"], est["kept_idx"], correction=mode, kbar=kb,
                        vbar=vb, kvar=kv, qbar=qb, sel=sel)
         err[name] = float(np.linalg.norm(r["o"][rows] - ref) / ref_norm)
@@ -91,4 +93,5 @@ def test_correction_variants_against_dense():
           + f"; strided: kept lists equal to the full estimate's {same:.3f}, kept density "
           f"{est_s['kept_cnt'].sum() / (wl.num_kv_heads * nb * (nb + 1) / 2):.4f}")
     assert err["variance"] < err["mean"] < err["none"], err
+    assert err["isotropic"] < err["mean"], err
     assert err["strided"] < err["none"], err

@@ -21,6 +21,7 @@ MUTANTS = {
     13: "chunk: partial first q-block mean divided by rows before the chunk too",
     14: "chunk: pruned blocks of the cached prefix get no correction",
     15: "variance variant: the full logit variance added instead of half of it",
+    16: "isotropic variance variant: variances summed, not averaged, over the dimensions",
 }
 
 
