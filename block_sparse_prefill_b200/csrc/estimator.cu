@@ -1,9 +1,9 @@
-// estimator.cu -- the block-score estimator of block-sparse prefill
-// ("computes a small sample of attention scores, finds the maximum, and attends
-// only to tokens that exceed a threshold relative to that max", lode.cx write-up
-// of FlashPrefill V2, section "How It Works"; "estimating scores at the block
-// level", aipulsen.com write-up), plus the small set-up and conversion passes
-// the attention call needs.
+// estimator.cu -- the block-score estimator of block-sparse prefill: a cheap
+// estimate of the attention scores, their maximum, and the blocks whose score
+// clears a threshold set relative to that maximum (lode.cx write-up of
+// FlashPrefill V2, section "How It Works"; the aipulsen.com write-up makes the
+// estimate per block), plus the small set-up and conversion passes the
+// attention call needs.
 //
 //   setup_kernel   validates cu_seqlens, numbers the blocks of the ragged batch
 //   pool_kernel    block means of Q, K, V (HBM-bound streaming pass, every input

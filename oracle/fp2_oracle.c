@@ -15,10 +15,11 @@
  * Definitions (the pages give them in words only; where they are silent the
  * plainest reading is taken and named):
  *   D0 blocks   Request b of length L_b is cut into blocks of Bs rows starting
- *               at its first token ("fixed-size blocks", 345tool.com page,
- *               section "Why block-sparse attention for prefill?"; stuffinsider
- *               page, "Technical Details").  n_j = rows of block j.  Token r sees
- *               tokens c <= r of the same request (causal prefill).
+ *               at its first token (blocks of one fixed size: 345tool.com page,
+ *               section "Why block-sparse attention for prefill?"; queries and
+ *               keys both cut into blocks: stuffinsider page, "Technical
+ *               Details").  n_j = rows of block j.  Token r sees tokens c <= r of
+ *               the same request (causal prefill).
  *               Chunked form (prefill of the last Lq_b of Lk_b tokens, the first
  *               P_b = Lk_b - Lq_b already in the KV cache; the pages name paged KV
  *               and continuous batching but not this case, so the plainest
@@ -28,22 +29,25 @@
  *               [P_b, Lk_b) and the first one may be partial.  Position p sees
  *               keys c <= p.  With P_b = 0 this is the plain definition.
  *   D1 estimate xbar_j = (1/n_j) sum_{r in j} x_r for x in {q, k, v}
- *               (reading of "computes a small sample of attention scores" /
- *               "estimating scores at the block level": block means), and
+ *               (the lode.cx page, "How It Works", estimates the scores from a
+ *               small sample and the aipulsen page does so per block; read here
+ *               as block means), and
  *               s[h,i,j] = tau * qbar[h,i] . kbar[g(h),j] for j <= i, g(h) = h / G.
  *   D2 keep     m = max_{j<=i} s[h,i,j]; head h keeps j iff s - m >= ln(alpha)
- *               ("finds the maximum, and attends only to tokens that exceed a
- *               threshold relative to that max"; read in the probability domain,
- *               exp(s - m) >= alpha).  A KV group keeps the union over its
- *               heads plus the diagonal block i.  alpha <= 0 keeps every j <= i.
+ *               (lode.cx page, "How It Works": only what clears a threshold
+ *               set relative to the maximum estimated score is attended; read in
+ *               the probability domain, exp(s - m) >= alpha).  A KV group keeps
+ *               the union over its heads plus the diagonal block i.  alpha <= 0
+ *               keeps every j <= i.
  *   D3 attend   For row r (head h) of q-block i with kept set K and pruned set
  *               P = {j < i not kept}:
  *               o = [sum_{c in K, c<=r} e^{l_c} v_c + sum_{j in P} n_j e^{lbar_j} vbar_j]
  *                 / [sum_{c in K, c<=r} e^{l_c}     + sum_{j in P} n_j e^{lbar_j}],
  *               l_c = tau q_r . k_c, lbar_j = tau q_r . kbar_j (reading of the
- *               "mean correction term that calibrates for the bias introduced by
- *               pruning": every pruned block replaced by n_j copies of its mean
- *               key and mean value).  LSE = ln(denominator).
+ *               correction term of the lode.cx page, "How It Works", which offsets
+ *               the bias that dropping blocks introduces: every pruned block
+ *               replaced by n_j copies of its mean key and mean value).
+ *               LSE = ln(denominator).
  *   D4 e4m3     inputs are codes times a per-(tensor, head) scale; the oracle
  *               dequantises them exactly in double.
  *   D3 variants (not the method as the pages give it; compared on approximation
