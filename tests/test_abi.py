@@ -230,3 +230,14 @@ def test_length_limit_is_tight(lib, dtype, name):
     gets as far as the first CUDA call and returns FP2_ERR_CUDA."""
     limit = _max_seq_blocks()[name]
     assert _attention_call(lib, "fp2_sparse_prefill", dtype, limit * 128) == 4
+
+
+def test_missing_library_fails_loudly(monkeypatch):
+    """Without libfp2.so every call raises: there is no CPU fallback."""
+    import block_sparse_prefill_b200 as fp2
+    monkeypatch.setattr(_lib, "_lib", None)
+    monkeypatch.setattr(_lib, "LIB_PATH", os.path.join(ROOT, "tests", "_build", "absent", "libfp2.so"))
+    with pytest.raises(RuntimeError, match="no CPU fallback"):
+        fp2.max_blocks(1, 1024)
+    with pytest.raises(RuntimeError, match="no CPU fallback"):
+        fp2.workspace_bytes(fp2.Params(num_q_heads=4, num_kv_heads=2), 1, 1024, 1024)
