@@ -19,7 +19,9 @@ By Jensen's inequality the mean correction undercounts a pruned block's mass by
 about exp(var / 2), which the variance term restores.  The test requires
 variance < mean < none and prints the errors (run with -s).  Set
 FP2_APPROX_SEQLEN=32768 to run the same study at 32K, and FP2_APPROX_ALPHA to change
-alpha.
+alpha.  FP2_APPROX_OUTLIERS="n,gain[,both]" scales n seeded key channels (and the
+same query channels with ",both") by gain: outlier channels, as in trained models,
+make the key variance anisotropic.
 """
 import math
 import os
@@ -32,6 +34,9 @@ from workloads import make_config
 
 SEQLEN = int(os.environ.get("FP2_APPROX_SEQLEN", "8192"))
 ALPHA = float(os.environ.get("FP2_APPROX_ALPHA", "0.05"))
+# "n,gain[,both]": multiply n seeded key channels (and the same query channels with
+# "both") by gain, for key variance that is not isotropic
+OUTLIERS = os.environ.get("FP2_APPROX_OUTLIERS", "")
 
 
 def _dense_rows(q, k, v, rows, hq, hkv, tau):
@@ -57,6 +62,14 @@ def test_correction_variants_against_dense():
     wl = make_config(2, seqlen=SEQLEN, alpha=ALPHA)
     orc = Oracle()
     q, k, v = wl.float_inputs()
+    if OUTLIERS:
+        parts = OUTLIERS.split(",")
+        ch = np.random.default_rng(3).choice(wl.head_dim, int(parts[0]), replace=False)
+        k = k.copy()
+        k[:, :, ch] *= float(parts[1])
+        if len(parts) > 2 and parts[2] == "both":
+            q = q.copy()
+            q[:, :, ch] *= float(parts[1])
     cu = wl.cu_seqlens
     tau = 1.0 / math.sqrt(wl.head_dim)
     qb = orc.block_means(q, cu, 128)
@@ -88,7 +101,8 @@ def test_correction_variants_against_dense():
                     == set(est_s["kept_idx"][t, g, :est_s["kept_cnt"][t, g]].tolist())
                     for t in range(nb) for g in range(wl.num_kv_heads)])
     density = est["kept_cnt"].sum() / (wl.num_kv_heads * nb * (nb + 1) / 2)
-    print(f"\n{SEQLEN} tokens, alpha {wl.alpha}, kept density {density:.4f}, q-blocks {sel.tolist()}: "
+    print(f"\n{SEQLEN} tokens, alpha {wl.alpha}, outliers '{OUTLIERS}', kept density {density:.4f}, "
+          f"q-blocks {sel.tolist()}: "
           + ", ".join(f"{k_} rel-L2 {v_:.4f}" for k_, v_ in err.items())
           + f"; strided: kept lists equal to the full estimate's {same:.3f}, kept density "
           f"{est_s['kept_cnt'].sum() / (wl.num_kv_heads * nb * (nb + 1) / 2):.4f}")
