@@ -12,6 +12,9 @@ all 32 query heads.  Corrections:
   pooled    the mean correction with the q-block's mean query (mode 3);
   isotropic the variance term with the key variance averaged over the
             dimensions (mode 4): one scalar per row times one per block;
+  hybrid8   the variance term with the 8 channels of largest total key
+            variance per KV head kept exactly and the rest averaged (mode 2
+            on variances whose other channels are replaced by their mean);
   strided   the mean correction, with kept lists estimated from every 8th
             query row of each block instead of all 128 (the estimator would
             read an eighth of Q).
@@ -83,9 +86,16 @@ def test_correction_variants_against_dense():
     ref = _dense_rows(q, k, v, rows, wl.num_q_heads, wl.num_kv_heads, tau)
     ref_norm = np.linalg.norm(ref)
     err = {}
-    for name, mode in (("none", 0), ("mean", 1), ("variance", 2), ("pooled", 3), ("isotropic", 4)):
+    # hybrid: per KV head, the 8 channels of largest total variance exact, the rest averaged
+    top = np.argsort(-kv.sum(axis=0), axis=1)[:, :8]                  # [Hkv, 8]
+    exact = np.zeros(kv.shape[1:], bool)
+    exact[np.arange(kv.shape[1])[:, None], top] = True
+    rest_mean = (kv * ~exact).sum(axis=2, keepdims=True) / (~exact).sum(axis=1)[None, :, None]
+    kv_hybrid = np.where(exact[None], kv, rest_mean)
+    for name, mode, kvar in (("none", 0, kv), ("mean", 1, kv), ("variance", 2, kv), ("pooled", 3, kv),
+                             ("isotropic", 4, kv), ("hybrid8", 2, kv_hybrid)):
         r = orc.attend(q, k, v, cu, 128, tau, est["kept_cnt"], est["kept_idx"], correction=mode, kbar=kb,
-                       vbar=vb, kvar=kv, qbar=qb, sel=sel)
+                       vbar=vb, kvar=kvar, qbar=qb, sel=sel)
         err[name] = float(np.linalg.norm(r["o"][rows] - ref) / ref_norm)
     # strided estimate: query means over rows 0, 8, 16, ... of each block; in the
     # subsampled sequence a block is 128 / 8 rows
