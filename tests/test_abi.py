@@ -241,3 +241,31 @@ def test_missing_library_fails_loudly(monkeypatch):
         fp2.max_blocks(1, 1024)
     with pytest.raises(RuntimeError, match="no CPU fallback"):
         fp2.workspace_bytes(fp2.Params(num_q_heads=4, num_kv_heads=2), 1, 1024, 1024)
+
+
+def test_plain_c_client_links_and_calls_the_library(lib):
+    """A C11 program built with gcc against include/fp2.h links libfp2.so and calls
+    the host-only entry points and an argument-error path (no device work)."""
+    import subprocess
+    os.makedirs(PROBE_DIR, exist_ok=True)
+    src = os.path.join(PROBE_DIR, f"c_client_{os.getpid()}.c")
+    exe = src[:-2]
+    libdir = os.path.dirname(_lib.LIB_PATH)
+    with open(src, "w") as f:
+        f.write('#include <stdio.h>\n#include "fp2.h"\nint main(void) {\n'
+                "    fp2_params p = {32, 8, 128, 128, 0.05f, 0.0f, 1, FP2_BF16, NULL, NULL, NULL};\n"
+                '    printf("%d %lld %d %d %s\\n", fp2_version(), (long long)fp2_max_blocks(1, 131072, 128),\n'
+                "           fp2_workspace_bytes(&p, 1, 131072, 131072) > 0,\n"
+                "           (int)fp2_estimate(NULL, NULL, NULL, NULL, NULL, 0, 0, 0, NULL, 0, 0, NULL, NULL, 0, NULL),\n"
+                "           fp2_status_string(FP2_ERR_INVALID_ARG));\n"
+                "    return 0;\n}\n")
+    try:
+        subprocess.run(["gcc", "-std=c11", "-Wall", "-Werror", "-I", os.path.dirname(HEADER), src,
+                        "-L", libdir, "-l:libfp2.so", f"-Wl,-rpath,{libdir}", "-o", exe], check=True)
+        out = subprocess.run([exe], check=True, capture_output=True, text=True).stdout.split()
+    finally:
+        for f in (src, exe):
+            if os.path.exists(f):
+                os.remove(f)
+    assert out[:4] == [str(lib.fp2_version()), "1025", "1", "1"], out
+    assert " ".join(out[4:]) == "invalid argument"
