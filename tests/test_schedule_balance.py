@@ -1,0 +1,91 @@
+"""Load balance of the attention kernel's persistent schedule (host model, no GPU).
+
+The attention kernel runs one CTA per SM (148).  The CTAs take work items (one
+q-block x two query heads of one KV head) from a shared counter, in the order
+the setup kernel writes: by the q-block's index in its request, largest first.
+A CTA that finishes takes the next item, which is greedy list scheduling.
+
+This test models an item's cost as:
+  - its kept K/V tiles, with kept lists from the oracle's estimator;
+  - its correction tiles, ceil(i / 128) for q-block i > 0;
+  - a fill of 2 tiles.
+It compares that order's makespan with the ideal (all work spread evenly) and
+with items ordered by their cost, which is known once the estimator has run.
+On these workloads the cost order is no worse (greedy list scheduling has no
+such guarantee in general).  With many items per CTA both orders are close to
+the ideal:
+  - the paged ragged batch, shortened to 32K, is within 1%;
+  - with FP2_SCHED_FULL=1, the 128K layer and the full batch are within 1%.
+A 32K single request shows the block-index order's tail.  FP2_SCHED_SEQLEN=n
+runs the single-request layer at n tokens and only reports the figures.
+"""
+import heapq
+import math
+import os
+
+import pytest
+
+from oracle.oracle import Oracle
+from workloads import make_config
+
+FULL = os.environ.get("FP2_SCHED_FULL", "") == "1"
+SEQLEN = int(os.environ.get("FP2_SCHED_SEQLEN", "0"))
+SMS = 148
+FILL_TILES = 2.0
+PAIRS = 2          # query-head pairs per KV head at G = 4
+
+
+def _item_costs(wl, kept_cnt):
+    """(q-block index, cost in tiles) of every work item."""
+    items = []
+    t = 0
+    for L in wl.seqlens:
+        for i in range((L + 127) // 128):
+            corr = (i + 127) // 128
+            for g in range(wl.num_kv_heads):
+                items += [(i, FILL_TILES + int(kept_cnt[t, g]) + corr)] * PAIRS
+            t += 1
+    return items
+
+
+def _makespan(costs, m=SMS):
+    """Greedy list scheduling: each item goes to the CTA that frees up first."""
+    busy = [0.0] * m
+    for c in costs:
+        heapq.heappush(busy, heapq.heappop(busy) + c)
+    return max(busy)
+
+
+def _spans(wl):
+    orc = Oracle()
+    q, k, _ = wl.float_inputs()
+    cu = wl.cu_seqlens
+    qb, kb = orc.block_means(q, cu, 128), orc.block_means(k, cu, 128)
+    est = orc.estimate(qb, kb, cu, 128, alpha=wl.alpha, tau=1.0 / math.sqrt(wl.head_dim))
+    items = _item_costs(wl, est["kept_cnt"])
+    ideal = sum(c for _, c in items) / SMS
+    by_index = _makespan([c for _, c in sorted(items, key=lambda x: -x[0])])
+    by_cost = _makespan(sorted((c for _, c in items), reverse=True))
+    return len(items), ideal, by_index, by_cost
+
+
+@pytest.mark.parametrize("cid", [2, 4])
+def test_persistent_schedule_balance(cid):
+    if SEQLEN and cid != 2:
+        pytest.skip("FP2_SCHED_SEQLEN studies the single-request layer")
+    if SEQLEN:
+        wl = make_config(cid, seqlen=SEQLEN)
+    elif FULL:
+        wl = make_config(cid)
+    else:
+        wl = make_config(cid, seqlen=32768)
+    n, ideal, by_index, by_cost = _spans(wl)
+    print(f"\nconfig {cid}, {wl.total_tokens} tokens: {n} items ({n / SMS:.1f} per CTA), ideal {ideal:.0f} "
+          f"tiles; block-index order +{by_index / ideal - 1:.2%}, cost order +{by_cost / ideal - 1:.2%}")
+    if SEQLEN:
+        return
+    assert by_cost <= by_index * 1.0001
+    if FULL or cid == 4:
+        assert by_index <= 1.01 * ideal
+    else:
+        assert by_index <= 1.05 * ideal
