@@ -3,12 +3,14 @@ from __future__ import annotations
 
 import glob
 import os
+import re
 import subprocess
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 LIB = os.path.join(HERE, "libfp2.so")
+REPORT = os.path.join(HERE, "_build", "ptxas.txt")   # ptxas -v output of the last build
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -48,7 +50,32 @@ def build(force: bool = False, verbose: bool = False) -> str:
     if verbose:
         print(res.stdout + res.stderr)
     os.replace(tmp, LIB)
+    os.makedirs(os.path.dirname(REPORT), exist_ok=True)
+    with open(REPORT, "w") as f:
+        f.write(res.stdout + res.stderr)
     return LIB
+
+
+def ptxas_report() -> list:
+    """Registers and spill bytes of every kernel, parsed from the last build's
+    ``-Xptxas -v`` output (rebuilding when that output is missing or stale):
+    a list of dicts with keys name, regs, spill_stores, spill_loads."""
+    if not os.path.exists(REPORT) or not os.path.exists(LIB) or os.path.getmtime(REPORT) < os.path.getmtime(LIB):
+        build(force=True)
+    kernels, cur = [], None
+    for line in open(REPORT):
+        m = re.search(r"Compiling entry function '([^']+)'", line)
+        if m:
+            cur = {"name": m.group(1), "regs": None, "spill_stores": None, "spill_loads": None}
+            kernels.append(cur)
+            continue
+        m = re.search(r"(\d+) bytes spill stores, (\d+) bytes spill loads", line)
+        if m and cur is not None:
+            cur["spill_stores"], cur["spill_loads"] = int(m.group(1)), int(m.group(2))
+        m = re.search(r"Used (\d+) registers", line)
+        if m and cur is not None:
+            cur["regs"] = int(m.group(1))
+    return kernels
 
 
 if __name__ == "__main__":
