@@ -27,6 +27,12 @@ What pins what (definitions D0-D4 in the oracle header):
                     blocks with an exactly diagonal key covariance; block variances
   isotropic_variance_term  D3 variant 4 on Hadamard blocks (isotropic covariance)
   pooled_reduces_to_rows  D3 variant 3 = row-wise correction for block-constant q
+
+``pin_near_threshold`` takes the mask comparison's band function
+(``oracle.oracle.near_threshold``) instead of an oracle build: hand-derived
+near / not-near flags (tests/golden/near_threshold_cases.json) on both sides of
+the band, with |threshold| below and above one, and a GQA union where one head
+of a group is near.
 """
 from __future__ import annotations
 
@@ -586,6 +592,23 @@ def pin_pooled_reduces_to_rows(orc):
     b = orc.attend(q, k, v, cu, 128, TAU, est["kept_cnt"], est["kept_idx"], correction=3, kbar=kb, vbar=vb,
                    qbar=qb)
     assert np.array_equal(a["o"], b["o"]) and np.array_equal(a["lse"], b["lse"]), "pooled != row-wise"
+
+
+def pin_near_threshold(fn):
+    """``fn(s, m, Hkv, alpha, None, rel)`` against the hand-derived flags of
+    tests/golden/near_threshold_cases.json; alpha <= 0 (nothing pruned) has no
+    near-threshold block."""
+    with open(os.path.join(GOLDEN, "near_threshold_cases.json")) as f:
+        c = json.load(f)
+    s = np.array([[[np.nan if x is None else x for x in row] for row in blk] for blk in c["s"]], np.float64)
+    m = np.array(c["m"], np.float64)
+    want = np.array(c["near"], bool)
+    got = np.asarray(fn(s, m, c["num_kv_heads"], c["alpha"], None, c["rel"]))
+    assert got.shape == want.shape, f"near-threshold flags of shape {got.shape}, expected {want.shape}"
+    bad = np.argwhere(got != want)
+    assert bad.size == 0, f"near-threshold flags differ at (q-block, KV head, key block) {bad.tolist()}"
+    none = np.asarray(fn(s, m, c["num_kv_heads"], 0.0, None, c["rel"]))
+    assert not none.any(), "alpha <= 0 prunes nothing, so no block can be near the threshold"
 
 
 ALL_PINS = [pin_dense_sdpa, pin_means_numpy, pin_bilinearity, pin_threshold_golden, pin_diagonal_kept,

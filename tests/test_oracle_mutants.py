@@ -1,7 +1,12 @@
 """Every mistake planted in the oracle (built with -DORC_MUTANT=n) must trip at
 least one pin, so the pins would notice such a mistake in the oracle itself."""
+import inspect
+import math
+
+import numpy as np
 import pytest
 
+from oracle import oracle as oracle_mod
 from oracle.oracle import Oracle
 import oracle_pins
 
@@ -36,3 +41,29 @@ def test_mutant_is_caught(mutant):
         except (AssertionError, ValueError):
             tripped.append(pin.__name__)
     assert tripped, f"planted mistake '{MUTANTS[mutant]}' passes every pin"
+
+
+# Planted mistakes in the mask comparison's band (oracle.oracle.near_threshold),
+# each one textual edit of the function's source.
+NEAR_MUTANTS = {
+    "band without the absolute floor of one": (
+        "band = rel * np.maximum(1.0, np.abs(thr))", "band = rel * np.abs(thr)"),
+    "band scaled by ln(alpha) instead of the threshold": (
+        "band = rel * np.maximum(1.0, np.abs(thr))", "band = rel * np.maximum(1.0, np.abs(0.0 * thr + math.log(alpha)))"),
+    "union over the wrong head axis (group h % Hkv)": (
+        "reshape(nblk, kept_shape_groups, G, nb_max).any(axis=2)",
+        "reshape(nblk, G, kept_shape_groups, nb_max).any(axis=1)"),
+    "distance to the row max instead of the threshold": (
+        "np.abs(s - thr[:, :, None])", "np.abs(s - m[:, :, None])"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(NEAR_MUTANTS))
+def test_near_threshold_mutant_is_caught(name):
+    old, new = NEAR_MUTANTS[name]
+    src = inspect.getsource(oracle_mod.near_threshold)
+    assert old in src, f"mutation site '{old}' not found in near_threshold"
+    ns = {"np": np, "math": math}
+    exec(src.replace(old, new), ns)
+    with pytest.raises(AssertionError):
+        oracle_pins.pin_near_threshold(ns["near_threshold"])
