@@ -499,12 +499,39 @@ def weak_scaling_value(world: int, flops_per_rank: float, ms_max: float) -> floa
     return world * flops_per_rank / (ms_max * 1e-3) / 1e12
 
 
-def cpu_baseline(wl, fracs=(0.25, 0.5)):
+def mask_parity(wl, est, gpu_cnt, gpu_idx, near_threshold):
+    """The GPU's kept lists against the oracle's (`est`, with scores): entries that differ
+    outside the near-threshold band (|s - (m + ln alpha)| <= 1e-3 max(1, |m + ln alpha|) for
+    some head of the group, oracle fp64 scores), differences the band excuses, blocks in the
+    band, and blocks compared (union of both lists).  `near_threshold` is the oracle's band
+    function (passed in by the CPU baseline leg, the one place the oracle is used)."""
+    near = near_threshold(est["s"], est["m"], wl.num_kv_heads, wl.alpha, None)
+    nblk, hkv = est["kept_cnt"].shape
+    outside = excused = compared = 0
+    for t in range(nblk):
+        for g in range(hkv):
+            a = set(gpu_idx[t, g, :gpu_cnt[t, g]].tolist())
+            b = set(est["kept_idx"][t, g, :est["kept_cnt"][t, g]].tolist())
+            compared += len(a | b)
+            for j in a ^ b:
+                if near[t, g, j]:
+                    excused += 1
+                else:
+                    outside += 1
+    return {"near_threshold_blocks": int(near.sum()), "excused_mismatches": excused,
+            "mismatches_outside_band": outside, "blocks_compared": compared,
+            "rule": "kept lists equal to the fp64 oracle's except blocks within 1e-3 (relative, floor 1) of "
+                    "the threshold m + ln(alpha) for some head of the group"}
+
+
+def cpu_baseline(wl, fracs=(0.25, 0.5), gpu_kept=None):
     """The oracle (fp64, OpenMP over host cores) on a bounded sample of the
     layer: the full estimator, plus attention on the q-blocks at the given
     fractions of the sequence (all heads); the per-layer time is extrapolated
-    from the sample by its share of the layer's attention work."""
-    from oracle.oracle import Oracle
+    from the sample by its share of the layer's attention work.  With
+    `gpu_kept` = (kept_cnt, kept_idx) of the GPU run, the result also holds the
+    mask comparison against the oracle's estimate (`mask_parity`)."""
+    from oracle.oracle import Oracle, near_threshold
     orc = Oracle()
     q, k, v = wl.float_inputs()
     cu = wl.cu_seqlens
@@ -512,8 +539,12 @@ def cpu_baseline(wl, fracs=(0.25, 0.5)):
     qb = orc.block_means(q, cu, 128, wl.q_scale)
     kb = orc.block_means(k, cu, 128, wl.k_scale)
     vb = orc.block_means(v, cu, 128, wl.v_scale)
-    est = orc.estimate(qb, kb, cu, 128, wl.alpha, 1.0 / math.sqrt(wl.head_dim))
+    est = orc.estimate(qb, kb, cu, 128, wl.alpha, 1.0 / math.sqrt(wl.head_dim), want_scores=gpu_kept is not None)
     t_est = time.perf_counter() - t0
+    parity = None
+    if gpu_kept is not None:
+        parity = mask_parity(wl, est, gpu_kept[0][:est["kept_cnt"].shape[0]], gpu_kept[1][:est["kept_cnt"].shape[0]],
+                             near_threshold)
     nblk = est["kept_cnt"].shape[0]
     sel = np.unique(np.array([min(nblk - 1, int(f * nblk)) for f in fracs], dtype=np.int64))
     t1 = time.perf_counter()
@@ -542,7 +573,7 @@ def cpu_baseline(wl, fracs=(0.25, 0.5)):
     except AttributeError:
         pass
     omp = int(os.environ.get("OMP_NUM_THREADS", cores))
-    return {
+    res = {
         "value": flops_all / t_layer / 1e12, "unit": "TFLOP/s", "cores": min(cores, omp), "kind": "oracle",
         "ms_per_layer": t_layer * 1e3,
         "sample": (f"fp64 oracle: full estimator ({t_est:.1f} s) + attention on {len(sel)} of {nblk} "
@@ -550,6 +581,9 @@ def cpu_baseline(wl, fracs=(0.25, 0.5)):
                    "attention work); "
                    "layer time extrapolated by work share"),
     }
+    if parity is not None:
+        res["mask_parity"] = parity
+    return res
 
 
 def ours(args):
@@ -616,6 +650,8 @@ def ours(args):
             "tflops_attention": (f8 + c8) / (a8 * 1e-3) / 1e12,
             "tensor_peak_tflops": peak8,
             "frac_attention": (f8 + c8) / (a8 * 1e-3) / 1e12 / peak8,
+            "tflops_attention_kept_pairs_only": f8 / (a8 * 1e-3) / 1e12,
+            "frac_attention_kept_pairs_only": f8 / (a8 * 1e-3) / 1e12 / peak8,
             "peak_note": note8,
             "frac_attention_of_2x_bf16": (f8 + c8) / (a8 * 1e-3) / 1e12 / (peaks["bf16_tflops"] * E4M3_OVER_BF16),
         }
@@ -676,9 +712,14 @@ def ours(args):
         "roofline": {
             "bound": "tensor", "achieved": ach_att, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
             "frac": ach_att / peaks["bf16_tflops"],
+            # the same kernel time over the kept-pair work alone (the effective TFLOP/s on kept
+            # blocks); the correction's share of the work is counted only in `frac`
+            "achieved_kept_pairs_only": flops / (ms_att * 1e-3) / 1e12,
+            "frac_kept_pairs_only": flops / (ms_att * 1e-3) / 1e12 / peaks["bf16_tflops"],
             "traffic": TRAFFIC_128K["attention"] if wl.max_seqlen == 131072 else None,
             "kernel": "attention_kernel<bf16> (fp2_sparse_prefill call)",
-            "work": "4*d flops per kept causal query-key pair + 4*d per (row, pruned block) correction term",
+            "work": "4*d flops per kept causal query-key pair + 4*d per (row, pruned block) correction term "
+                    "(kept pairs and the mean correction, both steps of the method)",
             "peak_kind": f"{peaks_kind} bf16 burst",
             # the timed steps run back to back and reach the power cap within ~0.1 s (clocks),
             # so the sustained-GEMM figure is shown beside the burst one
@@ -701,10 +742,35 @@ def ours(args):
     if comp is not None:
         line["comparators"] = comp
     if ctx.rank == 0 and ctx.world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(wl)
+        cb = cpu_baseline(wl, gpu_kept=(kept_cnt, kept_idx))
+        line["mask_parity"] = cb.pop("mask_parity")
+        line["cpu_baseline"] = cb
     if ctx.rank == 0:
         print(json.dumps(line), flush=True)
     ctx.close()
+
+
+def e4m3_only(args):
+    """The e4m3 layer alone (1 GPU): `--warmup` untimed and `--steps` timed layers, one JSON
+    line with its times.  Used to profile the e4m3 attention kernel without bf16 launches."""
+    import torch
+    import block_sparse_prefill_b200 as fp2
+    from workloads import make_config
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    wl8 = make_config(3, seqlen=args.seqlen)
+    st8 = setup_layer(wl8, dev)
+    tot8, est8, att8, _ = time_layer(st8, wl8, args.steps, args.warmup, DistCtx())
+    err = fp2.get_error(st8["ws"])
+    if err != 0:
+        raise RuntimeError(f"device error: {fp2.status_string(err)}")
+    f8, c8 = layer_work(wl8.seqlens, st8["meta"].kept_cnt.cpu().numpy(), st8["meta"].kept_idx.cpu().numpy(),
+                        wl8.num_q_heads, wl8.num_kv_heads)
+    a8 = statistics.mean(att8)
+    print(json.dumps({"workload": f"{wl8.max_seqlen // 1024}K e4m3 (Hq=32, Hkv=8, d=128, alpha=0.05)",
+                      "ms_per_layer": tot8 / args.steps, "ms_estimate": statistics.mean(est8),
+                      "ms_attention": a8, "tflops_attention": (f8 + c8) / (a8 * 1e-3) / 1e12,
+                      "tflops_attention_kept_pairs_only": f8 / (a8 * 1e-3) / 1e12}), flush=True)
 
 
 def reference(args):
@@ -752,11 +818,16 @@ def main():
                          "flash_attn), timed as context for the speedup at 1 GPU")
     ap.add_argument("--seqlen", type=int, default=None,
                     help="shorter sequence for profiling runs (default: the 128K workload)")
+    ap.add_argument("--e4m3-only", action="store_true",
+                    help="profiling aid: time only the e4m3 layer (config 3) and print its line, so that "
+                         "a profiler sees no bf16 launch")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
         reference(args)
+    elif args.e4m3_only:
+        e4m3_only(args)
     else:
         ours(args)
 

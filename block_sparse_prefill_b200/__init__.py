@@ -9,6 +9,15 @@ missing library raises.
     ws = Workspace(params, batch, total_tokens, max_seqlen, device)
     estimate(params, q, k, v, cu_seqlens, max_seqlen, meta, ws)
     sparse_prefill(params, q, k, v, cu_seqlens, max_seqlen, meta, out, ws, lse=lse)
+
+Paged KV cache: ``estimate(..., block_table=bt, num_pages=n)`` on the page
+pools, then ``prefill_paged(params, q, k_pool, v_pool, cu_seqlens, max_seqlen,
+bt, n, meta, out, ws, lse=lse)``.
+
+Chunked prefill (queries are the last rows of each request, the earlier keys
+already cached): ``estimate_chunked`` and ``prefill_chunked`` with
+``cu_seqlens_q`` (query rows) and ``cu_seqlens_k`` (keys); size the meta and the
+workspace by the total keys.
 """
 from __future__ import annotations
 
@@ -22,7 +31,8 @@ from . import _lib
 from ._lib import FP2_BF16, FP2_E4M3, STATUS
 
 __all__ = ["Params", "BlockMeta", "Workspace", "FP2Error", "max_blocks", "workspace_bytes",
-           "estimate", "sparse_prefill", "sparse_prefill_noalloc", "prefill_paged", "get_error",
+           "estimate", "sparse_prefill", "sparse_prefill_noalloc", "prefill_paged", "estimate_chunked",
+           "prefill_chunked", "get_error",
            "status_string", "version",
            "FP2_BF16", "FP2_E4M3"]
 
@@ -248,7 +258,10 @@ def sparse_prefill(params: Params, q, k, v, cu_seqlens, max_seqlen: int, meta: B
 
 def prefill_paged(params: Params, q, k_pool, v_pool, cu_seqlens, max_seqlen: int, block_table,
                   num_pages: int, meta: BlockMeta, out, ws: Workspace, lse=None, stream=None) -> None:
-    """``fp2_prefill_paged``: estimator + attention on a paged KV cache."""
+    """``fp2_prefill_paged``: ``sparse_prefill`` on a paged KV cache (K/V tiles read
+    page by page through ``block_table``).  ``meta`` is only read: fill it with
+    ``estimate(..., block_table=block_table, num_pages=num_pages)`` on the same
+    pools, or pass kept lists of your own."""
     where = "fp2_prefill_paged"
     if block_table is None:
         raise TypeError(f"{where}: block_table is required")
@@ -281,6 +294,71 @@ def sparse_prefill_noalloc(params: Params, q, k, v, cu_seqlens, max_seqlen: int,
                                                   int(max_seqlen), ctypes.byref(m), _ptr(out), _ptr(lse),
                                                   _ptr(device_status), _stream(stream)),
            "fp2_sparse_prefill_noalloc")
+
+
+def _chunk_args(params: Params, where: str, q, k, v, cu_q, cu_k, out=None, lse=None, block_table=None,
+                num_pages: int = 0):
+    """Layouts of a chunked call: q / out / lse [total_q, ...], k / v [total_k, Hkv, d] (or page
+    pools), cu_seqlens_q and cu_seqlens_k [batch + 1] int32."""
+    for name, t in (("cu_seqlens_q", cu_q), ("cu_seqlens_k", cu_k)):
+        if t is None:
+            raise TypeError(f"{where}: {name} is required")
+        _arg(t, name, (torch.int32,), (None,), where)
+    if cu_q.numel() != cu_k.numel() or cu_q.numel() < 1:
+        raise ValueError(f"{where}: cu_seqlens_q and cu_seqlens_k need the same batch + 1 >= 1 entries")
+    _arg(block_table, "block_table", (torch.int32,), (int(cu_q.numel()) - 1, None), where)
+    params.check(where)
+    io = (torch.bfloat16,) if params.dtype == FP2_BF16 else _E4M3_DTYPES
+    d, hq, hkv = params.head_dim, params.num_q_heads, params.num_kv_heads
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if t is None:
+            raise TypeError(f"{where}: {name} is required")
+    _arg(q, "q", io, (None, hq, d), where)
+    rows = None if block_table is None else int(num_pages) * params.block_size
+    _arg(k, "k", io, (rows, hkv, d), where)
+    _arg(v, "v", io, (int(k.shape[0]), hkv, d), where)
+    Tq = int(q.shape[0])
+    _arg(out, "out", (torch.bfloat16,), (Tq, hq, d), where)
+    _arg(lse, "lse", (torch.float32,), (Tq, hq), where)
+    _same_cuda(where, q=q, k=k, v=v, cu_seqlens_q=cu_q, cu_seqlens_k=cu_k, out=out, lse=lse,
+               block_table=block_table, q_scale=params.q_scale, k_scale=params.k_scale, v_scale=params.v_scale)
+
+
+def estimate_chunked(params: Params, q, k, v, cu_seqlens_q, cu_seqlens_k, total_k: int, max_seqlen_k: int,
+                     meta: BlockMeta, ws: Workspace, block_table: Optional[torch.Tensor] = None,
+                     num_pages: int = 0, stream=None) -> None:
+    """``fp2_estimate_chunked``: kept lists of the chunk's q-blocks (and the key-block
+    means of all keys) into ``meta``.  ``total_k`` = cu_seqlens_k[-1] (the keys of the
+    batch; with contiguous K/V, k.shape[0])."""
+    where = "fp2_estimate_chunked"
+    _chunk_args(params, where, q, k, v, cu_seqlens_q, cu_seqlens_k, block_table=block_table, num_pages=num_pages)
+    if block_table is None and int(total_k) != int(k.shape[0]):
+        raise ValueError(f"{where}: total_k = {total_k} but k has {k.shape[0]} rows")
+    p, m = params.c(), meta.c()
+    bt, mbps, npg = _bt_args(block_table, num_pages)
+    _check(_lib.load().fp2_estimate_chunked(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens_q),
+                                            _ptr(cu_seqlens_k), int(cu_seqlens_q.numel()) - 1, int(q.shape[0]),
+                                            int(total_k), int(max_seqlen_k), bt, mbps, npg, ctypes.byref(m),
+                                            ws.ptr, ws.nbytes, _stream(stream)),
+           where)
+
+
+def prefill_chunked(params: Params, q, k, v, cu_seqlens_q, cu_seqlens_k, total_k: int, max_seqlen_k: int,
+                    meta: BlockMeta, out, ws: Workspace, lse=None, block_table: Optional[torch.Tensor] = None,
+                    num_pages: int = 0, stream=None) -> None:
+    """``fp2_prefill_chunked``: attention of the chunk rows over the kept blocks of all
+    keys (+ mean correction), contiguous K/V or page pools through ``block_table``."""
+    where = "fp2_prefill_chunked"
+    _chunk_args(params, where, q, k, v, cu_seqlens_q, cu_seqlens_k, out, lse, block_table, num_pages)
+    if block_table is None and int(total_k) != int(k.shape[0]):
+        raise ValueError(f"{where}: total_k = {total_k} but k has {k.shape[0]} rows")
+    p, m = params.c(), meta.c()
+    bt, mbps, npg = _bt_args(block_table, num_pages)
+    _check(_lib.load().fp2_prefill_chunked(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens_q),
+                                           _ptr(cu_seqlens_k), int(cu_seqlens_q.numel()) - 1, int(q.shape[0]),
+                                           int(total_k), int(max_seqlen_k), bt, mbps, npg, ctypes.byref(m),
+                                           _ptr(out), _ptr(lse), ws.ptr, ws.nbytes, _stream(stream)),
+           where)
 
 
 def get_error(ws: Workspace, stream=None) -> int:

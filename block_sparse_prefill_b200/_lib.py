@@ -18,7 +18,7 @@ STATUS = {
 # every function the header declares
 EXPORTS = ["fp2_max_blocks", "fp2_workspace_bytes", "fp2_workspace_init", "fp2_estimate",
            "fp2_sparse_prefill", "fp2_prefill_paged", "fp2_get_error", "fp2_status_string",
-           "fp2_version", "fp2_sparse_prefill_noalloc"]
+           "fp2_version", "fp2_sparse_prefill_noalloc", "fp2_estimate_chunked", "fp2_prefill_chunked"]
 
 NOALLOC_SCRATCH_BYTES = 8 << 20  # FP2_NOALLOC_SCRATCH_BYTES
 
@@ -83,6 +83,12 @@ def load():
     lib.fp2_prefill_paged.argtypes = [_PP, _P, _P, _P, _P, _I32, _I64, _I32, _P, _I32, _I32, _PM, _P, _P,
                                       _P, _SZ, _P]
     lib.fp2_prefill_paged.restype = ctypes.c_int
+    lib.fp2_estimate_chunked.argtypes = [_PP, _P, _P, _P, _P, _P, _I32, _I64, _I64, _I32, _P, _I32, _I32, _PM,
+                                         _P, _SZ, _P]
+    lib.fp2_estimate_chunked.restype = ctypes.c_int
+    lib.fp2_prefill_chunked.argtypes = [_PP, _P, _P, _P, _P, _P, _I32, _I64, _I64, _I32, _P, _I32, _I32, _PM,
+                                        _P, _P, _P, _SZ, _P]
+    lib.fp2_prefill_chunked.restype = ctypes.c_int
     lib.fp2_get_error.argtypes = [_P, _P]
     lib.fp2_get_error.restype = ctypes.c_int
     lib.fp2_status_string.argtypes = [ctypes.c_int]

@@ -111,28 +111,36 @@ float tau_of(const fp2_params* p) {
 
 struct Problem {
     int32_t batch;
-    int64_t total_tokens;
-    int32_t max_seqlen;
-    int64_t max_blocks;   // host bound of sum_b nb_b
+    int64_t total_q;      // query rows (= total_k for plain prefill)
+    int64_t total_k;      // keys
+    int32_t max_seqlen;   // >= every request's keys
+    int64_t max_blocks;   // host bound of the key blocks sum_b ceil(Lk_b / bs) (>= q-blocks)
+    int64_t max_qblocks;  // host bound of the q-blocks (<= max_blocks)
     int32_t nb_need;      // ceil(max_seqlen / block)
     WsLayout ws;
 };
 
+// Plain prefill passes the same cu_seqlens and total for queries and keys.
 fp2_status check_problem(const fp2_params* p, const void* q, const void* k, const void* v,
-                         const int32_t* cu, int32_t batch, int64_t total_tokens,
-                         int32_t max_seqlen, void* workspace, size_t ws_bytes, Problem* out) {
+                         const int32_t* cu_q, const int32_t* cu_k, int32_t batch, int64_t total_q,
+                         int64_t total_k, int32_t max_seqlen, void* workspace, size_t ws_bytes,
+                         Problem* out) {
     fp2_status st = check_params(p);
     if (st != FP2_OK) return st;
-    if (batch < 0 || total_tokens < 0 || max_seqlen < 0) return FP2_ERR_INVALID_ARG;
-    if (total_tokens > (int64_t(1) << 31) - 1) return FP2_ERR_UNSUPPORTED;
-    if (batch > 0 && !cu) return FP2_ERR_INVALID_ARG;
-    if (total_tokens > 0 && (!q || !k || !v)) return FP2_ERR_INVALID_ARG;
+    if (batch < 0 || total_q < 0 || total_k < 0 || max_seqlen < 0) return FP2_ERR_INVALID_ARG;
+    if (total_q > total_k) return FP2_ERR_INVALID_ARG;
+    if (total_k > (int64_t(1) << 31) - 1) return FP2_ERR_UNSUPPORTED;
+    if (batch > 0 && (!cu_q || !cu_k)) return FP2_ERR_INVALID_ARG;
+    if ((total_q > 0 && !q) || (total_k > 0 && (!k || !v))) return FP2_ERR_INVALID_ARG;
     if ((q && !aligned(q, 16)) || (k && !aligned(k, 16)) || (v && !aligned(v, 16)))
         return FP2_ERR_INVALID_ARG;
     out->batch = batch;
-    out->total_tokens = total_tokens;
+    out->total_q = total_q;
+    out->total_k = total_k;
     out->max_seqlen = max_seqlen;
-    out->max_blocks = fp2_max_blocks(batch, total_tokens, kBlock);
+    out->max_blocks = fp2_max_blocks(batch, total_k, kBlock);
+    // a request's q-blocks: at most ceil(Lq / bs) + 1 (the first one partial)
+    out->max_qblocks = std::min<int64_t>(out->max_blocks, fp2_max_blocks(batch, total_q, kBlock) + batch);
     out->nb_need = (max_seqlen + kBlock - 1) / kBlock;
     out->ws = ws_layout(batch, out->max_blocks, p->num_q_heads, p->num_kv_heads, esize(p));
     if (!workspace || !aligned(workspace, 256) || ws_bytes < out->ws.total) return FP2_ERR_WORKSPACE;
@@ -168,23 +176,27 @@ bool score_tiling(int32_t G, int32_t* qt) {
 // tiles in y.
 fp2_status check_limits(const fp2_params* p, const Problem& pr, bool estimate, bool attention) {
     const int32_t nb_cap = pr.nb_need > 0 ? pr.nb_need : 1;
-    if (sizeof(int32_t) * (nb_cap + 1) > kMaxSmem) return FP2_ERR_UNSUPPORTED;
+    if (sizeof(int32_t) * (setup_bins(nb_cap, attention) + 1) > kMaxSmem) return FP2_ERR_UNSUPPORTED;
     if (estimate) {
         int32_t qt;
         if (!score_tiling(p->num_q_heads / p->num_kv_heads, &qt)) return FP2_ERR_UNSUPPORTED;
-        if ((pr.max_blocks + qt - 1) / qt + pr.batch > 65535) return FP2_ERR_UNSUPPORTED;
+        if ((pr.max_qblocks + qt - 1) / qt + pr.batch > 65535) return FP2_ERR_UNSUPPORTED;
     }
     if (attention && attn_smem_bytes(p->dtype == FP2_E4M3, pr.nb_need) > kMaxSmem)
         return FP2_ERR_UNSUPPORTED;
     return FP2_OK;
 }
 
-fp2_status run_setup(const Problem& pr, void* ws, const int32_t* cu, int32_t qt, bool paged,
-                     int32_t mbps, int64_t meta_blocks, cudaStream_t s) {
+// kept_cnt != NULL (the attention call): work items ordered by cost.
+fp2_status run_setup(const Problem& pr, void* ws, const int32_t* cu_q, const int32_t* cu_k, int32_t qt,
+                     bool paged, int32_t mbps, int64_t meta_blocks, cudaStream_t s,
+                     const int32_t* kept_cnt = nullptr, int32_t hkv = 0, int32_t correction = 0) {
     SetupArgs sa;
-    sa.cu = cu;
+    sa.cu_q = cu_q;
+    sa.cu_k = cu_k;
     sa.batch = pr.batch;
-    sa.total_tokens = pr.total_tokens;
+    sa.total_q = pr.total_q;
+    sa.total_k = pr.total_k;
     sa.max_seqlen = pr.max_seqlen;
     sa.qt = qt;
     sa.paged = paged ? 1 : 0;
@@ -193,10 +205,15 @@ fp2_status run_setup(const Problem& pr, void* ws, const int32_t* cu, int32_t qt,
     sa.nb_cap = pr.nb_need > 0 ? pr.nb_need : 1;
     sa.hdr = at<WsHeader>(ws, 0);
     sa.cu_blocks = at<int32_t>(ws, pr.ws.cu_blocks);
+    sa.cu_qblocks = at<int32_t>(ws, pr.ws.cu_qblocks);
     sa.cu_tiles = at<int32_t>(ws, pr.ws.cu_tiles);
     sa.blk_req = at<int32_t>(ws, pr.ws.blk_req);
+    sa.blk_req_q = at<int32_t>(ws, pr.ws.blk_req_q);
     sa.order = at<int32_t>(ws, pr.ws.order);
-    const size_t hist_bytes = sizeof(int32_t) * (sa.nb_cap + 1);
+    sa.kept_cnt = kept_cnt;
+    sa.hkv = hkv;
+    sa.correction = correction;
+    const size_t hist_bytes = sizeof(int32_t) * (setup_bins(sa.nb_cap, kept_cnt != nullptr) + 1);
     if (hist_bytes > kMaxSmem) return FP2_ERR_UNSUPPORTED;
     if (hist_bytes > 48 * 1024 &&
         cudaFuncSetAttribute(setup_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -207,18 +224,18 @@ fp2_status run_setup(const Problem& pr, void* ws, const int32_t* cu, int32_t qt,
 }
 
 fp2_status run_estimate(const fp2_params* p, const void* q, const void* k, const void* v,
-                        const int32_t* cu, const Problem& pr, const int32_t* block_table,
-                        int32_t mbps, int32_t num_pages, fp2_blockmeta* meta, void* ws,
-                        cudaStream_t s) {
+                        const int32_t* cu_q, const int32_t* cu_k, const Problem& pr,
+                        const int32_t* block_table, int32_t mbps, int32_t num_pages,
+                        fp2_blockmeta* meta, void* ws, cudaStream_t s) {
     const int32_t G = p->num_q_heads / p->num_kv_heads;
     fp2_status st = check_limits(p, pr, true, false);
     if (st != FP2_OK) return st;
     int32_t qt;
     score_tiling(G, &qt);
-    st = run_setup(pr, ws, cu, qt, block_table != nullptr, mbps, meta->max_blocks, s);
-    // an empty batch (no requests, or only empty ones) ends after the setup
-    // kernel has checked cu_seqlens: there is no block to pool or score
-    if (st != FP2_OK || pr.batch == 0 || pr.total_tokens == 0) return st;
+    st = run_setup(pr, ws, cu_q, cu_k, qt, block_table != nullptr, mbps, meta->max_blocks, s);
+    // a batch without query rows ends after the setup kernel has checked the
+    // cu_seqlens arrays: there is no q-block to score
+    if (st != FP2_OK || pr.batch == 0 || pr.total_q == 0) return st;
 
     const bool e4m3 = p->dtype == FP2_E4M3;
     WsHeader* hdr = at<WsHeader>(ws, 0);
@@ -247,17 +264,20 @@ fp2_status run_estimate(const fp2_params* p, const void* q, const void* k, const
     pa.paged[1] = pa.paged[2] = block_table ? 1 : 0;
     pa.first = 0;
     pa.last = meta->v_mean ? 3 : 2;
-    pa.cu = cu;
+    pa.cu_q = cu_q;
+    pa.cu_k = cu_k;
     pa.cu_blocks = at<int32_t>(ws, pr.ws.cu_blocks);
+    pa.cu_qblocks = at<int32_t>(ws, pr.ws.cu_qblocks);
     pa.blk_req = at<int32_t>(ws, pr.ws.blk_req);
+    pa.blk_req_q = at<int32_t>(ws, pr.ws.blk_req_q);
     pa.block_table = block_table;
     pa.max_blocks_per_seq = mbps;
     pa.num_pages = num_pages;
     pa.hdr = hdr;
-    const int32_t ys = pa.slabs[0] + pa.slabs[1] + (pa.last == 3 ? pa.slabs[2] : 0);
-    const int64_t kv_rows = block_table ? int64_t(num_pages) * kBlock : pr.total_tokens;
+    const int32_t yskv = pa.slabs[1] + (pa.last == 3 ? pa.slabs[2] : 0);
+    const int64_t kv_rows = block_table ? int64_t(num_pages) * kBlock : pr.total_k;
     CUtensorMap pq, pk, pv;
-    if (!make_map_pool(&pq, q, e4m3, p->num_q_heads, pr.total_tokens, pa.hb[0]) ||
+    if (!make_map_pool(&pq, q, e4m3, p->num_q_heads, pr.total_q, pa.hb[0]) ||
         !make_map_pool(&pk, k, e4m3, p->num_kv_heads, kv_rows, pa.hb[1]) ||
         !make_map_pool(&pv, v, e4m3, p->num_kv_heads, kv_rows, pa.hb[2]))
         return FP2_ERR_CUDA;
@@ -266,7 +286,7 @@ fp2_status run_estimate(const fp2_params* p, const void* q, const void* k, const
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
         return FP2_ERR_CUDA;
-    const int64_t units = pr.max_blocks * ys;
+    const int64_t units = pr.max_qblocks * pa.slabs[0] + pr.max_blocks * yskv;
     const unsigned pgrid = static_cast<unsigned>(units < sms ? units : sms);
     const size_t psmem = pool_smem_bytes(e4m3);
     if (cudaFuncSetAttribute(e4m3 ? pool_kernel<true> : pool_kernel<false>,
@@ -280,7 +300,10 @@ fp2_status run_estimate(const fp2_params* p, const void* q, const void* k, const
     if ((st = launched(cudaGetLastError())) != FP2_OK) return st;
 
     ScoreArgs sa;
+    sa.cu_q = cu_q;
+    sa.cu_k = cu_k;
     sa.cu_blocks = at<int32_t>(ws, pr.ws.cu_blocks);
+    sa.cu_qblocks = at<int32_t>(ws, pr.ws.cu_qblocks);
     sa.cu_tiles = at<int32_t>(ws, pr.ws.cu_tiles);
     sa.batch = pr.batch;
     sa.hq = p->num_q_heads;
@@ -308,24 +331,24 @@ fp2_status run_estimate(const fp2_params* p, const void* q, const void* k, const
     if (cudaFuncSetAttribute(score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess)
         return FP2_ERR_CUDA;
-    const int64_t tiles = (pr.max_blocks + qt - 1) / qt + pr.batch;  // <= 65535 (check_limits)
+    const int64_t tiles = (pr.max_qblocks + qt - 1) / qt + pr.batch;  // <= 65535 (check_limits)
     score_kernel<<<dim3(static_cast<unsigned>(p->num_kv_heads), static_cast<unsigned>(tiles)),
                    kScoreThreads, smem, s>>>(sa, tqh, tql, tkh, tkl);
     return launched(cudaGetLastError());
 }
 
 fp2_status run_attention(const fp2_params* p, const void* q, const void* k, const void* v,
-                         const int32_t* cu, const Problem& pr, const int32_t* block_table,
+                         const int32_t* cu_q, const int32_t* cu_k, const Problem& pr,
+                         const int32_t* block_table,
                          int32_t mbps, int32_t num_pages, const fp2_blockmeta* meta, void* out,
-                         float* lse, void* ws, cudaStream_t s, bool need_setup) {
+                         float* lse, void* ws, cudaStream_t s) {
     const bool e4m3 = p->dtype == FP2_E4M3;
     fp2_status st = check_limits(p, pr, false, true);
     if (st != FP2_OK) return st;
-    if (need_setup) {
-        st = run_setup(pr, ws, cu, 1, block_table != nullptr, mbps, meta->max_blocks, s);
-        if (st != FP2_OK) return st;
-    }
-    if (pr.batch == 0 || pr.total_tokens == 0) return FP2_OK;  // no rows to attend
+    st = run_setup(pr, ws, cu_q, cu_k, 1, block_table != nullptr, mbps, meta->max_blocks, s,
+                   meta->kept_cnt, p->num_kv_heads, p->correction);
+    if (st != FP2_OK) return st;
+    if (pr.batch == 0 || pr.total_q == 0) return FP2_OK;  // no rows to attend
     WsHeader* hdr = at<WsHeader>(ws, 0);
     void* kb_lp = at<void>(ws, pr.ws.kbar_lp);
     void* vb_lp = at<void>(ws, pr.ws.vbar_lp);
@@ -344,18 +367,20 @@ fp2_status run_attention(const fp2_params* p, const void* q, const void* k, cons
         meanlp_kernel<<<592, 256, 0, s>>>(ma);
         if ((st = launched(cudaGetLastError())) != FP2_OK) return st;
     }
-    const int64_t kv_rows = block_table ? int64_t(num_pages) * kBlock : pr.total_tokens;
+    const int64_t kv_rows = block_table ? int64_t(num_pages) * kBlock : pr.total_k;
     CUtensorMap tq, tk, tv, tkb, tvb;
-    if (!make_map(&tq, q, e4m3, p->num_q_heads, pr.total_tokens) ||
+    if (!make_map(&tq, q, e4m3, p->num_q_heads, pr.total_q) ||
         !make_map(&tk, k, e4m3, p->num_kv_heads, kv_rows) ||
         !make_map(&tv, v, e4m3, p->num_kv_heads, kv_rows) ||
         !make_map(&tkb, kb_lp, e4m3, p->num_kv_heads, pr.max_blocks) ||
         !make_map(&tvb, vb_lp, e4m3, p->num_kv_heads, pr.max_blocks))
         return FP2_ERR_CUDA;
     AttnArgs a;
-    a.cu = cu;
+    a.cu_q = cu_q;
+    a.cu_k = cu_k;
     a.cu_blocks = at<int32_t>(ws, pr.ws.cu_blocks);
-    a.blk_req = at<int32_t>(ws, pr.ws.blk_req);
+    a.cu_qblocks = at<int32_t>(ws, pr.ws.cu_qblocks);
+    a.blk_req_q = at<int32_t>(ws, pr.ws.blk_req_q);
     a.order = at<int32_t>(ws, pr.ws.order);
     a.block_table = block_table;
     a.max_blocks_per_seq = mbps;
@@ -378,7 +403,7 @@ fp2_status run_attention(const fp2_params* p, const void* q, const void* k, cons
     a.out = out;
     a.lse = lse;
     a.hdr = hdr;
-    return launched(launch_attention(e4m3, a, tq, tk, tv, tkb, tvb, pr.max_blocks, s));
+    return launched(launch_attention(e4m3, a, tq, tk, tv, tkb, tvb, pr.max_qblocks, s));
 }
 
 }  // namespace
@@ -403,61 +428,71 @@ fp2_status fp2_workspace_init(void* workspace, size_t ws_bytes, void* stream) {
     return launched(cudaMemsetAsync(workspace, 0, sizeof(WsHeader), static_cast<cudaStream_t>(stream)));
 }
 
-fp2_status fp2_estimate(const fp2_params* params, const void* q, const void* k, const void* v,
-                        const int32_t* cu_seqlens, int32_t batch, int64_t total_tokens,
-                        int32_t max_seqlen, const int32_t* block_table, int32_t max_blocks_per_seq,
-                        int32_t num_pages, fp2_blockmeta* meta, void* workspace, size_t ws_bytes,
-                        void* stream) {
+fp2_status fp2_estimate_chunked(const fp2_params* params, const void* q, const void* k, const void* v,
+                                const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int32_t batch,
+                                int64_t total_q, int64_t total_k, int32_t max_seqlen_k,
+                                const int32_t* block_table, int32_t max_blocks_per_seq, int32_t num_pages,
+                                fp2_blockmeta* meta, void* workspace, size_t ws_bytes, void* stream) {
     Problem pr;
-    fp2_status st = check_problem(params, q, k, v, cu_seqlens, batch, total_tokens, max_seqlen,
-                                  workspace, ws_bytes, &pr);
+    fp2_status st = check_problem(params, q, k, v, cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k,
+                                  max_seqlen_k, workspace, ws_bytes, &pr);
     if (st != FP2_OK) return st;
     if ((st = check_meta(meta, params, pr, false)) != FP2_OK) return st;
     if (block_table && (max_blocks_per_seq < 1 || num_pages < 1)) return FP2_ERR_INVALID_ARG;
     // page rows are int32 inside the kernels (TMA coordinates)
     if (block_table && int64_t(num_pages) * kBlock > (int64_t(1) << 31) - 1) return FP2_ERR_UNSUPPORTED;
-    return run_estimate(params, q, k, v, cu_seqlens, pr, block_table, max_blocks_per_seq, num_pages,
-                        meta, workspace, static_cast<cudaStream_t>(stream));
+    return run_estimate(params, q, k, v, cu_seqlens_q, cu_seqlens_k, pr, block_table, max_blocks_per_seq,
+                        num_pages, meta, workspace, static_cast<cudaStream_t>(stream));
+}
+
+fp2_status fp2_estimate(const fp2_params* params, const void* q, const void* k, const void* v,
+                        const int32_t* cu_seqlens, int32_t batch, int64_t total_tokens,
+                        int32_t max_seqlen, const int32_t* block_table, int32_t max_blocks_per_seq,
+                        int32_t num_pages, fp2_blockmeta* meta, void* workspace, size_t ws_bytes,
+                        void* stream) {
+    return fp2_estimate_chunked(params, q, k, v, cu_seqlens, cu_seqlens, batch, total_tokens, total_tokens,
+                                max_seqlen, block_table, max_blocks_per_seq, num_pages, meta, workspace,
+                                ws_bytes, stream);
+}
+
+fp2_status fp2_prefill_chunked(const fp2_params* params, const void* q, const void* k, const void* v,
+                               const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int32_t batch,
+                               int64_t total_q, int64_t total_k, int32_t max_seqlen_k,
+                               const int32_t* block_table, int32_t max_blocks_per_seq, int32_t num_pages,
+                               const fp2_blockmeta* meta, void* out, float* lse, void* workspace,
+                               size_t ws_bytes, void* stream) {
+    Problem pr;
+    fp2_status st = check_problem(params, q, k, v, cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k,
+                                  max_seqlen_k, workspace, ws_bytes, &pr);
+    if (st != FP2_OK) return st;
+    if ((st = check_meta(meta, params, pr, true)) != FP2_OK) return st;
+    if (block_table && (max_blocks_per_seq < 1 || num_pages < 1)) return FP2_ERR_INVALID_ARG;
+    // page rows are int32 inside the kernels (TMA coordinates)
+    if (block_table && int64_t(num_pages) * kBlock > (int64_t(1) << 31) - 1) return FP2_ERR_UNSUPPORTED;
+    if (total_q > 0 && (!out || !aligned(out, 16))) return FP2_ERR_INVALID_ARG;
+    if (lse && !aligned(lse, 4)) return FP2_ERR_INVALID_ARG;
+    return run_attention(params, q, k, v, cu_seqlens_q, cu_seqlens_k, pr, block_table, max_blocks_per_seq,
+                         num_pages, meta, out, lse, workspace, static_cast<cudaStream_t>(stream));
 }
 
 fp2_status fp2_sparse_prefill(const fp2_params* params, const void* q, const void* k, const void* v,
                               const int32_t* cu_seqlens, int32_t batch, int64_t total_tokens,
                               int32_t max_seqlen, const fp2_blockmeta* meta, void* out, float* lse,
                               void* workspace, size_t ws_bytes, void* stream) {
-    Problem pr;
-    fp2_status st = check_problem(params, q, k, v, cu_seqlens, batch, total_tokens, max_seqlen,
-                                  workspace, ws_bytes, &pr);
-    if (st != FP2_OK) return st;
-    if ((st = check_meta(meta, params, pr, true)) != FP2_OK) return st;
-    if (total_tokens > 0 && (!out || !aligned(out, 16))) return FP2_ERR_INVALID_ARG;
-    if (lse && !aligned(lse, 4)) return FP2_ERR_INVALID_ARG;
-    return run_attention(params, q, k, v, cu_seqlens, pr, nullptr, 0, 0, meta, out, lse, workspace,
-                         static_cast<cudaStream_t>(stream), true);
+    return fp2_prefill_chunked(params, q, k, v, cu_seqlens, cu_seqlens, batch, total_tokens, total_tokens,
+                               max_seqlen, nullptr, 0, 0, meta, out, lse, workspace, ws_bytes, stream);
 }
 
 fp2_status fp2_prefill_paged(const fp2_params* params, const void* q, const void* k_pool,
                              const void* v_pool, const int32_t* cu_seqlens, int32_t batch,
                              int64_t total_tokens, int32_t max_seqlen, const int32_t* block_table,
-                             int32_t max_blocks_per_seq, int32_t num_pages, fp2_blockmeta* meta,
+                             int32_t max_blocks_per_seq, int32_t num_pages, const fp2_blockmeta* meta,
                              void* out, float* lse, void* workspace, size_t ws_bytes, void* stream) {
-    Problem pr;
-    fp2_status st = check_problem(params, q, k_pool, v_pool, cu_seqlens, batch, total_tokens,
-                                  max_seqlen, workspace, ws_bytes, &pr);
-    if (st != FP2_OK) return st;
-    if ((st = check_meta(meta, params, pr, true)) != FP2_OK) return st;
-    if (batch > 0 && (!block_table || max_blocks_per_seq < 1 || num_pages < 1)) return FP2_ERR_INVALID_ARG;
-    // page rows are int32 inside the kernels (TMA coordinates)
-    if (int64_t(num_pages) * kBlock > (int64_t(1) << 31) - 1) return FP2_ERR_UNSUPPORTED;
-    if (total_tokens > 0 && (!out || !aligned(out, 16))) return FP2_ERR_INVALID_ARG;
-    if (lse && !aligned(lse, 4)) return FP2_ERR_INVALID_ARG;
-    // the attention's limits too, before the estimator is enqueued
-    if ((st = check_limits(params, pr, true, true)) != FP2_OK) return st;
-    const cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if ((st = run_estimate(params, q, k_pool, v_pool, cu_seqlens, pr, block_table, max_blocks_per_seq,
-                           num_pages, meta, workspace, s)) != FP2_OK)
-        return st;
-    return run_attention(params, q, k_pool, v_pool, cu_seqlens, pr, block_table, max_blocks_per_seq,
-                         num_pages, meta, out, lse, workspace, s, false);
+    if (batch > 0 && !block_table) return FP2_ERR_INVALID_ARG;
+    if (batch > 0 && (max_blocks_per_seq < 1 || num_pages < 1)) return FP2_ERR_INVALID_ARG;
+    return fp2_prefill_chunked(params, q, k_pool, v_pool, cu_seqlens, cu_seqlens, batch, total_tokens,
+                               total_tokens, max_seqlen, block_table, max_blocks_per_seq, num_pages, meta,
+                               out, lse, workspace, ws_bytes, stream);
 }
 
 fp2_status fp2_get_error(void* workspace, void* stream) {
@@ -488,7 +523,7 @@ const char* fp2_status_string(fp2_status status) {
     return "unknown status";
 }
 
-int32_t fp2_version(void) { return 100; }
+int32_t fp2_version(void) { return 200; }
 
 }  // extern "C"
 
@@ -520,29 +555,6 @@ fp2_status noalloc_scratch(void** addr) {
     return FP2_OK;
 }
 
-// The attention call reads none of the estimator's split means, so its
-// scratch is the workspace layout without those regions.
-WsLayout noalloc_layout(const Problem& pr, const fp2_params* p) {
-    WsLayout w;
-    size_t off = 256;
-    w.cu_blocks = off;
-    off = align256(off + sizeof(int32_t) * (pr.batch + 1));
-    w.cu_tiles = off;
-    off = align256(off + sizeof(int32_t) * (pr.batch + 1));
-    w.blk_req = off;
-    off = align256(off + sizeof(int32_t) * pr.max_blocks);
-    w.order = off;
-    off = align256(off + sizeof(int32_t) * pr.max_blocks);
-    w.qsplit = off;
-    w.ksplit = off;
-    w.kbar_lp = off;
-    off = align256(off + size_t(esize(p)) * pr.max_blocks * p->num_kv_heads * kHeadDim);
-    w.vbar_lp = off;
-    off = align256(off + size_t(esize(p)) * pr.max_blocks * p->num_kv_heads * kHeadDim);
-    w.total = off;
-    return w;
-}
-
 }  // namespace
 
 extern "C" fp2_status fp2_sparse_prefill_noalloc(const fp2_params* params, const void* q,
@@ -564,21 +576,27 @@ extern "C" fp2_status fp2_sparse_prefill_noalloc(const fp2_params* params, const
     if (device_status && !aligned(device_status, 4)) return FP2_ERR_INVALID_ARG;
     Problem pr;
     pr.batch = batch;
-    pr.total_tokens = total_tokens;
+    pr.total_q = total_tokens;
+    pr.total_k = total_tokens;
     pr.max_seqlen = max_seqlen;
     pr.max_blocks = fp2_max_blocks(batch, total_tokens, kBlock);
+    pr.max_qblocks = pr.max_blocks;
     pr.nb_need = (max_seqlen + kBlock - 1) / kBlock;
-    pr.ws = noalloc_layout(pr, params);
+    // the attention call reads none of the estimator's split means
+    pr.ws = ws_layout(batch, pr.max_blocks, params->num_q_heads, params->num_kv_heads, esize(params),
+                      false);
     if (pr.ws.total > FP2_NOALLOC_SCRATCH_BYTES) return FP2_ERR_WORKSPACE;  // over the static maximum
     if ((st = check_meta(meta, params, pr, true)) != FP2_OK) return st;
+    // every host-side rejection before anything is enqueued
+    if ((st = check_limits(params, pr, false, true)) != FP2_OK) return st;
     void* scratch = nullptr;
     if ((st = noalloc_scratch(&scratch)) != FP2_OK) return st;
     const cudaStream_t s = static_cast<cudaStream_t>(stream);
     // the error flag is the only scratch state that must start at zero; every
     // other region is rewritten by the kernels of this call
     if (cudaMemsetAsync(scratch, 0, sizeof(WsHeader), s) != cudaSuccess) return FP2_ERR_CUDA;
-    st = run_attention(params, q, k, v, cu_seqlens, pr, nullptr, 0, 0, meta, out, lse, scratch, s,
-                       true);
+    st = run_attention(params, q, k, v, cu_seqlens, cu_seqlens, pr, nullptr, 0, 0, meta, out, lse, scratch,
+                       s);
     if (st != FP2_OK) return st;
     if (device_status &&
         cudaMemcpyAsync(device_status, scratch, sizeof(int32_t), cudaMemcpyDeviceToDevice, s) !=

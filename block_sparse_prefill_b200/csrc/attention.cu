@@ -56,16 +56,6 @@ constexpr int kThreads = 384;
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr int kSchedWarp = 10;
-// When > 0, every kEmuEvery-th pair of attention weights is exponentiated on
-// the FMA pipe (exp2_poly2) instead of MUFU (per dtype).  Measured on B200 at
-// 128K (bf16, attention call): off 4.77 ms, 1/8 4.77 ms, 1/4 5.08 ms, 1/2
-// 5.90 ms -- the bf16 softmax is bound by instruction issue, not by MUFU.
-#ifndef FP2_EXP_EMU_BF16
-#define FP2_EXP_EMU_BF16 0
-#endif
-#ifndef FP2_EXP_EMU_E4M3
-#define FP2_EXP_EMU_E4M3 0
-#endif
 constexpr uint32_t kTmemCols = 512;
 // Registers per thread after the split.  setmaxnreg only redistributes the
 // registers the CTA was launched with (384 threads x 168 = 64512), so
@@ -93,7 +83,6 @@ struct Cfg {
     // bf16: no offset, and O is rescaled only for jumps above 2^8.
     static constexpr float kPOffset = kE4M3 ? 8.f : 0.f;
     static constexpr float kRescale = kE4M3 ? 0.75f : 8.f;
-    static constexpr int kEmuEvery = kE4M3 ? FP2_EXP_EMU_E4M3 : FP2_EXP_EMU_BF16;
 };
 
 struct Bars {
@@ -132,8 +121,13 @@ struct SmemMisc {
 // and the correction tile list follow the header.
 struct ItemMeta {
     int32_t stop;     // 1: no work left
-    int32_t t, b, i, g, h0, ntiles, nrows, qrow0, cb, cnt, ncorr, nwords;
-    int32_t pad[3];
+    int32_t t, b, i, g, h0, ntiles;
+    int32_t nkeys;    // keys of the diagonal block (< 128: the V rows past them are zeroed)
+    int32_t r_lo, r_hi;  // rows [r_lo, r_hi) of the Q tile are query rows (stored)
+    int32_t qrow0;    // row of q / out of the tile's row 0 (rows outside [r_lo, r_hi)
+                      // belong to another request, or lie before row 0: never stored)
+    int32_t cb, cnt, ncorr, nwords;
+    int32_t pad[1];
 };
 
 template <bool kE4M3>
@@ -278,8 +272,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       regs_dec<kOtherRegs>();
       if (warp == kSchedWarp) {
         // ---- scheduler: next work item -> metadata buffer ----------------
-        const int32_t per_blk = a.hkv * a.pairs;
-        const int32_t n_items = hdr->total_blocks * per_blk;
+        const int32_t n_items = hdr->total_qblocks * a.hkv * a.pairs;
         for (int32_t k = 0;; ++k) {
             const int32_t buf = k & 1;
             if (!warp_wait(&bars.meta_empty[buf], ((k >> 1) & 1) ^ 1, hdr, abort, 500000 + k)) break;
@@ -294,14 +287,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 break;
             }
-            const int32_t t = a.order[item / per_blk];
-            const int32_t rem = item % per_blk;
-            const int32_t g = rem / a.pairs;
-            const int32_t hp = rem % a.pairs;
-            const int32_t b = a.blk_req[t];
+            const int32_t code = a.order[item / a.pairs];   // t * hkv + g, heaviest first
+            const int32_t t = code / a.hkv;
+            const int32_t g = code % a.hkv;
+            const int32_t hp = item % a.pairs;
+            const int32_t b = a.blk_req_q[t];
             const int32_t cb = a.cu_blocks[b];
-            const int32_t i = t - cb;
-            const int32_t L = a.cu[b + 1] - a.cu[b];
+            const ReqSpan span = req_span(a.cu_q, a.cu_k, b);
+            const int32_t i = span.i0 + t - a.cu_qblocks[b];   // absolute block index
             int32_t* klist = klist_of(m);
             uint32_t* pruned = pruned_of(m);
             int32_t* ctiles = ctiles_of(m);
@@ -363,7 +356,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     row = page * kBlock;
                 } else {
-                    row = a.cu[b] + j * kBlock;
+                    row = a.cu_k[b] + j * kBlock;
                 }
                 klist[e] = row;
             }
@@ -376,8 +369,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 m->g = g;
                 m->h0 = g * a.G + 2 * hp;
                 m->ntiles = min(2, a.G - 2 * hp);
-                m->nrows = min(kBlock, L - i * kBlock);
-                m->qrow0 = a.cu[b] + i * kBlock;
+                m->nkeys = min(kBlock, span.lk - i * kBlock);
+                m->r_lo = max(0, span.p - i * kBlock);
+                m->r_hi = m->nkeys;
+                m->qrow0 = a.cu_q[b] + i * kBlock - span.p;
                 m->cb = cb;
                 m->cnt = cnt;
                 m->ncorr = nc;
@@ -406,7 +401,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             ItemMeta* m = meta(buf);
             if (m->stop) break;
             const int32_t ntiles = m->ntiles, cnt = m->cnt, ntot = m->cnt + m->ncorr;
-            const int32_t nrows = m->nrows, g = m->g, cb = m->cb;
+            const int32_t nrows = m->nkeys, g = m->g, cb = m->cb;
             const int32_t* klist = klist_of(m);
             const int32_t* ctiles = ctiles_of(m);
             const int32_t item_base = issued;
@@ -513,7 +508,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ItemMeta* m = meta(buf);
                 if (m->stop) break;
                 const int32_t ntiles = m->ntiles, ntot = m->cnt + m->ncorr;
-                const bool partial = m->nrows < kBlock;
+                const bool partial = m->nkeys < kBlock;
                 if (a.test_wait_timeout && k == 0 &&
                     !(ok = mbar_wait(&bars.never, 0, hdr, abort, 900000)))
                     break;
@@ -592,9 +587,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             const int32_t cnt = m->cnt, ntot = m->cnt + m->ncorr, nwords = m->nwords;
             float qk = a.scale_log2;
-            if (kE4M3) qk *= a.q_scale[m->h0 + qt] * a.k_scale[m->g];
-            // correction tiles: +log2(128) after scaling == +7/qk before it
-            const float corr_bias = 7.f / qk;
+            // e4m3: a zero scale (an all-zero head) makes every logit 0; the floor keeps
+            // masked (-inf) scores at -inf instead of -inf * 0 = NaN
+            if (kE4M3) qk = fmaxf(qk * a.q_scale[m->h0 + qt] * a.k_scale[m->g], 1.17549435e-38f);
             float m_ref = -INFINITY;
             float l = 0.f;      // row sum of the weights the PV MMA uses (O normaliser)
             float l_lse = 0.f;  // row sum before P is rounded to the MMA precision (LSE)
@@ -621,12 +616,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const uint32_t bits = (w0 + wi < nwords) ? pruned[w0 + wi] : 0u;
 #pragma unroll
                         for (int c = 0; c < 32; ++c)
-                            sv[wi * 32 + c] =
-                                ((bits >> c) & 1u)
-                                    ? __float_as_uint(__uint_as_float(sv[wi * 32 + c]) + corr_bias)
-                                    : __float_as_uint(-INFINITY);
+                            if (!((bits >> c) & 1u)) sv[wi * 32 + c] = __float_as_uint(-INFINITY);
                     }
                 }
+                // a correction column stands for the 128 keys of a pruned block: its
+                // weight is 128 e^{lbar}, i.e. +log2(128) on the scaled logit
+                const float bias = (n >= cnt) ? 7.f : 0.f;
                 // row max over 4 independent 3-input max chains
                 float mxp[4];
 #pragma unroll
@@ -636,7 +631,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mxp[(c >> 1) & 3] =
                         fmax3(mxp[(c >> 1) & 3], __uint_as_float(sv[c]), __uint_as_float(sv[c + 1]));
                 const float mx = fmax3(mxp[0], mxp[1], fmaxf(mxp[2], mxp[3]));
-                const float m_new = fmaxf(m_ref, mx * qk);
+                const float m_new = fmaxf(m_ref, fmaf(mx, qk, bias));
                 const bool need = m_new > m_ref + C::kRescale;
                 if (__any_sync(0xffffffffu, need)) {
                     const float f = need ? ex2(m_ref - m_new) : 1.f;
@@ -661,10 +656,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
                 // P = exp2(s * qk - m + offset) in the MMA precision, written over S
-                const float neg = C::kPOffset - ((m_ref == -INFINITY) ? 0.f : m_ref);
-                // exp2 of packed pairs (MUFU; optionally some pairs on the FMA pipe), in
-                // two halves of 64 keys: the first half's P goes to TMEM (asynchronously)
-                // while the second half is computed
+                const float neg = C::kPOffset + bias - ((m_ref == -INFINITY) ? 0.f : m_ref);
+                // exp2 of packed pairs (MUFU), in two halves of 64 keys: the first
+                // half's P goes to TMEM (asynchronously) while the second half is computed
                 float2 rsp[4];
 #pragma unroll
                 for (int j = 0; j < 4; ++j) rsp[j] = make_float2(0.f, 0.f);
@@ -677,13 +671,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int c = 64 * hf; c < 64 * hf + 64; c += 2) {
                         float2 x = ffma2(make_float2(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])),
                                          make_float2(qk, qk), make_float2(neg, neg));
-                        if (C::kEmuEvery > 0 &&
-                            ((c >> 1) % (C::kEmuEvery > 0 ? C::kEmuEvery : 1)) == C::kEmuEvery - 1) {
-                            x = exp2_poly2(x);
-                        } else {
-                            x.x = ex2(x.x);
-                            x.y = ex2(x.y);
-                        }
+                        x.x = ex2(x.x);
+                        x.y = ex2(x.y);
                         sv[c] = __float_as_uint(x.x);
                         sv[c + 1] = __float_as_uint(x.y);
                         rsp[(c >> 1) & 3] = fadd2(rsp[(c >> 1) & 3], x);
@@ -723,7 +712,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             // ---- epilogue: O / l -> bf16 ------------------------------------
             if (ok && ntot > 0 && (ok = warp_wait(&bars.o_done[qt], (items++) & 1, hdr, abort, 420000))) {
-                const int32_t g = m->g, h = m->h0 + qt, nrows = m->nrows, qrow0 = m->qrow0;
+                const int32_t g = m->g, h = m->h0 + qt, r_lo = m->r_lo, r_hi = m->r_hi, qrow0 = m->qrow0;
+                const bool store = r >= r_lo && r < r_hi;
                 tc_fence_after();
                 float inv = 1.f / l;
                 if (kE4M3) inv *= a.v_scale[g];
@@ -734,7 +724,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     uint32_t ov[32];
                     tmem_ld32(o_addr + c0, ov);
                     tmem_wait_ld();
-                    if (r < nrows) {
+                    if (store) {
                         uint32_t pk[16];
 #pragma unroll
                         for (int c = 0; c < 16; ++c)
@@ -746,7 +736,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             dst[c] = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
                     }
                 }
-                if (a.lse && r < nrows) {
+                if (a.lse && store) {
                     const float m_use = ((m_ref == -INFINITY) ? 0.f : m_ref) - C::kPOffset;
                     a.lse[static_cast<int64_t>(qrow0 + r) * a.hq + h] =
                         (m_use + __log2f(l_lse)) * 0.69314718055994530942f;

@@ -25,55 +25,85 @@ namespace fp2 {
 // ---------------------------------------------------------------------------
 // set-up
 // ---------------------------------------------------------------------------
+// Cost of the attention work item (q-block t = block i of its request, KV
+// head g) in tile steps: its kept tiles, its correction tiles (128 pruned-block
+// means each, when the correction is on) and 2 steps of pipeline fill.  The kept
+// count is clamped to [1, i + 1]; the attention kernel checks the list itself.
+__device__ __forceinline__ int32_t item_cost(const SetupArgs& a, int32_t t, int32_t i, int32_t g) {
+    const int32_t c = min(max(a.kept_cnt[static_cast<int64_t>(t) * a.hkv + g], 1), i + 1);
+    const int32_t pruned = i + 1 - c;
+    const int32_t corr = (a.correction && pruned > 0) ? min((i + 127) / 128, pruned) : 0;
+    return c + corr + 2;
+}
+
 __global__ void setup_kernel(SetupArgs a) {
-    extern __shared__ int32_t hist[];  // [nb_cap + 1]
+    extern __shared__ int32_t hist[];  // [setup_bins(nb_cap, cost) + 1]
     __shared__ int32_t ok;
+    const bool cost = a.kept_cnt != nullptr;
+    const int32_t nbins = setup_bins(a.nb_cap, cost);
     if (threadIdx.x == 0) {
         int32_t good = 1, bad = -1;
-        int32_t nb_acc = 0, nt_acc = 0;
-        if (a.cu[0] != 0) { good = 0; bad = 0; }
+        int32_t nb_acc = 0, nq_acc = 0, nt_acc = 0;
+        if (a.cu_q[0] != 0 || a.cu_k[0] != 0) { good = 0; bad = 0; }
         a.cu_blocks[0] = 0;
+        a.cu_qblocks[0] = 0;
         a.cu_tiles[0] = 0;
         for (int32_t b = 0; good && b < a.batch; ++b) {
-            const int32_t L = a.cu[b + 1] - a.cu[b];
-            if (L < 0 || L > a.max_seqlen) { good = 0; bad = b + 1; break; }
-            const int32_t nb = (L + kBlock - 1) / kBlock;
+            const int32_t lk = a.cu_k[b + 1] - a.cu_k[b];
+            const int32_t lq = a.cu_q[b + 1] - a.cu_q[b];
+            if (lq < 0 || lk < lq || lk > a.max_seqlen) { good = 0; bad = b + 1; break; }
+            const int32_t nb = (lk + kBlock - 1) / kBlock;
             if (a.paged && nb > a.max_blocks_per_seq) { good = 0; bad = b + 1; break; }
+            const int32_t nq = nb - req_span(a.cu_q, a.cu_k, b).i0;
             nb_acc += nb;
-            nt_acc += (nb + a.qt - 1) / a.qt;
+            nq_acc += nq;
+            nt_acc += (nq + a.qt - 1) / a.qt;
             a.cu_blocks[b + 1] = nb_acc;
+            a.cu_qblocks[b + 1] = nq_acc;
             a.cu_tiles[b + 1] = nt_acc;
         }
-        if (good && a.cu[a.batch] != a.total_tokens) { good = 0; bad = a.batch; }
+        if (good && (a.cu_q[a.batch] != a.total_q || a.cu_k[a.batch] != a.total_k)) { good = 0; bad = a.batch; }
         if (good && nb_acc > a.max_blocks) { good = 0; bad = a.batch; }
         a.hdr->valid = good;
         a.hdr->total_blocks = good ? nb_acc : 0;
+        a.hdr->total_qblocks = good ? nq_acc : 0;
         a.hdr->work_next = 0;
         if (!good) set_error(a.hdr, FP2_ERR_BAD_INDEX, bad);
         ok = good;
     }
-    for (int32_t e = threadIdx.x; e <= a.nb_cap; e += blockDim.x) hist[e] = 0;
+    for (int32_t e = threadIdx.x; e <= nbins; e += blockDim.x) hist[e] = 0;
     __syncthreads();
     if (!ok) return;
-    for (int32_t b = 0; b < a.batch; ++b)
-        for (int32_t t = a.cu_blocks[b] + threadIdx.x; t < a.cu_blocks[b + 1]; t += blockDim.x) {
+    // request of every key block and q-block; histogram of the sort key: the
+    // q-block's absolute index in its request, or the cost of each (q-block,
+    // KV head) work item
+    for (int32_t b = 0; b < a.batch; ++b) {
+        for (int32_t t = a.cu_blocks[b] + threadIdx.x; t < a.cu_blocks[b + 1]; t += blockDim.x)
             a.blk_req[t] = b;
-            atomicAdd(&hist[t - a.cu_blocks[b]], 1);
+        const int32_t i0 = req_span(a.cu_q, a.cu_k, b).i0, cq = a.cu_qblocks[b];
+        for (int32_t t = cq + threadIdx.x; t < a.cu_qblocks[b + 1]; t += blockDim.x) {
+            a.blk_req_q[t] = b;
+            const int32_t i = i0 + t - cq;
+            if (!cost)
+                atomicAdd(&hist[i], 1);
+            else
+                for (int32_t g = 0; g < a.hkv; ++g) atomicAdd(&hist[item_cost(a, t, i, g)], 1);
         }
+    }
     __syncthreads();
-    // order: blocks sorted by their index in the request, largest first (the
-    // causal kept lists grow with it), so the persistent attention kernel
-    // takes the longest work items first.  Exclusive scan of the histogram in
-    // descending index order: each thread scans a contiguous run of bins, the
-    // runs' totals are scanned across the block.
+    // order: largest key first (the causal kept lists grow with the block index,
+    // so either key puts the longest work items first for the persistent
+    // attention kernel).  Exclusive scan of the histogram in descending key
+    // order: each thread scans a contiguous run of bins, the runs' totals are
+    // scanned across the block.
     {
         __shared__ int32_t wsum[32];
         const int32_t tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
         const int32_t nwarps = (blockDim.x + 31) >> 5;
-        const int32_t per = (a.nb_cap + blockDim.x - 1) / blockDim.x;
-        const int32_t p0 = min(a.nb_cap, tid * per), p1 = min(a.nb_cap, p0 + per);
+        const int32_t per = (nbins + blockDim.x - 1) / blockDim.x;
+        const int32_t p0 = min(nbins, tid * per), p1 = min(nbins, p0 + per);
         int32_t local = 0;
-        for (int32_t p = p0; p < p1; ++p) local += hist[a.nb_cap - 1 - p];
+        for (int32_t p = p0; p < p1; ++p) local += hist[nbins - 1 - p];
         int32_t incl = local;
         for (int32_t o = 1; o < 32; o <<= 1) {
             const int32_t y = __shfl_up_sync(0xffffffffu, incl, o);
@@ -93,16 +123,24 @@ __global__ void setup_kernel(SetupArgs a) {
         __syncthreads();
         int32_t run = wsum[warp] + incl - local;
         for (int32_t p = p0; p < p1; ++p) {
-            const int32_t j = a.nb_cap - 1 - p;
+            const int32_t j = nbins - 1 - p;
             const int32_t c = hist[j];
             hist[j] = run;
             run += c;
         }
     }
     __syncthreads();
-    for (int32_t b = 0; b < a.batch; ++b)
-        for (int32_t t = a.cu_blocks[b] + threadIdx.x; t < a.cu_blocks[b + 1]; t += blockDim.x)
-            a.order[atomicAdd(&hist[t - a.cu_blocks[b]], 1)] = t;
+    for (int32_t b = 0; b < a.batch; ++b) {
+        const int32_t i0 = req_span(a.cu_q, a.cu_k, b).i0, cq = a.cu_qblocks[b];
+        for (int32_t t = cq + threadIdx.x; t < a.cu_qblocks[b + 1]; t += blockDim.x) {
+            const int32_t i = i0 + t - cq;
+            if (!cost)
+                a.order[atomicAdd(&hist[i], 1)] = t;
+            else
+                for (int32_t g = 0; g < a.hkv; ++g)
+                    a.order[atomicAdd(&hist[item_cost(a, t, i, g)], 1)] = t * a.hkv + g;
+        }
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -131,22 +169,44 @@ struct PoolSmem {
 };
 
 struct PoolUnit {
-    int32_t x, y, t, b, j, n;
+    int32_t x, y, t, b;  // tensor, column slab, block (q-block for x = 0, else key block), request
+    int64_t row0;        // first row of the block in the tensor (before paging)
+    int32_t j;           // key block index in the request (x > 0)
+    int32_t n;           // rows of the block
 };
 
-// unit u -> (tensor, slab, block, request, block index in the request, valid rows)
-__device__ __forceinline__ PoolUnit pool_unit(const PoolArgs& a, int32_t u, int32_t ys) {
+// Units: the q-blocks' column slabs of Q first (ysq per q-block), then the key
+// blocks' slabs of K and V (yskv per key block).  A q-block holds the query rows
+// at positions [max(P, bs i), min(Lk, bs i + bs)); a key block the keys
+// [bs j, min(Lk, bs j + bs)).
+__device__ __forceinline__ PoolUnit pool_unit(const PoolArgs& a, int32_t u, int32_t nq, int32_t ysq,
+                                              int32_t yskv) {
     PoolUnit p;
-    p.t = u / ys;
-    p.y = u % ys;
-    p.x = a.first;
+    if (u < nq * ysq) {
+        p.x = 0;
+        p.t = u / ysq;
+        p.y = u % ysq;
+        p.b = a.blk_req_q[p.t];
+        const ReqSpan r = req_span(a.cu_q, a.cu_k, p.b);
+        const int32_t i = r.i0 + p.t - a.cu_qblocks[p.b];
+        const int32_t lo = max(r.p, i * kBlock);
+        p.j = i;
+        p.row0 = a.cu_q[p.b] + static_cast<int64_t>(lo - r.p);
+        p.n = min(r.lk, i * kBlock + kBlock) - lo;
+        return p;
+    }
+    u -= nq * ysq;
+    p.t = u / yskv;
+    p.y = u % yskv;
+    p.x = max(a.first, 1);
     while (p.x < a.last - 1 && p.y >= a.slabs[p.x]) {
         p.y -= a.slabs[p.x];
         ++p.x;
     }
     p.b = a.blk_req[p.t];
     p.j = p.t - a.cu_blocks[p.b];
-    p.n = min(kBlock, a.cu[p.b + 1] - a.cu[p.b] - p.j * kBlock);
+    p.row0 = a.cu_k[p.b] + static_cast<int64_t>(p.j) * kBlock;
+    p.n = min(kBlock, a.cu_k[p.b + 1] - a.cu_k[p.b] - p.j * kBlock);
     return p;
 }
 
@@ -213,9 +273,11 @@ __global__ void __launch_bounds__(kPoolThreads, 1)
     volatile int32_t* abort = &ps->abort;
     WsHeader* hdr = a.hdr;
     if (!hdr->valid) return;
-    int32_t ys = 0;
-    for (int x = a.first; x < a.last; ++x) ys += a.slabs[x];
-    const int32_t units = hdr->total_blocks * ys;
+    const int32_t ysq = a.first == 0 ? a.slabs[0] : 0;
+    int32_t yskv = 0;
+    for (int x = max(a.first, 1); x < a.last; ++x) yskv += a.slabs[x];
+    const int32_t nq = hdr->total_qblocks;
+    const int32_t units = nq * ysq + hdr->total_blocks * yskv;
     const int32_t tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid == 0) {
         for (int st = 0; st < kPoolStages; ++st) {
@@ -234,8 +296,8 @@ __global__ void __launch_bounds__(kPoolThreads, 1)
             int32_t cnt = 0;
             bool ok = true;
             for (int32_t u = blockIdx.x; ok && u < units; u += gridDim.x) {
-                const PoolUnit p = pool_unit(a, u, ys);
-                int64_t row0;
+                const PoolUnit p = pool_unit(a, u, nq, ysq, yskv);
+                int64_t row0 = p.row0;
                 if (a.paged[p.x]) {
                     int32_t page = a.block_table[static_cast<int64_t>(p.b) * a.max_blocks_per_seq + p.j];
                     if (page < 0 || page >= a.num_pages) {
@@ -243,8 +305,6 @@ __global__ void __launch_bounds__(kPoolThreads, 1)
                         page = 0;
                     }
                     row0 = static_cast<int64_t>(page) * kBlock;
-                } else {
-                    row0 = a.cu[p.b] + static_cast<int64_t>(p.j) * kBlock;
                 }
                 const uint32_t bytes = static_cast<uint32_t>(a.hb[p.x]) * kHeadDim * kEsz * kPoolStageRows;
                 const int32_t nsub = (p.n + kPoolStageRows - 1) / kPoolStageRows;
@@ -270,7 +330,7 @@ __global__ void __launch_bounds__(kPoolThreads, 1)
         int32_t cnt = 0;
         bool ok = true;
         for (int32_t u = blockIdx.x; u < units; u += gridDim.x) {
-            const PoolUnit p = pool_unit(a, u, ys);
+            const PoolUnit p = pool_unit(a, u, nq, ysq, yskv);
             const int32_t x = p.x;
             const int32_t row_bytes = a.hb[x] * kHeadDim * kEsz;   // one row of the slab
             const int32_t ncols = a.heads[x] * kHeadDim;
@@ -414,10 +474,12 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
     const int32_t b = lo;
     const int32_t g = blockIdx.x;
     const int32_t G = a.G;
-    const int32_t cb = a.cu_blocks[b];
-    const int32_t nb = a.cu_blocks[b + 1] - cb;
-    const int32_t i0 = (tile - a.cu_tiles[b]) * a.qt;
-    const int32_t nq = min(a.qt, nb - i0);
+    const int32_t cb = a.cu_blocks[b];                  // first key block of the request
+    const int32_t cq = a.cu_qblocks[b];                 // first q-block of the request
+    const int32_t nbq = a.cu_qblocks[b + 1] - cq;
+    const int32_t l0 = (tile - a.cu_tiles[b]) * a.qt;   // the tile's first q-block (in the request)
+    const int32_t nq = min(a.qt, nbq - l0);
+    const int32_t i0 = req_span(a.cu_q, a.cu_k, b).i0 + l0;  // its absolute block index
     const int32_t nrows = nq * G;
     const int32_t nchunk = (i0 + nq - 1) / 128 + 1;
     const int32_t steps = 2 * nchunk;
@@ -444,7 +506,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
 
     if (warp == 4) {
         if (lane == 0) {
-            const int32_t qrow = (g * static_cast<int32_t>(a.max_blocks) + cb + i0) * G;
+            const int32_t qrow = (g * static_cast<int32_t>(a.max_blocks) + cq + l0) * G;
             const int32_t krow = g * static_cast<int32_t>(a.max_blocks) + cb;
             mbar_arrive_expect_tx(&ss->q_full, 2 * kTileQ);
             for (int ch = 0; ch < 2; ++ch) {
@@ -514,7 +576,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         int32_t cnt = 0;  // kept blocks of this q-block (group leader lane / owner thread)
         const bool leader = lanes_group ? (valid && hh == 0) : (r < nq);
         const int32_t lead_i = lanes_group ? i : i0 + r;
-        const int64_t own_row = static_cast<int64_t>(cb + (lead_i - i0) + i0) * a.hkv + g;
+        const int64_t own_row = static_cast<int64_t>(cq + l0 + (lead_i - i0)) * a.hkv + g;
         bool ok = true;
         for (int32_t idx = 0; idx < steps; ++idx) {
             const int32_t s = idx & 1;
@@ -573,7 +635,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
                     if (i >= j0 && i < j0 + 128) bits[(i - j0) >> 5] |= 1u << ((i - j0) & 31);  // diagonal
                 }
                 if (a.score_dbg) {
-                    float* dbg = a.score_dbg + (static_cast<int64_t>(cb + i) * a.hq + h) * a.nb_max;
+                    float* dbg = a.score_dbg + (static_cast<int64_t>(cq + l0 + ii) * a.hq + h) * a.nb_max;
 #pragma unroll
                     for (int e = 0; e < 128; ++e)
                         if (j0 + e <= i) dbg[j0 + e] = __uint_as_float(v[e]) * a.tau - m;

@@ -12,21 +12,36 @@ constexpr int kPoolThreads = 544;  // 16 consumer warps (4 row groups x 128 colu
 constexpr int kScoreThreads = 160; // score_kernel: 4 epilogue warps + 1 TMA/MMA warp
 
 struct SetupArgs {
-    const int32_t* cu;
+    const int32_t* cu_q;     // [batch + 1] query rows
+    const int32_t* cu_k;     // [batch + 1] keys (= cu_q for plain prefill)
     int32_t batch;
-    int64_t total_tokens;
-    int32_t max_seqlen;
+    int64_t total_q;
+    int64_t total_k;
+    int32_t max_seqlen;      // >= every request's keys
     int32_t qt;  // q-blocks per estimator tile
     int32_t paged;
     int32_t max_blocks_per_seq;
     int64_t max_blocks;
     int32_t nb_cap;  // >= blocks of the longest request (histogram bins)
+    // attention call: order the (q-block, KV head) work items by their cost
+    // (kept tiles + correction tiles), heaviest first; NULL: blocks by index
+    const int32_t* kept_cnt;   // [max_blocks, hkv]
+    int32_t hkv;
+    int32_t correction;
     WsHeader* hdr;
-    int32_t* cu_blocks;
-    int32_t* cu_tiles;
-    int32_t* blk_req;
-    int32_t* order;
+    int32_t* cu_blocks;   // key blocks
+    int32_t* cu_qblocks;  // q-blocks
+    int32_t* cu_tiles;    // estimator tiles of q-blocks
+    int32_t* blk_req;     // request of every key block
+    int32_t* blk_req_q;   // request of every q-block
+    int32_t* order;  // kept_cnt == NULL: global q-blocks; else codes t * hkv + g (t a q-block)
 };
+
+// Histogram bins of the setup kernel: block index (< nb_cap) or item cost
+// (kept tiles <= nb_cap, correction tiles <= ceil(nb_cap / 128), fill 2).
+__host__ __device__ inline int32_t setup_bins(int32_t nb_cap, bool cost) {
+    return cost ? nb_cap + (nb_cap + 127) / 128 + 3 : nb_cap;
+}
 
 struct PoolArgs {
     float* out[3];           // fp32 means (NULL = not written): -, k_mean, v_mean
@@ -37,9 +52,12 @@ struct PoolArgs {
     int32_t slabs[3];        // column slabs per block of each tensor
     int32_t paged[3];
     int32_t first, last;     // tensors [first, last) of q, k, v are pooled
-    const int32_t* cu;
+    const int32_t* cu_q;
+    const int32_t* cu_k;
     const int32_t* cu_blocks;
+    const int32_t* cu_qblocks;
     const int32_t* blk_req;
+    const int32_t* blk_req_q;
     const int32_t* block_table;
     int32_t max_blocks_per_seq;
     int32_t num_pages;
@@ -49,7 +67,10 @@ struct PoolArgs {
 };
 
 struct ScoreArgs {
+    const int32_t* cu_q;
+    const int32_t* cu_k;
     const int32_t* cu_blocks;
+    const int32_t* cu_qblocks;
     const int32_t* cu_tiles;
     int32_t batch;
     int32_t hq, hkv, G;
@@ -78,10 +99,12 @@ struct MeanLpArgs {
 };
 
 struct AttnArgs {
-    const int32_t* cu;
-    const int32_t* cu_blocks;
-    const int32_t* blk_req;
-    const int32_t* order;        // global blocks, heaviest (largest block index) first
+    const int32_t* cu_q;
+    const int32_t* cu_k;
+    const int32_t* cu_blocks;    // key blocks (rows of the correction operands)
+    const int32_t* cu_qblocks;
+    const int32_t* blk_req_q;
+    const int32_t* order;        // work items t * hkv + g (q-block, KV head), heaviest first
     const int32_t* block_table;  // NULL = contiguous K/V
     int32_t max_blocks_per_seq;
     int32_t num_pages;

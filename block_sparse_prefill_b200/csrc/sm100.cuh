@@ -307,27 +307,6 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
     return r;
 }
 
-// 2^x for a pair of inputs on the FMA pipe instead of MUFU: x = n + f with
-// n = round(x) (the 1.5 * 2^23 rounding constant) and f in [-1/2, 1/2];
-// 2^f by a degree-3 polynomial with minimax relative error 7.5e-5 on that
-// interval (Remez exchange; coefficients from exp2_poly.py); 2^n added to the
-// exponent field.  Inputs are clamped at -126 so that the exponent cannot wrap
-// (the result there is ~1e-38, i.e. zero for the attention weights).
-__device__ __forceinline__ float2 exp2_poly2(float2 x) {
-    constexpr float kRound = 12582912.f;  // 1.5 * 2^23
-    x.x = fmaxf(x.x, -126.f);
-    x.y = fmaxf(x.y, -126.f);
-    const float2 t = fadd2(x, make_float2(kRound, kRound));
-    const float2 n = fadd2(t, make_float2(-kRound, -kRound));
-    const float2 f = ffma2(n, make_float2(-1.f, -1.f), x);
-    float2 p = ffma2(make_float2(5.517166853e-02f, 5.517166853e-02f), f,
-                     make_float2(2.426111251e-01f, 2.426111251e-01f));
-    p = ffma2(p, f, make_float2(6.932609677e-01f, 6.932609677e-01f));
-    p = ffma2(p, f, make_float2(9.999280572e-01f, 9.999280572e-01f));
-    return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
-                       __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
-}
-
 // Sum of the four e4m3 values packed in `w` (exact decode to f16x2, f16x2 adds).
 __device__ __forceinline__ __half2 e4m3x4_sum2(uint32_t w) {
     uint32_t lo, hi;

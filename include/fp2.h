@@ -96,7 +96,8 @@ typedef struct fp2_params {
     float sm_scale;            /* softmax scale tau; 0 selects 1/sqrt(head_dim) */
     int32_t correction;        /* 0: drop pruned blocks; 1: mean correction */
     int32_t dtype;             /* fp2_dtype */
-    const float* q_scale;      /* e4m3 only: device [Hq] dequantisation scales */
+    const float* q_scale;      /* e4m3 only: device [Hq] dequantisation scales, finite and
+                                  >= 0 (an all-zero head may have scale 0) */
     const float* k_scale;      /* e4m3 only: device [Hkv] */
     const float* v_scale;      /* e4m3 only: device [Hkv] */
 } fp2_params;
@@ -129,29 +130,52 @@ size_t fp2_workspace_bytes(const fp2_params* params, int32_t batch, int64_t tota
  * on a new workspace before its first use. */
 fp2_status fp2_workspace_init(void* workspace, size_t ws_bytes, void* stream);
 
-/* Estimator (block means, block scores, row max, alpha threshold, GQA union,
- * compaction).  Writes meta->kept_cnt, kept_idx, k_mean, v_mean (v_mean only
- * when non-NULL) and score_dbg (when non-NULL).
+/* fp2_estimate -- the block-score estimator and the max-relative threshold.
+ * Defined by: lode.cx, "How It Works" (a small sample of attention scores,
+ * its maximum, and the blocks above a threshold relative to that maximum);
+ * aipulsen.com (scores estimated at the block level); aimodeling.com, "From
+ * Prototype to Production" (max-based dynamic thresholding).  The sample is
+ * read here as the block-mean score (exact mean of the block pair's token
+ * logits), the threshold as exp(s - m) >= alpha (see the readings above).
+ * Computes block means, block scores, per-head row maximum, alpha threshold,
+ * GQA union, forced diagonal and the ascending kept lists.  Writes
+ * meta->kept_cnt, kept_idx, k_mean, v_mean (v_mean only when non-NULL) and
+ * score_dbg (when non-NULL).
  *   q            [total_tokens, Hq, d]
  *   k, v         contiguous [total_tokens, Hkv, d] when block_table == NULL,
  *                else page pools [num_pages * block_size, Hkv, d]
  *   block_table  NULL (contiguous) or [batch, max_blocks_per_seq] page indices
  *   num_pages    pages in the pools (paged mode; ignored otherwise); num_pages *
- *                block_size < 2^31, else FP2_ERR_UNSUPPORTED */
+ *                block_size < 2^31, else FP2_ERR_UNSUPPORTED
+ * Errors: bad arguments or sizes are returned before anything is enqueued; a
+ * bad cu_seqlens or a page index outside the pool is flagged on the device. */
 fp2_status fp2_estimate(const fp2_params* params, const void* q, const void* k, const void* v,
                         const int32_t* cu_seqlens, int32_t batch, int64_t total_tokens,
                         int32_t max_seqlen, const int32_t* block_table,
                         int32_t max_blocks_per_seq, int32_t num_pages, fp2_blockmeta* meta,
                         void* workspace, size_t ws_bytes, void* stream);
 
-/* Sparse attention over the kept blocks of `meta` (from fp2_estimate on the
- * same inputs) with contiguous K/V, plus the mean correction when
- * params->correction != 0.  Writes out (bf16) and, when non-NULL, lse.
+/* fp2_sparse_prefill -- sparse attention over the kept blocks with the mean
+ * correction, contiguous K/V.
+ * Defined by: lode.cx, "How It Works" (attend only what passes the threshold;
+ * a mean correction term compensates what pruning removes) and the operator
+ * list after it (PackGQA: the query heads of a KV head share its K/V tiles;
+ * FP8); aimodeling.com, "From Prototype to Production" (the mean correction
+ * suppresses the approximation error; FP8 inference); stuffinsider.com,
+ * "Technical Details" (query and key blocks; prefill, all queries in one pass).
+ * Attends over the kept blocks of `meta` (from fp2_estimate on the same
+ * inputs, or any caller-made lists that are ascending, in [0, i] and end with
+ * the diagonal block i), plus the mean correction when params->correction != 0
+ * (then meta->k_mean and v_mean must hold the block means).  Writes out (bf16)
+ * and, when non-NULL, lse.  `meta` is only read.
  * Length limit of the attention calls (this one, fp2_prefill_paged and
  * fp2_sparse_prefill_noalloc): a work item keeps its kept-block list in shared
  * memory, so ceil(max_seqlen / block_size) may be at most FP2_MAX_SEQ_BLOCKS_BF16
  * (4133 blocks, 529024 tokens) for bf16 and FP2_MAX_SEQ_BLOCKS_E4M3 (8075
- * blocks, 1033600 tokens) for e4m3; longer returns FP2_ERR_UNSUPPORTED. */
+ * blocks, 1033600 tokens) for e4m3; longer returns FP2_ERR_UNSUPPORTED.
+ * Errors: bad arguments or sizes are returned before anything is enqueued; a
+ * kept list that breaks the rules above is flagged on the device
+ * (FP2_ERR_BAD_INDEX) and replaced by the diagonal block alone. */
 #define FP2_MAX_SEQ_BLOCKS_BF16 4133
 #define FP2_MAX_SEQ_BLOCKS_E4M3 8075
 fp2_status fp2_sparse_prefill(const fp2_params* params, const void* q, const void* k,
@@ -160,15 +184,63 @@ fp2_status fp2_sparse_prefill(const fp2_params* params, const void* q, const voi
                               const fp2_blockmeta* meta, void* out, float* lse, void* workspace,
                               size_t ws_bytes, void* stream);
 
-/* One whole prefill attention layer on a paged KV cache: fp2_estimate on the
- * page pools (writing `meta`) followed by the sparse attention, whose K/V
- * tiles are fetched page by page through block_table. */
+/* fp2_prefill_paged -- fp2_sparse_prefill on a paged KV cache.
+ * Defined by: aimodeling.com, "From Prototype to Production" (native support
+ * of a paged KV cache and continuous batching, as an attention backend of a
+ * serving framework); lode.cx, after the operator list (paged KV cache and
+ * continuous batching).
+ * Same computation and arguments as fp2_sparse_prefill, with the K/V tiles of
+ * logical block j of request b read from page block_table[b][j] of the pools
+ * k_pool / v_pool [num_pages * block_size, Hkv, d].  `meta` comes from
+ * fp2_estimate on the same pools and block table (or from the caller) and is
+ * only read.  num_pages * block_size < 2^31, else FP2_ERR_UNSUPPORTED.  A page
+ * index outside [0, num_pages) is flagged on the device (FP2_ERR_BAD_INDEX) and
+ * page 0 is read in its place. */
 fp2_status fp2_prefill_paged(const fp2_params* params, const void* q, const void* k_pool,
                              const void* v_pool, const int32_t* cu_seqlens, int32_t batch,
                              int64_t total_tokens, int32_t max_seqlen, const int32_t* block_table,
-                             int32_t max_blocks_per_seq, int32_t num_pages, fp2_blockmeta* meta,
-                             void* out, float* lse, void* workspace, size_t ws_bytes,
-                             void* stream);
+                             int32_t max_blocks_per_seq, int32_t num_pages,
+                             const fp2_blockmeta* meta, void* out, float* lse, void* workspace,
+                             size_t ws_bytes, void* stream);
+
+/* fp2_estimate_chunked / fp2_prefill_chunked -- chunked prefill on a KV cache
+ * that already holds a prefix of each request.
+ * Defined by: aimodeling.com, "From Prototype to Production" (paged KV cache and
+ * continuous batching in a serving framework's attention backend); the
+ * write-ups do not treat chunks, so the plainest extension is taken.  Request
+ * b has Lk_b keys (cu_seqlens_k) and computes only its last Lq_b <= Lk_b query
+ * rows (cu_seqlens_q), at positions P_b = Lk_b - Lq_b .. Lk_b - 1: query row t
+ * of the chunk sees keys c <= P_b + t.  Key blocks are as in plain prefill.
+ * q-blocks keep the request's absolute grid of block_size positions, so the
+ * request has q-blocks i = floor(P_b / bs) .. ceil(Lk_b / bs) - 1 (none when
+ * Lq_b = 0), the first one holding the query rows from P_b on; qbar of a
+ * q-block is the mean of the query rows it holds.  With cu_seqlens_q ==
+ * cu_seqlens_k these are fp2_estimate and fp2_sparse_prefill / fp2_prefill_paged.
+ *   q            [total_q, Hq, d] (the chunk rows); out [total_q, Hq, d]; lse [total_q, Hq]
+ *   k, v         contiguous [total_k, Hkv, d] (all keys) when block_table == NULL,
+ *                else page pools as in fp2_prefill_paged
+ *   meta         kept_cnt / kept_idx rows: q-blocks, numbered globally in request
+ *                order (request b's q-blocks follow those of the requests before
+ *                it); their entries are key-block indices j <= i of the request.
+ *                k_mean / v_mean rows: key blocks (sum_b ceil(Lk_b / bs) of them),
+ *                so max_blocks >= fp2_max_blocks(batch, total_k, bs)
+ *   max_seqlen_k >= every Lk_b; the workspace from
+ *                fp2_workspace_bytes(params, batch, total_k, max_seqlen_k)
+ * Errors as for the plain calls; Lq_b > Lk_b is flagged on the device. */
+fp2_status fp2_estimate_chunked(const fp2_params* params, const void* q, const void* k, const void* v,
+                                const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                                int32_t batch, int64_t total_q, int64_t total_k,
+                                int32_t max_seqlen_k, const int32_t* block_table,
+                                int32_t max_blocks_per_seq, int32_t num_pages,
+                                fp2_blockmeta* meta, void* workspace, size_t ws_bytes,
+                                void* stream);
+fp2_status fp2_prefill_chunked(const fp2_params* params, const void* q, const void* k, const void* v,
+                               const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                               int32_t batch, int64_t total_q, int64_t total_k,
+                               int32_t max_seqlen_k, const int32_t* block_table,
+                               int32_t max_blocks_per_seq, int32_t num_pages,
+                               const fp2_blockmeta* meta, void* out, float* lse, void* workspace,
+                               size_t ws_bytes, void* stream);
 
 /* Synchronises `stream`, returns the first device-side error recorded in the
  * workspace since the last call (FP2_OK if none) and clears it. */

@@ -30,16 +30,22 @@ def test_bad_page_index_is_reported_and_cleared():
     wl = make_workload([700, 300], 8, 2, alpha=0.1, seed=5, paged=True)
     params, meta, ws, out = _setup(wl)
     cu = torch.from_numpy(wl.cu_seqlens).cuda()
+    good = torch.from_numpy(wl.block_table).cuda()
     bt = wl.block_table.copy()
     bt[1, 1] = wl.num_pages + 17                     # outside the pool
+    bad = torch.from_numpy(bt).cuda()
     q, kp, vp = wl.q.cuda(), wl.k_pool.cuda(), wl.v_pool.cuda()
-    fp2.prefill_paged(params, q, kp, vp, cu, wl.max_seqlen, torch.from_numpy(bt).cuda(), wl.num_pages,
-                      meta, out, ws)
+    # the estimator's pooling pass checks every page it reads
+    fp2.estimate(params, q, kp, vp, cu, wl.max_seqlen, meta, ws, block_table=bad, num_pages=wl.num_pages)
     assert fp2.get_error(ws) == BAD_INDEX
     assert fp2.get_error(ws) == 0, "fp2_get_error must clear the flag"
+    # the attention's scheduler checks the pages of the kept blocks (block 1 of request
+    # 1 is always kept: it is that q-block's diagonal)
+    fp2.estimate(params, q, kp, vp, cu, wl.max_seqlen, meta, ws, block_table=good, num_pages=wl.num_pages)
+    fp2.prefill_paged(params, q, kp, vp, cu, wl.max_seqlen, bad, wl.num_pages, meta, out, ws)
+    assert fp2.get_error(ws) == BAD_INDEX
     # the same workspace serves a valid call afterwards
-    fp2.prefill_paged(params, q, kp, vp, cu, wl.max_seqlen, torch.from_numpy(wl.block_table).cuda(),
-                      wl.num_pages, meta, out, ws)
+    fp2.prefill_paged(params, q, kp, vp, cu, wl.max_seqlen, good, wl.num_pages, meta, out, ws)
     assert fp2.get_error(ws) == 0
     assert torch.isfinite(out.float()).all()
 
