@@ -10,6 +10,7 @@
  * or constant with the CUDA library; the two meet only through the seeded
  * inputs.  All arithmetic is IEEE double (no fast-math), one plain loop per
  * definition below, no blocking or fusion beyond what the definition states.
+ * (-DORC_FP32 builds the same code in float: the timed CPU baseline only.)
  * OpenMP only splits independent (q-block, head) rows across host cores.
  *
  * Definitions (the pages give them in words only; where they are silent the
@@ -88,6 +89,19 @@
 #ifndef ORC_MUTANT
 #define ORC_MUTANT 0
 #endif
+
+/* The arithmetic type: IEEE double for the parity reference; the same code
+ * built with -DORC_FP32 runs in float (the timed CPU baseline only; parity is
+ * always checked against the double build). */
+#ifdef ORC_FP32
+typedef float real;
+#define EXP expf
+#define LOG logf
+#else
+typedef double real;
+#define EXP exp
+#define LOG log
+#endif
 #define MUT(n) (ORC_MUTANT == (n))
 
 /* D0: number of blocks of a request of length L. */
@@ -129,8 +143,8 @@ int64_t orc_total_blocks(const int32_t* cu, const int64_t* pos0, int B, int Bs) 
 /* D1: block means of a dequantised input x[T, H, d] (value * scale[h]).  Row
  * t of request b is at position pos0[b] + t (pos0 NULL: 0); the mean of a
  * block runs over its positions that hold rows.  out: [total_blocks, H, d]. */
-void orc_block_means(const float* x, const double* scale, const int32_t* cu, const int64_t* pos0,
-                     int B, int H, int d, int Bs, double* out) {
+void orc_block_means(const float* x, const real* scale, const int32_t* cu, const int64_t* pos0,
+                     int B, int H, int d, int Bs, real* out) {
     int64_t* cb = (int64_t*)malloc(sizeof(int64_t) * (B + 1));
     block_offsets(cu, pos0, B, Bs, cb);
     for (int b = 0; b < B; ++b) {
@@ -143,15 +157,15 @@ void orc_block_means(const float* x, const double* scale, const int32_t* cu, con
             int64_t i = i0 + t;
             int64_t lo = i * Bs > p0 ? i * Bs : p0;                       /* first position */
             int64_t hi = (i + 1) * Bs < p0 + L ? (i + 1) * Bs : p0 + L;   /* one past the last */
-            double denom = MUT(5) ? (double)Bs
-                         : MUT(13) ? (double)(hi - i * Bs)              /* mutant: counts P's rows */
-                         : (double)(hi - lo);
+            real denom = MUT(5) ? (real)Bs
+                         : MUT(13) ? (real)(hi - i * Bs)              /* mutant: counts P's rows */
+                         : (real)(hi - lo);
             for (int h = 0; h < H; ++h) {
                 for (int c = 0; c < d; ++c) {
-                    double s = 0.0;
+                    real s = 0.0;
                     for (int64_t p = lo; p < hi; ++p) {
                         int64_t row = cu[b] + (p - p0);
-                        s += (double)x[(row * H + h) * (int64_t)d + c] * scale[h];
+                        s += (real)x[(row * H + h) * (int64_t)d + c] * scale[h];
                     }
                     out[((cb[b] + t) * H + h) * (int64_t)d + c] = s / denom;
                 }
@@ -164,8 +178,8 @@ void orc_block_means(const float* x, const double* scale, const int32_t* cu, con
 /* Per-dimension variance of the dequantised rows inside every block, around the
  * block means `mean` (from orc_block_means with the same arguments):
  * out[t, h, c] = (1/n) sum_{r in t} (x[r, h, c] * scale[h] - mean[t, h, c])^2. */
-void orc_block_vars(const float* x, const double* scale, const int32_t* cu, const int64_t* pos0,
-                    int B, int H, int d, int Bs, const double* mean, double* out) {
+void orc_block_vars(const float* x, const real* scale, const int32_t* cu, const int64_t* pos0,
+                    int B, int H, int d, int Bs, const real* mean, real* out) {
     int64_t* cb = (int64_t*)malloc(sizeof(int64_t) * (B + 1));
     block_offsets(cu, pos0, B, Bs, cb);
     for (int b = 0; b < B; ++b) {
@@ -181,13 +195,13 @@ void orc_block_vars(const float* x, const double* scale, const int32_t* cu, cons
             for (int h = 0; h < H; ++h) {
                 for (int c = 0; c < d; ++c) {
                     int64_t at = ((cb[b] + t) * H + h) * (int64_t)d + c;
-                    double s = 0.0;
+                    real s = 0.0;
                     for (int64_t p = lo; p < hi; ++p) {
                         int64_t row = cu[b] + (p - p0);
-                        double e = (double)x[(row * H + h) * (int64_t)d + c] * scale[h] - mean[at];
+                        real e = (real)x[(row * H + h) * (int64_t)d + c] * scale[h] - mean[at];
                         s += e * e;
                     }
-                    out[at] = s / (double)(hi - lo);
+                    out[at] = s / (real)(hi - lo);
                 }
             }
         }
@@ -196,9 +210,9 @@ void orc_block_vars(const float* x, const double* scale, const int32_t* cu, cons
 }
 
 /* D1 score of one (head, q-block, k-block) pair. */
-static double block_score(const double* qbar, const double* kbar, int64_t qb, int64_t kb, int h,
-                          int g, int Hq, int Hkv, int d, double tau) {
-    double dot = 0.0;
+static real block_score(const real* qbar, const real* kbar, int64_t qb, int64_t kb, int h,
+                          int g, int Hq, int Hkv, int d, real tau) {
+    real dot = 0.0;
     for (int c = 0; c < d; ++c)
         dot += qbar[(qb * Hq + h) * (int64_t)d + c] * kbar[(kb * Hkv + g) * (int64_t)d + c];
     return MUT(7) ? dot : tau * dot;
@@ -214,11 +228,11 @@ static double block_score(const double* qbar, const double* kbar, int64_t qb, in
  *   m_out    [total q-blocks, Hq] row maxima (NULL to skip).
  * Returns 0, -1 when a request has more than nb_max key blocks, -3 when one
  * has more queries than keys. */
-int orc_estimate(const double* qbar, const double* kbar, const int32_t* cu_q, const int32_t* cu_k,
-                 int B, int Hq, int Hkv, int d, int Bs, double tau, double alpha, int nb_max,
-                 int32_t* kept_cnt, int32_t* kept_idx, double* s_out, double* m_out) {
+int orc_estimate(const real* qbar, const real* kbar, const int32_t* cu_q, const int32_t* cu_k,
+                 int B, int Hq, int Hkv, int d, int Bs, real tau, real alpha, int nb_max,
+                 int32_t* kept_cnt, int32_t* kept_idx, real* s_out, real* m_out) {
     int G = Hq / Hkv;
-    double ln_alpha = alpha > 0 ? log(alpha) : -INFINITY;
+    real ln_alpha = alpha > 0 ? LOG(alpha) : -INFINITY;
     int64_t* P = chunk_starts(cu_q, cu_k, B);
     if (!P) return -3;
     for (int b = 0; b < B; ++b)
@@ -234,14 +248,14 @@ int orc_estimate(const double* qbar, const double* kbar, const int32_t* cu_q, co
         for (int64_t t = 0; t < nbq; ++t) {
             int64_t i = i0 + t;                       /* block index in the request */
             int64_t qb = cbq[b] + t;                  /* global q-block id */
-            double* s = (double*)malloc(sizeof(double) * (i + 1));
+            real* s = (real*)malloc(sizeof(real) * (i + 1));
             unsigned char* keep = (unsigned char*)malloc(i + 1);
             for (int g = 0; g < Hkv; ++g) {
                 memset(keep, 0, i + 1);
                 for (int hh = 0; hh < G; ++hh) {
                     int h = g * G + hh;
                     int gk = MUT(3) ? h % Hkv : g;  /* mutant: wrong head -> group map */
-                    double m = -INFINITY;
+                    real m = -INFINITY;
                     for (int64_t j = 0; j <= i; ++j) {
                         s[j] = block_score(qbar, kbar, qb, cbk[b] + j, h, gk, Hq, Hkv, d, tau);
                         if (s[j] > m) m = s[j];
@@ -299,12 +313,12 @@ static int list_ok(const int32_t* idx, int32_t cnt, int64_t i) {
  * Returns 0, -1 on an invalid kept list, -2 on a bad q-block id, -3 when a
  * request has more queries than keys, -4 on a bad correction mode or a missing
  * array it needs. */
-int orc_attend(const float* q, const float* k, const float* v, const double* qs, const double* ks,
-               const double* vs, const int32_t* cu_q, const int32_t* cu_k, int B, int Hq, int Hkv,
-               int d, int Bs, double tau, const int32_t* kept_cnt, const int32_t* kept_idx,
-               int nb_max, int correction, const double* kbar, const double* vbar,
-               const double* kvar, const double* qbar, const int64_t* sel, int64_t nsel,
-               double* o, double* lse, double* wsum) {
+int orc_attend(const float* q, const float* k, const float* v, const real* qs, const real* ks,
+               const real* vs, const int32_t* cu_q, const int32_t* cu_k, int B, int Hq, int Hkv,
+               int d, int Bs, real tau, const int32_t* kept_cnt, const int32_t* kept_idx,
+               int nb_max, int correction, const real* kbar, const real* vbar,
+               const real* kvar, const real* qbar, const int64_t* sel, int64_t nsel,
+               real* o, real* lse, real* wsum) {
     int G = Hq / Hkv;
     int64_t* P = chunk_starts(cu_q, cu_k, B);
     if (!P) return -3;
@@ -349,16 +363,16 @@ int orc_attend(const float* q, const float* k, const float* v, const double* qs,
             unsigned char* kept = (unsigned char*)calloc(i + 1, 1);
             for (int32_t t = 0; t < cnt; ++t) kept[idx[t]] = 1;
             int64_t nmax = (int64_t)cnt * Bs + i + 1;
-            double* lg = (double*)malloc(sizeof(double) * nmax);     /* logits */
-            const double** vrow = (const double**)malloc(sizeof(double*) * nmax);
-            double* vbuf = (double*)malloc(sizeof(double) * (size_t)cnt * Bs * d);
-            double* qd = (double*)malloc(sizeof(double) * d);
-            double* acc = (double*)malloc(sizeof(double) * d);
+            real* lg = (real*)malloc(sizeof(real) * nmax);     /* logits */
+            const real** vrow = (const real**)malloc(sizeof(real*) * nmax);
+            real* vbuf = (real*)malloc(sizeof(real) * (size_t)cnt * Bs * d);
+            real* qd = (real*)malloc(sizeof(real) * d);
+            real* acc = (real*)malloc(sizeof(real) * d);
             int64_t lo = i * Bs > p0 ? i * Bs : p0;                   /* positions of the block's rows */
             int64_t hi = (i + 1) * Bs < L ? (i + 1) * Bs : L;
             for (int64_t p = lo; p < hi; ++p) {
                 int64_t grow = cu_q[b] + (p - p0);
-                for (int c = 0; c < d; ++c) qd[c] = (double)q[(grow * Hq + h) * (int64_t)d + c] * qs[h];
+                for (int c = 0; c < d; ++c) qd[c] = (real)q[(grow * Hq + h) * (int64_t)d + c] * qs[h];
                 int64_t n = 0;
                 int64_t nv = 0;
                 for (int32_t t = 0; t < cnt; ++t) {
@@ -370,13 +384,13 @@ int orc_attend(const float* q, const float* k, const float* v, const double* qs,
                                     : (kp <= p);
                         if (kp >= L || !visible) continue;
                         int64_t krow = cu_k[b] + kp;
-                        double dot = 0.0;
+                        real dot = 0.0;
                         for (int c = 0; c < d; ++c)
-                            dot += qd[c] * ((double)k[(krow * Hkv + g) * (int64_t)d + c] * ks[g]);
+                            dot += qd[c] * ((real)k[(krow * Hkv + g) * (int64_t)d + c] * ks[g]);
                         lg[n] = tau * dot;
-                        double* vr = vbuf + nv * d;
-                        double vsc = MUT(10) ? 1.0 : vs[g];
-                        for (int c = 0; c < d; ++c) vr[c] = (double)v[(krow * Hkv + g) * (int64_t)d + c] * vsc;
+                        real* vr = vbuf + nv * d;
+                        real vsc = MUT(10) ? 1.0 : vs[g];
+                        for (int c = 0; c < d; ++c) vr[c] = (real)v[(krow * Hkv + g) * (int64_t)d + c] * vsc;
                         vrow[n] = vr;
                         ++n;
                         ++nv;
@@ -388,22 +402,22 @@ int orc_attend(const float* q, const float* k, const float* v, const double* qs,
                         if (kept[j]) continue;
                         int64_t kb = cbk[b] + j;
                         int64_t nj = (L - j * Bs) < Bs ? (L - j * Bs) : Bs;
-                        const double* kj = kbar + (kb * Hkv + g) * (int64_t)d;
-                        double dot = 0.0;
+                        const real* kj = kbar + (kb * Hkv + g) * (int64_t)d;
+                        real dot = 0.0;
                         if (correction == 3) {        /* block-pooled: qbar of q-block i */
-                            const double* qi = qbar + (qb * Hq + h) * (int64_t)d;
+                            const real* qi = qbar + (qb * Hq + h) * (int64_t)d;
                             for (int c = 0; c < d; ++c) dot += qi[c] * kj[c];
                         } else {
                             for (int c = 0; c < d; ++c) dot += qd[c] * kj[c];
                         }
-                        lg[n] = tau * dot + (MUT(1) ? 0.0 : log((double)nj));
+                        lg[n] = tau * dot + (MUT(1) ? 0.0 : LOG((real)nj));
                         if (correction == 2 || correction == 4) {   /* second-order (variance) term */
-                            const double* vj = kvar + (kb * Hkv + g) * (int64_t)d;
-                            double q2v = 0.0;
+                            const real* vj = kvar + (kb * Hkv + g) * (int64_t)d;
+                            real q2v = 0.0;
                             if (correction == 2) {
                                 for (int c = 0; c < d; ++c) q2v += qd[c] * qd[c] * vj[c];
                             } else {                  /* |q|^2 times the mean variance */
-                                double q2 = 0.0, vm = 0.0;
+                                real q2 = 0.0, vm = 0.0;
                                 for (int c = 0; c < d; ++c) { q2 += qd[c] * qd[c]; vm += vj[c]; }
                                 q2v = q2 * (MUT(16) ? vm : vm / d);
                             }
@@ -413,20 +427,20 @@ int orc_attend(const float* q, const float* k, const float* v, const double* qs,
                         ++n;
                     }
                 }
-                double m = -INFINITY;
+                real m = -INFINITY;
                 for (int64_t t = 0; t < n; ++t) if (lg[t] > m) m = lg[t];
-                double den = 0.0;
+                real den = 0.0;
                 for (int c = 0; c < d; ++c) acc[c] = 0.0;
                 for (int64_t t = 0; t < n; ++t) {
-                    double e = exp(lg[t] - m);
+                    real e = EXP(lg[t] - m);
                     den += e;
                     for (int c = 0; c < d; ++c) acc[c] += e * vrow[t][c];
                 }
                 for (int c = 0; c < d; ++c) o[(grow * Hq + h) * (int64_t)d + c] = acc[c] / den;
-                lse[grow * Hq + h] = MUT(11) ? log(den) : m + log(den);
+                lse[grow * Hq + h] = MUT(11) ? LOG(den) : m + LOG(den);
                 if (wsum) {
-                    double ws = 0.0;
-                    for (int64_t t = 0; t < n; ++t) ws += exp(lg[t] - m) / den;
+                    real ws = 0.0;
+                    for (int64_t t = 0; t < n; ++t) ws += EXP(lg[t] - m) / den;
                     wsum[grow * Hq + h] = ws;
                 }
             }

@@ -25,18 +25,21 @@ _lock = threading.Lock()
 _cache = {}
 
 
-def lib_path(mutant: int = 0) -> str:
+def lib_path(mutant: int = 0, fp32: bool = False) -> str:
+    if fp32:
+        return os.path.join(_BUILD, "liboracle_fp32.so")
     return os.path.join(_BUILD, "liboracle.so" if mutant == 0 else f"liboracle_mut{mutant}.so")
 
 
-def build(mutant: int = 0, force: bool = False) -> str:
-    """Compile the oracle with gcc (IEEE double, OpenMP). Returns the .so path."""
-    out = lib_path(mutant)
+def build(mutant: int = 0, force: bool = False, fp32: bool = False) -> str:
+    """Compile the oracle with gcc (IEEE double, OpenMP; ``fp32``: the same code in
+    float, the timed CPU baseline's build). Returns the .so path."""
+    out = lib_path(mutant, fp32)
     os.makedirs(_BUILD, exist_ok=True)
     if force or not os.path.exists(out) or os.path.getmtime(out) < os.path.getmtime(_SRC):
         tmp = out + f".tmp{os.getpid()}"
         cmd = ["gcc", "-O2", "-fno-fast-math", "-ffp-contract=off", "-fopenmp", "-fPIC", "-shared",
-               f"-DORC_MUTANT={mutant}", _SRC, "-o", tmp, "-lm"]
+               f"-DORC_MUTANT={mutant}", *(["-DORC_FP32"] if fp32 else []), _SRC, "-o", tmp, "-lm"]
         subprocess.run(cmd, check=True)
         os.replace(tmp, out)
     return out
@@ -44,15 +47,16 @@ def build(mutant: int = 0, force: bool = False) -> str:
 
 _P = ctypes.c_void_p
 _I = ctypes.c_int
-_D = ctypes.c_double
 _L = ctypes.c_int64
 
 
-def _load(mutant: int = 0):
+def _load(mutant: int = 0, fp32: bool = False):
+    key = (mutant, fp32)
+    _D = ctypes.c_float if fp32 else ctypes.c_double   # the oracle's `real` scalars
     with _lock:
-        if mutant in _cache:
-            return _cache[mutant]
-        lib = ctypes.CDLL(build(mutant))
+        if key in _cache:
+            return _cache[key]
+        lib = ctypes.CDLL(build(mutant, fp32=fp32))
         lib.orc_total_blocks.argtypes = [_P, _P, _I, _I]
         lib.orc_total_blocks.restype = _L
         lib.orc_block_means.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _P]
@@ -65,7 +69,7 @@ def _load(mutant: int = 0):
                                    _I, _P, _P, _P, _P, _P, _L, _P, _P, _P]
         lib.orc_attend.restype = _I
         lib.orc_mutant_id.restype = _I
-        _cache[mutant] = lib
+        _cache[key] = lib
         return lib
 
 
@@ -75,10 +79,6 @@ def _ptr(a: Optional[np.ndarray]):
 
 def _f32(a):
     return np.ascontiguousarray(a, dtype=np.float32)
-
-
-def _f64(a):
-    return np.ascontiguousarray(a, dtype=np.float64)
 
 
 def _i32(a):
@@ -100,9 +100,15 @@ def chunk_starts(cu_seqlens_q, cu_seqlens_k) -> np.ndarray:
 class Oracle:
     """fp64 CPU reference of the estimator (D1, D2) and the attention (D3)."""
 
-    def __init__(self, mutant: int = 0):
-        self.lib = _load(mutant)
+    def __init__(self, mutant: int = 0, fp32: bool = False):
+        """``fp32``: the float build of the same code (the timed CPU baseline only;
+        every parity check uses the double build)."""
+        self.lib = _load(mutant, fp32)
         self.mutant = mutant
+        self.real = np.float32 if fp32 else np.float64
+
+    def _r(self, a):
+        return np.ascontiguousarray(a, dtype=self.real)
 
     # D0
     def total_blocks(self, cu_seqlens, block_size: int, pos0=None) -> int:
@@ -118,8 +124,8 @@ class Oracle:
         x = _f32(x)
         T, H, d = x.shape
         cu, p0 = _i32(cu_seqlens), _i64(pos0)
-        sc = _f64(np.ones(H) if scale is None else scale)
-        out = np.zeros((self.total_blocks(cu, block_size, p0), H, d), np.float64)
+        sc = self._r(np.ones(H) if scale is None else scale)
+        out = np.zeros((self.total_blocks(cu, block_size, p0), H, d), self.real)
         self.lib.orc_block_means(_ptr(x), _ptr(sc), _ptr(cu), _ptr(p0), len(cu) - 1, H, d, block_size,
                                  _ptr(out))
         return out
@@ -129,8 +135,8 @@ class Oracle:
         ``mean`` (``block_means`` of the same arguments); the D3 variance variant."""
         x = _f32(x)
         T, H, d = x.shape
-        cu, p0, mean = _i32(cu_seqlens), _i64(pos0), _f64(mean)
-        sc = _f64(np.ones(H) if scale is None else scale)
+        cu, p0, mean = _i32(cu_seqlens), _i64(pos0), self._r(mean)
+        sc = self._r(np.ones(H) if scale is None else scale)
         out = np.zeros_like(mean)
         self.lib.orc_block_vars(_ptr(x), _ptr(sc), _ptr(cu), _ptr(p0), len(cu) - 1, H, d, block_size,
                                 _ptr(mean), _ptr(out))
@@ -142,7 +148,7 @@ class Oracle:
         """Returns dict(kept_cnt [nb, Hkv], kept_idx [nb, Hkv, nb_max], s, m).
         ``cu_seqlens`` counts query rows, ``cu_seqlens_k`` keys (None: the same,
         plain prefill); nb counts q-blocks."""
-        qbar, kbar, cu = _f64(qbar), _f64(kbar), _i32(cu_seqlens)
+        qbar, kbar, cu = self._r(qbar), self._r(kbar), _i32(cu_seqlens)
         cuk = cu if cu_seqlens_k is None else _i32(cu_seqlens_k)
         nblk, Hq, d = qbar.shape
         Hkv = kbar.shape[1]
@@ -151,8 +157,8 @@ class Oracle:
             nb_max = max(1, int(max([(int(L) + block_size - 1) // block_size for L in lens] or [1])))
         cnt = np.zeros((nblk, Hkv), np.int32)
         idx = np.full((nblk, Hkv, nb_max), -1, np.int32)
-        s = np.full((nblk, Hq, nb_max), np.nan) if want_scores else None
-        m = np.full((nblk, Hq), np.nan) if want_scores else None
+        s = np.full((nblk, Hq, nb_max), np.nan, self.real) if want_scores else None
+        m = np.full((nblk, Hq), np.nan, self.real) if want_scores else None
         rc = self.lib.orc_estimate(_ptr(qbar), _ptr(kbar), _ptr(cu), _ptr(cuk), len(cu) - 1, Hq, Hkv, d,
                                    block_size, tau, alpha, nb_max, _ptr(cnt), _ptr(idx), _ptr(s), _ptr(m))
         if rc != 0:
@@ -176,17 +182,17 @@ class Oracle:
         Hkv = k.shape[1]
         kept_cnt, kept_idx = _i32(kept_cnt), _i32(kept_idx)
         nb_max = kept_idx.shape[2]
-        qs = _f64(np.ones(Hq) if q_scale is None else q_scale)
-        ks = _f64(np.ones(Hkv) if k_scale is None else k_scale)
-        vs = _f64(np.ones(Hkv) if v_scale is None else v_scale)
+        qs = self._r(np.ones(Hq) if q_scale is None else q_scale)
+        ks = self._r(np.ones(Hkv) if k_scale is None else k_scale)
+        vs = self._r(np.ones(Hkv) if v_scale is None else v_scale)
         mode = int(correction)
         if mode:
-            kbar, vbar = _f64(kbar), _f64(vbar)
-        kvar = None if mode not in (2, 4) else _f64(kvar)
-        qbar = None if mode != 3 else _f64(qbar)
-        o = np.full((T, Hq, d), np.nan)
-        lse = np.full((T, Hq), np.nan)
-        ws = np.full((T, Hq), np.nan) if want_wsum else None
+            kbar, vbar = self._r(kbar), self._r(vbar)
+        kvar = None if mode not in (2, 4) else self._r(kvar)
+        qbar = None if mode != 3 else self._r(qbar)
+        o = np.full((T, Hq, d), np.nan, self.real)
+        lse = np.full((T, Hq), np.nan, self.real)
+        ws = np.full((T, Hq), np.nan, self.real) if want_wsum else None
         selv = None if sel is None else np.ascontiguousarray(sel, dtype=np.int64)
         rc = self.lib.orc_attend(_ptr(q), _ptr(k), _ptr(v), _ptr(qs), _ptr(ks), _ptr(vs), _ptr(cu),
                                  _ptr(cuk), len(cu) - 1, Hq, Hkv, d, block_size, tau, _ptr(kept_cnt),
