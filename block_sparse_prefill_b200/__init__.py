@@ -130,13 +130,15 @@ def _check_args(params: "Params", where: str, q, k, v, cu_seqlens, out=None, lse
 
 @dataclasses.dataclass
 class Params:
-    """Mirror of ``fp2_params``.  Scales are device tensors (e4m3 only)."""
+    """Mirror of ``fp2_params``.  Scales are device tensors (e4m3 only).
+    ``correction``: False / 0 none, True / 1 the mean correction, 2 the mean
+    correction with the variance term (needs ``BlockMeta.k_var``)."""
 
     num_q_heads: int
     num_kv_heads: int
     alpha: float = 0.05
     sm_scale: float = 0.0
-    correction: bool = True
+    correction: int = True
     dtype: int = FP2_BF16
     q_scale: Optional[torch.Tensor] = None
     k_scale: Optional[torch.Tensor] = None
@@ -157,7 +159,7 @@ class Params:
 
     def c(self) -> _lib.fp2_params:
         return _lib.fp2_params(self.num_q_heads, self.num_kv_heads, self.head_dim, self.block_size,
-                               float(self.alpha), float(self.sm_scale), 1 if self.correction else 0,
+                               float(self.alpha), float(self.sm_scale), int(self.correction),
                                int(self.dtype), _ptr(self.q_scale), _ptr(self.k_scale),
                                _ptr(self.v_scale))
 
@@ -201,6 +203,7 @@ class BlockMeta:
     score_dbg: Optional[torch.Tensor]
     nb_max: int
     max_blocks: int
+    k_var: Optional[torch.Tensor] = None   # [max_blocks, Hkv] fp32 mean key variance per block
 
     @staticmethod
     def empty(params: Params, batch: int, total_tokens: int, max_seqlen: int, device="cuda",
@@ -215,11 +218,13 @@ class BlockMeta:
             v_mean=torch.zeros((mb, hkv, HEAD_DIM), dtype=torch.float32, device=device),
             score_dbg=(torch.full((mb, params.num_q_heads, nbm), float("nan"), dtype=torch.float32,
                                   device=device) if scores else None),
-            nb_max=nbm, max_blocks=mb)
+            nb_max=nbm, max_blocks=mb,
+            k_var=torch.zeros((mb, hkv), dtype=torch.float32, device=device))
 
     def c(self) -> _lib.fp2_blockmeta:
         return _lib.fp2_blockmeta(_ptr(self.kept_cnt), _ptr(self.kept_idx), _ptr(self.k_mean),
-                                  _ptr(self.v_mean), _ptr(self.score_dbg), self.nb_max, self.max_blocks)
+                                  _ptr(self.v_mean), _ptr(self.score_dbg), self.nb_max, self.max_blocks,
+                                  _ptr(self.k_var))
 
 
 def _bt_args(block_table: Optional[torch.Tensor], num_pages: int):

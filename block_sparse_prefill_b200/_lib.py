@@ -48,6 +48,7 @@ class fp2_blockmeta(ctypes.Structure):
         ("score_dbg", ctypes.c_void_p),
         ("nb_max", ctypes.c_int32),
         ("max_blocks", ctypes.c_int32),
+        ("k_var", ctypes.c_void_p),
     ]
 
 

@@ -95,7 +95,7 @@ fp2_status check_params(const fp2_params* p) {
     if (p->num_q_heads < 1 || p->num_kv_heads < 1 || p->num_q_heads % p->num_kv_heads != 0)
         return FP2_ERR_INVALID_ARG;
     if (p->dtype != FP2_BF16 && p->dtype != FP2_E4M3) return FP2_ERR_INVALID_ARG;
-    if (p->correction != 0 && p->correction != 1) return FP2_ERR_INVALID_ARG;
+    if (p->correction < 0 || p->correction > 2) return FP2_ERR_INVALID_ARG;
     if (std::isnan(p->alpha) || p->alpha > 1.f) return FP2_ERR_INVALID_ARG;
     if (!std::isfinite(p->sm_scale) || p->sm_scale < 0.f) return FP2_ERR_INVALID_ARG;
     if (p->head_dim <= 0 || p->block_size <= 0) return FP2_ERR_INVALID_ARG;
@@ -150,6 +150,7 @@ fp2_status check_problem(const fp2_params* p, const void* q, const void* k, cons
 fp2_status check_meta(const fp2_blockmeta* m, const fp2_params* p, const Problem& pr, bool need_v) {
     if (!m || !m->kept_cnt || !m->kept_idx || !m->k_mean) return FP2_ERR_INVALID_ARG;
     if (need_v && p->correction && !m->v_mean) return FP2_ERR_INVALID_ARG;
+    if (need_v && p->correction == 2 && !m->k_var) return FP2_ERR_INVALID_ARG;
     if (m->nb_max < pr.nb_need || m->nb_max < 1) return FP2_ERR_INVALID_ARG;
     if (m->max_blocks < 0) return FP2_ERR_INVALID_ARG;
     if (!aligned(m->k_mean, 16) || (m->v_mean && !aligned(m->v_mean, 16))) return FP2_ERR_INVALID_ARG;
@@ -182,7 +183,7 @@ fp2_status check_limits(const fp2_params* p, const Problem& pr, bool estimate, b
         if (!score_tiling(p->num_q_heads / p->num_kv_heads, &qt)) return FP2_ERR_UNSUPPORTED;
         if ((pr.max_qblocks + qt - 1) / qt + pr.batch > 65535) return FP2_ERR_UNSUPPORTED;
     }
-    if (attention && attn_smem_bytes(p->dtype == FP2_E4M3, pr.nb_need) > kMaxSmem)
+    if (attention && attn_smem_bytes(p->dtype == FP2_E4M3, pr.nb_need, p->correction == 2) > kMaxSmem)
         return FP2_ERR_UNSUPPORTED;
     return FP2_OK;
 }
@@ -244,6 +245,7 @@ fp2_status run_estimate(const fp2_params* p, const void* q, const void* k, const
     pa.out[0] = nullptr;
     pa.out[1] = meta->k_mean;
     pa.out[2] = meta->v_mean;
+    pa.kvar = meta->k_var;
     pa.split[0] = at<uint16_t>(ws, pr.ws.qsplit);
     pa.split[1] = at<uint16_t>(ws, pr.ws.ksplit);
     pa.G = G;
@@ -394,6 +396,8 @@ fp2_status run_attention(const fp2_params* p, const void* q, const void* k, cons
     a.G = p->num_q_heads / p->num_kv_heads;
     a.pairs = (a.G + 1) / 2;
     a.correction = p->correction;
+    a.k_var = meta->k_var;
+    a.var_coef = 0.5f * tau_of(p) * tau_of(p) * 1.4426950408889634f;
     // test hook (tests/test_gpu_errors.py): make one bounded wait run out
     a.test_wait_timeout = std::getenv("FP2_TEST_WAIT_TIMEOUT") != nullptr ? 1 : 0;
     a.scale_log2 = tau_of(p) * 1.4426950408889634f;

@@ -90,6 +90,8 @@ struct Bars {
     uint64_t q_empty;     // the last S MMAs of a work item have read Q (committed right
                           // after them, so the next item's Q loads during the item's
                           // last tile step)
+    uint64_t q_read;      // correction 2: the softmax warps have read |q_r|^2 off the Q
+                          // tile (one arrival per softmax warp and item)
     uint64_t s_full[2];
     uint64_t p_full[2];
     uint64_t o_done[2];   // the last PV of Q tile t in a work item has finished
@@ -135,11 +137,23 @@ __host__ __device__ constexpr size_t tiles_bytes() {
     return static_cast<size_t>(2 + Cfg<kE4M3>::kSlots) * Cfg<kE4M3>::kTileBytes;
 }
 
-// One metadata buffer: header, kept list, pruned bitmask, correction tile list.
-__host__ __device__ inline size_t meta_bytes(int32_t nb_cap) {
+// End of the operand tiles and SmemMisc, rounded up to 16 bytes: where the two
+// metadata buffers begin.
+template <bool kE4M3>
+__host__ __device__ constexpr size_t misc_end() {
+    return (tiles_bytes<kE4M3>() + sizeof(SmemMisc) + 15) & ~size_t(15);
+}
+
+// One metadata buffer: header, kept list, pruned bitmask, correction tile list
+// and (correction 2) the variance coefficient of every column of the correction
+// tiles (16-byte aligned, after the lists).
+__host__ __device__ inline size_t meta_lists_bytes(int32_t nb_cap) {
     const size_t b = sizeof(ItemMeta) +
                      sizeof(int32_t) * (nb_cap + (nb_cap + 31) / 32 + (nb_cap + 127) / 128 + 4);
     return (b + 15) & ~size_t(15);
+}
+__host__ __device__ inline size_t meta_bytes(int32_t nb_cap, bool var) {
+    return meta_lists_bytes(nb_cap) + (var ? sizeof(float) * 128 * ((nb_cap + 127) / 128) : 0);
 }
 
 // Byte offset of K-major operand step k inside a tile (Q or K).
@@ -208,7 +222,9 @@ __device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint3
 
 }  // namespace
 
-template <bool kE4M3>
+// kVar: correction 2 (the variance term), a separate instantiation so that the
+// other corrections keep their own register allocation.
+template <bool kE4M3, bool kVar>
 __global__ void __launch_bounds__(kThreads, 1)
     attention_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CUtensorMap tq,
                      const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
@@ -221,8 +237,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t* q_s = smem;                                  // 2 tiles
     uint8_t* kv_s = smem + 2 * C::kTileBytes;             // kSlots tiles
     SmemMisc* misc = reinterpret_cast<SmemMisc*>(smem + tiles_bytes<kE4M3>());
-    uint8_t* meta_base = reinterpret_cast<uint8_t*>(misc + 1);
-    const size_t meta_stride = meta_bytes(a.nb_cap);
+    // metadata buffers start 16-byte aligned (correction 2 reads them as float4)
+    uint8_t* meta_base = smem + misc_end<kE4M3>();
+    constexpr bool var = kVar;
+    const size_t meta_stride = meta_bytes(a.nb_cap, var);
     Bars& bars = misc->bars;
     volatile int32_t* abort = &misc->abort;
     WsHeader* hdr = a.hdr;
@@ -238,6 +256,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto ctiles_of = [&](ItemMeta* m) {
         return reinterpret_cast<int32_t*>(pruned_of(m) + (a.nb_cap + 31) / 32);
     };
+    auto cvals_of = [&](ItemMeta* m) {
+        return reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(m) + meta_lists_bytes(a.nb_cap));
+    };
 
     // ---- set-up ------------------------------------------------------------
     if (warp == kMmaWarp) {
@@ -247,6 +268,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (tid == 0) {
         mbar_init(&bars.q_full, 1);
         mbar_init(&bars.q_empty, 1);
+        mbar_init(&bars.q_read, 8);
         for (int s = 0; s < 2; ++s) {
             mbar_init(&bars.s_full[s], 1);
             mbar_init(&bars.p_full[s], 128);
@@ -343,6 +365,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                     nc += __popc(mask);
                 }
             }
+            if (var) {
+                // correction 2: tau^2 / 2 log2(e) kvar_j of every column of the
+                // correction tiles (0 where the column is masked)
+                float* cv = cvals_of(m);
+                for (int32_t e = 0; e < nc; ++e) {
+                    const int32_t j0 = ctiles[e] * 128;
+                    for (int32_t c = lane; c < 128; c += 32) {
+                        const int32_t j = j0 + c;
+                        const bool pr = j < i && ((pruned[j >> 5] >> (j & 31)) & 1u);
+                        cv[e * 128 + c] =
+                            pr ? a.var_coef * a.k_var[static_cast<int64_t>(cb + j) * a.hkv + g] : 0.f;
+                    }
+                }
+            }
             // kept blocks -> the first K/V row of each (a page of the pool, or the
             // request's rows), so the producer's per-tile work is one shared-memory read
             for (int32_t e = lane; e < cnt; e += 32) {
@@ -412,6 +448,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     // while the previous item's last MMAs still read the Q buffer
                     if (leader) {
                         if (k > 0) ok = mbar_wait(&bars.q_empty, (k - 1) & 1, hdr, abort, 520000 + k);
+                        if (ok && var && k > 0)
+                            ok = mbar_wait(&bars.q_read, (k - 1) & 1, hdr, abort, 525000 + k);
                         if (ok) {
                             ++nq;
                             mbar_arrive_expect_tx(&bars.q_full, ntiles * C::kTileBytes);
@@ -582,7 +620,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (m->stop) break;
             if (qt >= m->ntiles) {
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&bars.meta_empty[buf]);
+                if (lane == 0) {
+                    if (var) mbar_arrive(&bars.q_read);
+                    mbar_arrive(&bars.meta_empty[buf]);
+                }
                 continue;
             }
             const int32_t cnt = m->cnt, ntot = m->cnt + m->ncorr, nwords = m->nwords;
@@ -590,6 +631,38 @@ __global__ void __launch_bounds__(kThreads, 1)
             // e4m3: a zero scale (an all-zero head) makes every logit 0; the floor keeps
             // masked (-inf) scores at -inf instead of -inf * 0 = NaN
             if (kE4M3) qk = fmaxf(qk * a.q_scale[m->h0 + qt] * a.k_scale[m->g], 1.17549435e-38f);
+            // correction 2: w = |q_r|^2 (dequantised), read off the Q tile, whose 16-byte
+            // units of row r sit in the 128-byte swizzle order (the sum does not care)
+            float w = 0.f;
+            if (var) {
+                if (!(ok = warp_wait(&bars.q_full, k & 1, hdr, abort, 405000))) break;
+                const uint8_t* qrow = q_s + qt * C::kTileBytes + r * 128;
+#pragma unroll
+                for (int ch = 0; ch < C::kChunks; ++ch)
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        const uint4 x4 = *reinterpret_cast<const uint4*>(qrow + ch * 16384 + u * 16);
+                        const uint32_t wd[4] = {x4.x, x4.y, x4.z, x4.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            if (kE4M3) {
+                                const float2 lo = __half22float2(e4m3x2_to_half2(wd[e] & 0xFFFFu));
+                                const float2 hi = __half22float2(e4m3x2_to_half2(wd[e] >> 16));
+                                w = fmaf(lo.x, lo.x, fmaf(lo.y, lo.y, fmaf(hi.x, hi.x, fmaf(hi.y, hi.y, w))));
+                            } else {
+                                const float a0 = __uint_as_float(wd[e] << 16);
+                                const float a1 = __uint_as_float(wd[e] & 0xFFFF0000u);
+                                w = fmaf(a0, a0, fmaf(a1, a1, w));
+                            }
+                        }
+                    }
+                if (kE4M3) {
+                    const float qs = a.q_scale[m->h0 + qt];
+                    w *= qs * qs;
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars.q_read);
+            }
             float m_ref = -INFINITY;
             float l = 0.f;      // row sum of the weights the PV MMA uses (O normaliser)
             float l_lse = 0.f;  // row sum before P is rounded to the MMA precision (LSE)
@@ -622,6 +695,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // a correction column stands for the 128 keys of a pruned block: its
                 // weight is 128 e^{lbar}, i.e. +log2(128) on the scaled logit
                 const float bias = (n >= cnt) ? 7.f : 0.f;
+                // scale of the tile's values in the max and the exponent: qk, or 1 for
+                // correction 2's tiles, whose scaled logits get + w * coef_j here
+                float sc = qk;
+                if (var && n >= cnt) {
+                    const float4* cv = reinterpret_cast<const float4*>(cvals_of(m) + (n - cnt) * 128);
+#pragma unroll
+                    for (int c4 = 0; c4 < 32; ++c4) {
+                        const float4 cc = cv[c4];
+                        sv[4 * c4] = __float_as_uint(fmaf(w, cc.x, __uint_as_float(sv[4 * c4]) * qk));
+                        sv[4 * c4 + 1] = __float_as_uint(fmaf(w, cc.y, __uint_as_float(sv[4 * c4 + 1]) * qk));
+                        sv[4 * c4 + 2] = __float_as_uint(fmaf(w, cc.z, __uint_as_float(sv[4 * c4 + 2]) * qk));
+                        sv[4 * c4 + 3] = __float_as_uint(fmaf(w, cc.w, __uint_as_float(sv[4 * c4 + 3]) * qk));
+                    }
+                    sc = 1.f;
+                }
                 // row max over 4 independent 3-input max chains
                 float mxp[4];
 #pragma unroll
@@ -631,7 +719,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mxp[(c >> 1) & 3] =
                         fmax3(mxp[(c >> 1) & 3], __uint_as_float(sv[c]), __uint_as_float(sv[c + 1]));
                 const float mx = fmax3(mxp[0], mxp[1], fmaxf(mxp[2], mxp[3]));
-                const float m_new = fmaxf(m_ref, fmaf(mx, qk, bias));
+                const float m_new = fmaxf(m_ref, fmaf(mx, sc, bias));
                 const bool need = m_new > m_ref + C::kRescale;
                 if (__any_sync(0xffffffffu, need)) {
                     const float f = need ? ex2(m_ref - m_new) : 1.f;
@@ -670,7 +758,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int c = 64 * hf; c < 64 * hf + 64; c += 2) {
                         float2 x = ffma2(make_float2(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])),
-                                         make_float2(qk, qk), make_float2(neg, neg));
+                                         make_float2(sc, sc), make_float2(neg, neg));
                         x.x = ex2(x.x);
                         x.y = ex2(x.y);
                         sv[c] = __float_as_uint(x.x);
@@ -757,42 +845,47 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-size_t attn_smem_bytes(bool e4m3, int32_t nb_cap) {
+size_t attn_smem_bytes(bool e4m3, int32_t nb_cap, bool var) {
     const size_t tiles = e4m3 ? tiles_bytes<true>() : tiles_bytes<false>();
-    return 1024 + tiles + sizeof(SmemMisc) + 2 * meta_bytes(nb_cap);
+    return 1024 + (e4m3 ? misc_end<true>() : misc_end<false>()) + 2 * meta_bytes(nb_cap, var);
+}
+
+template <bool kE4M3, bool kVar>
+cudaError_t launch_one(const AttnArgs& a, const CUtensorMap& tq, const CUtensorMap& tk,
+                       const CUtensorMap& tv, const CUtensorMap& tkb, const CUtensorMap& tvb,
+                       unsigned grid, size_t smem, cudaStream_t stream) {
+    // the setmaxnreg split assumes the kernel was built with kLaunchRegs per
+    // thread; with fewer, the softmax warps' register request could never be met
+    cudaFuncAttributes fa;
+    cudaError_t err = cudaFuncGetAttributes(&fa, attention_kernel<kE4M3, kVar>);
+    if (err != cudaSuccess) return err;
+    if (fa.numRegs < kLaunchRegs) return cudaErrorInvalidConfiguration;
+    err = cudaFuncSetAttribute(attention_kernel<kE4M3, kVar>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               int(smem));
+    if (err != cudaSuccess) return err;
+    attention_kernel<kE4M3, kVar><<<grid, kThreads, smem, stream>>>(a, tq, tk, tv, tkb, tvb);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_attention(bool e4m3, const AttnArgs& a, const CUtensorMap& tq,
                              const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tkb,
                              const CUtensorMap& tvb, int64_t max_blocks, cudaStream_t stream) {
-    const size_t smem = attn_smem_bytes(e4m3, a.nb_cap);
+    const bool var = a.correction == 2;
+    const size_t smem = attn_smem_bytes(e4m3, a.nb_cap, var);
     const int64_t items = max_blocks * a.hkv * a.pairs;
     if (items <= 0) return cudaSuccess;
-    // the setmaxnreg split assumes the kernel was built with kLaunchRegs per
-    // thread; with fewer, the softmax warps' register request could never be met
-    cudaFuncAttributes fa;
-    cudaError_t err = e4m3 ? cudaFuncGetAttributes(&fa, attention_kernel<true>)
-                           : cudaFuncGetAttributes(&fa, attention_kernel<false>);
-    if (err != cudaSuccess) return err;
-    if (fa.numRegs < kLaunchRegs) return cudaErrorInvalidConfiguration;
     // persistent: one CTA per SM, work items taken from a counter in the workspace
     int dev = 0, sms = 0;
+    cudaError_t err;
     if ((err = cudaGetDevice(&dev)) != cudaSuccess) return err;
     if ((err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
         return err;
     const unsigned grid = static_cast<unsigned>(items < sms ? items : sms);
-    if (e4m3) {
-        err = cudaFuncSetAttribute(attention_kernel<true>,
-                                   cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-        if (err != cudaSuccess) return err;
-        attention_kernel<true><<<grid, kThreads, smem, stream>>>(a, tq, tk, tv, tkb, tvb);
-    } else {
-        err = cudaFuncSetAttribute(attention_kernel<false>,
-                                   cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-        if (err != cudaSuccess) return err;
-        attention_kernel<false><<<grid, kThreads, smem, stream>>>(a, tq, tk, tv, tkb, tvb);
-    }
-    return cudaGetLastError();
+    if (e4m3)
+        return var ? launch_one<true, true>(a, tq, tk, tv, tkb, tvb, grid, smem, stream)
+                   : launch_one<true, false>(a, tq, tk, tv, tkb, tvb, grid, smem, stream);
+    return var ? launch_one<false, true>(a, tq, tk, tv, tkb, tvb, grid, smem, stream)
+               : launch_one<false, false>(a, tq, tk, tv, tkb, tvb, grid, smem, stream);
 }
 
 }  // namespace fp2

@@ -220,6 +220,14 @@ struct PoolVec;
 template <>
 struct PoolVec<false> {  // 8 bf16 per 16 bytes
     static constexpr int N = 8;
+    __device__ static void unpack(float* x, uint4 v) {
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            x[2 * i] = __uint_as_float(w[i] << 16);
+            x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+        }
+    }
     __device__ static void add(float* acc, uint4 v) {
         const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
@@ -232,6 +240,22 @@ struct PoolVec<false> {  // 8 bf16 per 16 bytes
 template <>
 struct PoolVec<true> {  // 16 e4m3 per 16 bytes
     static constexpr int N = 16;
+    __device__ static void unpack(float* x, uint4 v) {
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            __half2_raw lo = __nv_cvt_fp8x2_to_halfraw2(
+                static_cast<__nv_fp8x2_storage_t>(w[i] & 0xFFFF), __NV_E4M3);
+            __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2(
+                static_cast<__nv_fp8x2_storage_t>(w[i] >> 16), __NV_E4M3);
+            float2 a = __half22float2(*reinterpret_cast<__half2*>(&lo));
+            float2 b = __half22float2(*reinterpret_cast<__half2*>(&hi));
+            x[4 * i] = a.x;
+            x[4 * i + 1] = a.y;
+            x[4 * i + 2] = b.x;
+            x[4 * i + 3] = b.y;
+        }
+    }
     __device__ static void add(float* acc, uint4 v) {
         const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
@@ -336,9 +360,14 @@ __global__ void __launch_bounds__(kPoolThreads, 1)
             const int32_t ncols = a.heads[x] * kHeadDim;
             const int32_t col = p.y * a.hb[x] * kHeadDim + tc * N;
             const bool active = tc * 16 < row_bytes && col < ncols;
+            // key units with a variance output also sum (x - shift)^2, the shift
+            // being the block's first row (no cancellation for a large mean)
+            const bool var_unit = x == 1 && a.kvar != nullptr;
             float acc[N];
+            float sh[N];
+            float sq = 0.f;
 #pragma unroll
-            for (int e = 0; e < N; ++e) acc[e] = 0.f;
+            for (int e = 0; e < N; ++e) acc[e] = sh[e] = 0.f;
             const int32_t nsub = (p.n + kPoolStageRows - 1) / kPoolStageRows;
             for (int32_t sub = 0; sub < nsub; ++sub, ++cnt) {
                 const int32_t st = cnt % kPoolStages;
@@ -348,9 +377,24 @@ __global__ void __launch_bounds__(kPoolThreads, 1)
                 if (ok && active) {
                     const uint8_t* base = stages + st * kPoolStageBytes + tc * 16;
                     const int32_t nr = min(kPoolStageRows, p.n - sub * kPoolStageRows);
+                    if (!var_unit) {
 #pragma unroll 4
-                    for (int32_t rr = rg; rr < nr; rr += 4)
-                        V::add(acc, *reinterpret_cast<const uint4*>(base + rr * row_bytes));
+                        for (int32_t rr = rg; rr < nr; rr += 4)
+                            V::add(acc, *reinterpret_cast<const uint4*>(base + rr * row_bytes));
+                    } else {
+                        if (sub == 0) V::unpack(sh, *reinterpret_cast<const uint4*>(base));
+#pragma unroll 2
+                        for (int32_t rr = rg; rr < nr; rr += 4) {
+                            float xv[N];
+                            V::unpack(xv, *reinterpret_cast<const uint4*>(base + rr * row_bytes));
+#pragma unroll
+                            for (int e = 0; e < N; ++e) {
+                                acc[e] += xv[e];
+                                const float dv = xv[e] - sh[e];
+                                sq = fmaf(dv, dv, sq);
+                            }
+                        }
+                    }
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&ps->empty[st]);
@@ -358,8 +402,36 @@ __global__ void __launch_bounds__(kPoolThreads, 1)
             if (rg > 0) {
 #pragma unroll
                 for (int e = 0; e < N; ++e) red[rg - 1][tc][e] = acc[e];
+                red[rg - 1][tc][N] = sq;
             }
             named_sync_pool();
+            if (rg == 0 && var_unit) {
+                // mean key variance of every head of the slab: per lane, the sum over
+                // its columns of E[(x - s)^2] - (mean - s)^2; then the lanes of a head
+                // (warp-aligned groups of 128 / N) add up, and the first one writes
+                float lv = 0.f;
+                if (active && ok) {
+#pragma unroll
+                    for (int g = 0; g < 3; ++g) sq += red[g][tc][N];
+                    float m2 = 0.f;
+#pragma unroll
+                    for (int e = 0; e < N; ++e) {
+                        float tot = acc[e];
+#pragma unroll
+                        for (int g = 0; g < 3; ++g) tot += red[g][tc][e];
+                        const float dm = tot / static_cast<float>(p.n) - sh[e];
+                        m2 = fmaf(dm, dm, m2);
+                    }
+                    lv = sq / static_cast<float>(p.n) - m2;
+                }
+#pragma unroll
+                for (int o = 1; o < kHeadDim / N; o <<= 1) lv += __shfl_xor_sync(0xffffffffu, lv, o);
+                if (active && ok && (tc % (kHeadDim / N)) == 0) {
+                    const int32_t h = col / kHeadDim;
+                    const float s = a.scale[x] ? a.scale[x][h] : 1.f;
+                    a.kvar[static_cast<int64_t>(p.t) * a.heads[x] + h] = fmaxf(lv, 0.f) * s * s / kHeadDim;
+                }
+            }
             if (rg == 0 && active && ok) {
 #pragma unroll
                 for (int g = 0; g < 3; ++g)

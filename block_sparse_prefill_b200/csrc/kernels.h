@@ -45,6 +45,8 @@ __host__ __device__ inline int32_t setup_bins(int32_t nb_cap, bool cost) {
 
 struct PoolArgs {
     float* out[3];           // fp32 means (NULL = not written): -, k_mean, v_mean
+    float* kvar;             // NULL, or [max_blocks, Hkv]: key variance of every block, averaged
+                             // over the dimensions (dequantised)
     uint16_t* split[2];      // bf16 hi/lo means of q (grouped rows) and k, see WsLayout
     const float* scale[3];   // per-head dequantisation scales (NULL = 1)
     int32_t heads[3];
@@ -113,7 +115,9 @@ struct AttnArgs {
     int32_t nb_max;              // row stride of kept_idx
     int32_t nb_cap;              // >= key blocks of the longest request (shared-memory lists)
     int32_t hq, hkv, G, pairs;   // pairs = ceil(G / 2) CTAs per (q-block, KV head)
-    int32_t correction;
+    int32_t correction;          // 0 none, 1 mean, 2 mean with the variance term
+    const float* k_var;          // correction 2: [max_blocks, Hkv] mean key variance per block
+    float var_coef;              // correction 2: tau^2 / 2 * log2(e)
     int32_t test_wait_timeout;   // 1: the MMA issuer waits on a barrier nothing completes
                                  // (tests the bounded-wait timeout and abort path)
     float scale_log2;            // tau * log2(e)
@@ -139,8 +143,9 @@ __global__ void score_kernel(const __grid_constant__ ScoreArgs a,
 size_t score_smem_bytes();
 __global__ void meanlp_kernel(MeanLpArgs a);
 
-// Shared-memory bytes of the attention kernel for a kept-list capacity.
-size_t attn_smem_bytes(bool e4m3, int32_t nb_cap);
+// Shared-memory bytes of the attention kernel for a kept-list capacity (var:
+// correction 2, which stages one variance per pruned block).
+size_t attn_smem_bytes(bool e4m3, int32_t nb_cap, bool var);
 // Launches the persistent attention kernel: one CTA per SM, taking work items
 // (q-block, KV head, query-head pair) from a counter in the workspace.
 cudaError_t launch_attention(bool e4m3, const AttnArgs& a, const CUtensorMap& tq,

@@ -307,6 +307,17 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
     return r;
 }
 
+// The two e4m3 values in the low 16 bits of `w` as f16x2 (exact).
+__device__ __forceinline__ __half2 e4m3x2_to_half2(uint32_t w) {
+    uint32_t r;
+    asm("{\n\t.reg .b16 a;\n\t"
+        "cvt.u16.u32 a, %1;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %0, a;\n\t}"
+        : "=r"(r)
+        : "r"(w));
+    return *reinterpret_cast<__half2*>(&r);
+}
+
 // Sum of the four e4m3 values packed in `w` (exact decode to f16x2, f16x2 adds).
 __device__ __forceinline__ __half2 e4m3x4_sum2(uint32_t w) {
     uint32_t lo, hi;

@@ -94,7 +94,8 @@ typedef struct fp2_params {
     int32_t block_size;        /* must be 128; also the KV page size */
     float alpha;               /* threshold; <= 0 keeps every causal block; must be <= 1 */
     float sm_scale;            /* softmax scale tau; 0 selects 1/sqrt(head_dim) */
-    int32_t correction;        /* 0: drop pruned blocks; 1: mean correction */
+    int32_t correction;        /* 0: drop pruned blocks; 1: mean correction; 2: mean correction
+                                  with the variance term (see fp2_sparse_prefill) */
     int32_t dtype;             /* fp2_dtype */
     const float* q_scale;      /* e4m3 only: device [Hq] dequantisation scales, finite and
                                   >= 0 (an all-zero head may have scale 0) */
@@ -114,6 +115,10 @@ typedef struct fp2_blockmeta {
                                   entries j > i are left untouched */
     int32_t nb_max;            /* row stride of kept_idx / score_dbg, >= ceil(max_seqlen / block_size) */
     int32_t max_blocks;        /* capacity in blocks, >= sum_b ceil(L_b / block_size) */
+    float* k_var;              /* optional (NULL): [max_blocks, Hkv] fp32, the key variance of
+                                  every block averaged over the head dimensions (dequantised);
+                                  written by the estimator when non-NULL, needed when
+                                  correction == 2 */
 } fp2_blockmeta;
 
 /* Upper bound of sum_b ceil(L_b / block_size) for any batch of `batch` requests
@@ -168,16 +173,29 @@ fp2_status fp2_estimate(const fp2_params* params, const void* q, const void* k, 
  * the diagonal block i), plus the mean correction when params->correction != 0
  * (then meta->k_mean and v_mean must hold the block means).  Writes out (bf16)
  * and, when non-NULL, lse.  `meta` is only read.
+ * correction == 2 adds to every pruned block's corrected logit the second-order
+ * term (sm_scale^2 / 2) |q_r|^2 kvar_j, kvar_j = meta->k_var (the block's key
+ * variance averaged over the dimensions): by Jensen's inequality the plain mean
+ * correction undercounts a block's mass by about e^{var/2} of its logits, and
+ * this term restores it when the keys' variance is spread evenly over the
+ * dimensions.  It is an extension of the write-ups' mean correction (lode.cx,
+ * "How It Works"; aimodeling.com: the correction suppresses the approximation
+ * error), not a step they state.  Its length limit is lower: the attention
+ * stages one variance per pruned block, so ceil(max_seqlen / block_size) may be
+ * at most FP2_MAX_SEQ_BLOCKS_VAR_BF16 (2048 blocks, 262144 tokens) for bf16 or
+ * FP2_MAX_SEQ_BLOCKS_VAR_E4M3 (4096 blocks, 524288 tokens) for e4m3.
  * Length limit of the attention calls (this one, fp2_prefill_paged and
  * fp2_sparse_prefill_noalloc): a work item keeps its kept-block list in shared
  * memory, so ceil(max_seqlen / block_size) may be at most FP2_MAX_SEQ_BLOCKS_BF16
- * (4133 blocks, 529024 tokens) for bf16 and FP2_MAX_SEQ_BLOCKS_E4M3 (8075
- * blocks, 1033600 tokens) for e4m3; longer returns FP2_ERR_UNSUPPORTED.
+ * (4129 blocks, 528512 tokens) for bf16 and FP2_MAX_SEQ_BLOCKS_E4M3 (8071
+ * blocks, 1033088 tokens) for e4m3; longer returns FP2_ERR_UNSUPPORTED.
  * Errors: bad arguments or sizes are returned before anything is enqueued; a
  * kept list that breaks the rules above is flagged on the device
  * (FP2_ERR_BAD_INDEX) and replaced by the diagonal block alone. */
-#define FP2_MAX_SEQ_BLOCKS_BF16 4133
-#define FP2_MAX_SEQ_BLOCKS_E4M3 8075
+#define FP2_MAX_SEQ_BLOCKS_BF16 4129
+#define FP2_MAX_SEQ_BLOCKS_E4M3 8071
+#define FP2_MAX_SEQ_BLOCKS_VAR_BF16 2048
+#define FP2_MAX_SEQ_BLOCKS_VAR_E4M3 4096
 fp2_status fp2_sparse_prefill(const fp2_params* params, const void* q, const void* k,
                               const void* v, const int32_t* cu_seqlens, int32_t batch,
                               int64_t total_tokens, int32_t max_seqlen,

@@ -74,6 +74,7 @@ def run_gpu(wl, alpha=None, correction=True, paged=False, scores=False, lse=True
         "kept_idx": meta.kept_idx[:nblk].cpu().numpy(),
         "k_mean": meta.k_mean[:nblk].cpu().numpy(),
         "v_mean": meta.v_mean[:nblk].cpu().numpy(),
+        "k_var": meta.k_var[:nblk].cpu().numpy(),
         "o": out.float().cpu().numpy(),
         "lse": lse_t.cpu().numpy() if lse else None,
         "score_dbg": meta.score_dbg[:nblk].cpu().numpy() if scores else None,

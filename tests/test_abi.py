@@ -75,7 +75,8 @@ def _estimate(lib, p, **kw):
     (dict(alpha=1.5), 1),
     (dict(alpha=float("nan")), 1),
     (dict(sm_scale=-1.0), 1),
-    (dict(correction=2), 1),
+    (dict(correction=3), 1),
+    (dict(correction=-1), 1),
     (dict(dtype=7), 1),
     (dict(dtype=1), 1),          # e4m3 without scales
 ])
@@ -196,15 +197,15 @@ def test_prototypes_match_the_ctypes_declarations(lib):
 def _max_seq_blocks():
     text = open(HEADER).read()
     return {name: int(re.search(rf"#define FP2_MAX_SEQ_BLOCKS_{name}\s+(\d+)", text).group(1))
-            for name in ("BF16", "E4M3")}
+            for name in ("BF16", "E4M3", "VAR_BF16", "VAR_E4M3")}
 
 
-def _attention_call(lib, fn, dtype, max_seqlen):
+def _attention_call(lib, fn, dtype, max_seqlen, correction=1):
     """An attention call with fake (never dereferenced) device addresses."""
     sc = 4096 if dtype else None
-    p = _lib.fp2_params(32, 8, 128, 128, 0.05, 0.0, 1, dtype, sc, sc, sc)
+    p = _lib.fp2_params(32, 8, 128, 128, 0.05, 0.0, correction, dtype, sc, sc, sc)
     nb = (max_seqlen + 127) // 128
-    m = _lib.fp2_blockmeta(4096, 4096, 4096, 4096, None, nb, nb + 1)
+    m = _lib.fp2_blockmeta(4096, 4096, 4096, 4096, None, nb, nb + 1, 4096)
     a = ctypes.c_void_p(4096)
     if fn == "fp2_prefill_paged":
         return lib.fp2_prefill_paged(ctypes.byref(p), a, a, a, a, 1, max_seqlen, max_seqlen, a, nb, nb,
@@ -213,23 +214,26 @@ def _attention_call(lib, fn, dtype, max_seqlen):
                                   a, None, ctypes.c_void_p(1 << 20), 1 << 40, None)
 
 
+LIMITS = [(0, "BF16", 1), (1, "E4M3", 1), (0, "VAR_BF16", 2), (1, "VAR_E4M3", 2)]
+
+
 @pytest.mark.parametrize("fn", ["fp2_sparse_prefill", "fp2_prefill_paged"])
-@pytest.mark.parametrize("dtype,name", [(0, "BF16"), (1, "E4M3")])
-def test_length_limit_rejected_before_any_launch(lib, fn, dtype, name):
-    """One block past the documented limit returns FP2_ERR_UNSUPPORTED, and the
-    paged call returns it before enqueueing its estimator."""
+@pytest.mark.parametrize("dtype,name,corr", LIMITS)
+def test_length_limit_rejected_before_any_launch(lib, fn, dtype, name, corr):
+    """One block past the documented limit returns FP2_ERR_UNSUPPORTED before anything
+    is enqueued."""
     limit = _max_seq_blocks()[name]
-    assert _attention_call(lib, fn, dtype, limit * 128 + 1) == 2
+    assert _attention_call(lib, fn, dtype, limit * 128 + 1, corr) == 2
 
 
 @pytest.mark.skipif(__import__("torch").cuda.is_available(),
                     reason="the accepted call would launch kernels on fake addresses")
-@pytest.mark.parametrize("dtype,name", [(0, "BF16"), (1, "E4M3")])
-def test_length_limit_is_tight(lib, dtype, name):
+@pytest.mark.parametrize("dtype,name,corr", LIMITS)
+def test_length_limit_is_tight(lib, dtype, name, corr):
     """At the documented limit every host check passes: without a GPU the call
     gets as far as the first CUDA call and returns FP2_ERR_CUDA."""
     limit = _max_seq_blocks()[name]
-    assert _attention_call(lib, "fp2_sparse_prefill", dtype, limit * 128) == 4
+    assert _attention_call(lib, "fp2_sparse_prefill", dtype, limit * 128, corr) == 4
 
 
 def test_missing_library_fails_loudly(monkeypatch):
@@ -269,3 +273,13 @@ def test_plain_c_client_links_and_calls_the_library(lib):
                 os.remove(f)
     assert out[:4] == [str(lib.fp2_version()), "1025", "1", "1"], out
     assert " ".join(out[4:]) == "invalid argument"
+
+
+def test_variance_correction_needs_k_var(lib):
+    """correction = 2 reads the block key variances: an attention call whose meta has no
+    k_var is an argument error (nothing enqueued); the estimator does not need it."""
+    p = _params(correction=2)
+    a = ctypes.c_void_p(4096)
+    m = _lib.fp2_blockmeta(4096, 4096, 4096, 4096, None, 8, 9)      # k_var NULL
+    assert lib.fp2_sparse_prefill(ctypes.byref(p), a, a, a, a, 1, 1024, 1024, ctypes.byref(m), a, None,
+                                  ctypes.c_void_p(1 << 20), 1 << 40, None) == 1

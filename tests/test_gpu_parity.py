@@ -217,3 +217,46 @@ def test_e4m3_head_with_zero_scale():
     assert np.isfinite(g["o"]).all() and np.isfinite(g["lse"]).all()
     _check_masks(wl, g)
     _check_outputs(wl, g, True, max_abs=E4M3_MAX_ABS, mean_abs=1.0, lse_abs=E4M3_MAX_ABS)
+
+
+def _check_variance(wl, g, sel=None, max_abs=BF16_MAX_ABS, mean_abs=BF16_MEAN_ABS, lse_abs=2e-2):
+    """Correction 2 against the oracle's correction with the isotropic variance term
+    (its mode 4) on the GPU's lists, and the per-block mean key variances."""
+    orc = oracle()
+    q, k, v = wl.float_inputs()
+    cu = wl.cu_seqlens
+    kbar = orc.block_means(k, cu, 128, wl.k_scale)
+    vbar = orc.block_means(v, cu, 128, wl.v_scale)
+    kvar = orc.block_vars(k, cu, 128, kbar, wl.k_scale)
+    want = kvar.mean(axis=2)
+    assert np.abs(g["k_var"] - want).max() <= 1e-4 * max(1.0, np.abs(want).max()), "block key variances"
+    ref = orc.attend(q, k, v, cu, 128, tau(wl), g["kept_cnt"], g["kept_idx"], correction=4, kbar=kbar, vbar=vbar,
+                     kvar=kvar, q_scale=wl.q_scale, k_scale=wl.k_scale, v_scale=wl.v_scale, sel=sel)
+    rows = None if sel is None else rows_of_blocks(cu, sel)
+    mx, mn = out_errors(g["o"], ref["o"], rows)
+    assert mx <= max_abs and mn <= mean_abs, f"output max-abs {mx:.3e} mean-abs {mn:.3e}"
+    lm, _ = out_errors(g["lse"], ref["lse"], rows)
+    assert lm < lse_abs, f"lse max-abs {lm:.3e}"
+
+
+@pytest.mark.parametrize("paged", [False, True])
+@pytest.mark.parametrize("dtype", ["bf16", "e4m3"])
+def test_variance_correction(dtype, paged):
+    """correction = 2: the mean correction plus (tau^2 / 2) |q_r|^2 kvar_j on every pruned
+    block, G = 4 and G = 3 (one query head alone in its last work item)."""
+    for hq, hkv, seed in ((8, 2, 61), (6, 2, 62)):
+        wl = make_workload([1000, 700, 2000, 129, 1], hq, hkv, alpha=0.1, seed=seed, dtype=dtype, paged=paged)
+        g = run_gpu(wl, correction=2, paged=paged)
+        _check_masks(wl, g)
+        if dtype == "bf16":
+            _check_variance(wl, g)
+        else:
+            _check_variance(wl, g, max_abs=E4M3_MAX_ABS, mean_abs=1.0, lse_abs=E4M3_MAX_ABS)
+
+
+def test_variance_correction_32k_sampled():
+    wl = make_config(1)
+    g = run_gpu(wl, correction=2)
+    nblk = g["kept_cnt"].shape[0]
+    sel = sample_blocks(nblk, 12, seed=21, include=(0, nblk - 1))
+    _check_variance(wl, g, sel=sel)

@@ -2,8 +2,11 @@
 
 The attention kernel runs one CTA per SM (148).  The CTAs take work items (one
 q-block x two query heads of one KV head) from a shared counter, in the order
-the setup kernel writes: by the q-block's index in its request, largest first.
-A CTA that finishes takes the next item, which is greedy list scheduling.
+the attention call's setup kernel writes: by the item's cost (kept tiles +
+correction tiles + fill, the cost modelled below; `item_cost` in estimator.cu),
+largest first.  A CTA that finishes takes the next item, which is greedy list
+scheduling.  The block-index order (the q-block's index in its request, largest
+first) is what the kernel used before; it is kept here for comparison.
 
 This test models an item's cost as:
   - its kept K/V tiles, with kept lists from the oracle's estimator;
