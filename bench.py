@@ -37,9 +37,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 E4M3_OVER_BF16 = 2.0  # nominal dense ratio (4.5 / 2.25 PFLOP/s)
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch of the 128K bf16 layer's
 # kernels, from one single-pass ncu capture each of the kernels as they stand (attention:
-# 6.26 GB read + 1.06 GB written; pooling: 1.61 GB + 0.03 GB).  Reported only for that
+# 6.40 GB read + 1.06 GB written; pooling: 1.61 GB + 0.03 GB).  Reported only for that
 # workload; to be captured again whenever these kernels change.
-TRAFFIC_128K = {"attention": 7.32e9, "pool": 1.64e9}
+TRAFFIC_128K = {"attention": 7.47e9, "pool": 1.64e9}
 
 
 def load_peaks():
@@ -546,7 +546,7 @@ def mask_parity(wl, est, gpu_cnt, gpu_idx, near_threshold):
                     "the threshold m + ln(alpha) for some head of the group"}
 
 
-def cpu_baseline(wl, n_sample=16, shift=0, gpu_kept=None):
+def cpu_baseline(wl, n_sample=48, shift=0, gpu_kept=None):
     """The oracle on a bounded sample of the layer, timed on the host cores: its float
     build (the same code as the double parity build, compiled with -DORC_FP32; OpenMP
     over the host cores) runs the full estimator, then attention on `n_sample` q-blocks
@@ -801,6 +801,52 @@ def e4m3_only(args):
                       "tflops_attention_kept_pairs_only": f8 / (a8 * 1e-3) / 1e12}), flush=True)
 
 
+def paged_batch(args):
+    """The paged ragged batch alone (1 GPU): 8 requests with lengths log-uniform in [4096,
+    131072] (this seed: 4K-75K tokens, 177K in all), K/V in a page pool in seeded random
+    order; `--warmup` untimed and `--steps` timed layers of fp2_estimate (on the pool) +
+    fp2_prefill_paged; one JSON line."""
+    import torch
+    import block_sparse_prefill_b200 as fp2
+    from workloads import make_config
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    wl = make_config(4)
+    params = fp2.Params(num_q_heads=wl.num_q_heads, num_kv_heads=wl.num_kv_heads, alpha=wl.alpha)
+    T, B = wl.total_tokens, wl.batch
+    q, kp, vp = wl.q.to(dev), wl.k_pool.to(dev), wl.v_pool.to(dev)
+    cu = torch.from_numpy(wl.cu_seqlens).to(dev)
+    bt = torch.from_numpy(wl.block_table).to(dev)
+    meta = fp2.BlockMeta.empty(params, B, T, wl.max_seqlen, dev)
+    ws = fp2.Workspace(params, B, T, wl.max_seqlen, dev)
+    out = torch.empty((T, wl.num_q_heads, 128), dtype=torch.bfloat16, device=dev)
+
+    def layer():
+        fp2.estimate(params, q, kp, vp, cu, wl.max_seqlen, meta, ws, block_table=bt, num_pages=wl.num_pages)
+        fp2.prefill_paged(params, q, kp, vp, cu, wl.max_seqlen, bt, wl.num_pages, meta, out, ws)
+
+    for _ in range(args.warmup):
+        layer()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        layer()
+    e1.record()
+    torch.cuda.synchronize()
+    err = fp2.get_error(ws)
+    if err != 0:
+        raise RuntimeError(f"device error: {fp2.status_string(err)}")
+    ms = e0.elapsed_time(e1) / args.steps
+    f, c = layer_work(wl.seqlens, meta.kept_cnt.cpu().numpy(), meta.kept_idx.cpu().numpy(), wl.num_q_heads,
+                      wl.num_kv_heads)
+    print(json.dumps({"workload": f"paged ragged batch: {B} requests, {T} tokens ({min(wl.seqlens)}-"
+                                  f"{max(wl.seqlens)}), Hq=32, Hkv=8, d=128, bf16, alpha=0.05, pool pages in "
+                                  "random order",
+                      "ms_per_layer": ms, "tflops_layer_kept_pairs": f / (ms * 1e-3) / 1e12,
+                      "tflops_layer_with_correction": (f + c) / (ms * 1e-3) / 1e12}), flush=True)
+
+
 def reference(args):
     """The CPU oracle as the reference arm, on bounded samples of the layer."""
     rank = int(os.environ.get("RANK", "0"))
@@ -848,6 +894,9 @@ def main():
                     help="shorter sequence for profiling runs (default: the 128K workload)")
     ap.add_argument("--no-approx", action="store_true",
                     help="skip the approximation-quality study (its extra attention calls) in profiling runs")
+    ap.add_argument("--paged-batch", action="store_true",
+                    help="time the paged ragged batch (8 requests, 4K-75K tokens, one page pool) instead of "
+                         "the 128K layer")
     ap.add_argument("--e4m3-only", action="store_true",
                     help="profiling aid: time only the e4m3 layer (config 3) and print its line, so that "
                          "a profiler sees no bf16 launch")
@@ -858,6 +907,8 @@ def main():
         reference(args)
     elif args.e4m3_only:
         e4m3_only(args)
+    elif args.paged_batch:
+        paged_batch(args)
     else:
         ours(args)
 

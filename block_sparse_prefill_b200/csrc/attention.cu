@@ -59,10 +59,12 @@ constexpr int kSchedWarp = 10;
 constexpr uint32_t kTmemCols = 512;
 // Registers per thread after the split.  setmaxnreg only redistributes the
 // registers the CTA was launched with (384 threads x 168 = 64512), so
-// 256 x kSoftmaxRegs + 128 x kOtherRegs must not exceed that: 53248 + 11264.
+// 256 x kSoftmaxRegs + 128 x kOtherRegs must not exceed that: 55296 + 9216.
+// With 216 the softmax keeps a whole row of S without spilling (208 spilled);
+// the producer, issuer and scheduler fit in 72.
 constexpr int kLaunchRegs = 168;
-constexpr int kSoftmaxRegs = 208;
-constexpr int kOtherRegs = 88;
+constexpr int kSoftmaxRegs = 216;
+constexpr int kOtherRegs = 72;
 static_assert(256 * kSoftmaxRegs + 128 * kOtherRegs <= kThreads * kLaunchRegs,
               "register split exceeds the launch allocation");
 
@@ -695,20 +697,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // a correction column stands for the 128 keys of a pruned block: its
                 // weight is 128 e^{lbar}, i.e. +log2(128) on the scaled logit
                 const float bias = (n >= cnt) ? 7.f : 0.f;
-                // scale of the tile's values in the max and the exponent: qk, or 1 for
-                // correction 2's tiles, whose scaled logits get + w * coef_j here
-                float sc = qk;
+                // correction 2: the scaled logit of a correction column gets + w coef_j,
+                // i.e. the raw score gets + (w / qk) coef_j (one packed FMA per pair)
+                const float sc = qk;
                 if (var && n >= cnt) {
                     const float4* cv = reinterpret_cast<const float4*>(cvals_of(m) + (n - cnt) * 128);
+                    const float wq = w / qk;
 #pragma unroll
                     for (int c4 = 0; c4 < 32; ++c4) {
                         const float4 cc = cv[c4];
-                        sv[4 * c4] = __float_as_uint(fmaf(w, cc.x, __uint_as_float(sv[4 * c4]) * qk));
-                        sv[4 * c4 + 1] = __float_as_uint(fmaf(w, cc.y, __uint_as_float(sv[4 * c4 + 1]) * qk));
-                        sv[4 * c4 + 2] = __float_as_uint(fmaf(w, cc.z, __uint_as_float(sv[4 * c4 + 2]) * qk));
-                        sv[4 * c4 + 3] = __float_as_uint(fmaf(w, cc.w, __uint_as_float(sv[4 * c4 + 3]) * qk));
+                        const float2 lo = ffma2(make_float2(wq, wq), make_float2(cc.x, cc.y),
+                                                make_float2(__uint_as_float(sv[4 * c4]), __uint_as_float(sv[4 * c4 + 1])));
+                        const float2 hi = ffma2(make_float2(wq, wq), make_float2(cc.z, cc.w),
+                                                make_float2(__uint_as_float(sv[4 * c4 + 2]), __uint_as_float(sv[4 * c4 + 3])));
+                        sv[4 * c4] = __float_as_uint(lo.x);
+                        sv[4 * c4 + 1] = __float_as_uint(lo.y);
+                        sv[4 * c4 + 2] = __float_as_uint(hi.x);
+                        sv[4 * c4 + 3] = __float_as_uint(hi.y);
                     }
-                    sc = 1.f;
                 }
                 // row max over 4 independent 3-input max chains
                 float mxp[4];

@@ -21,10 +21,15 @@ def pytest_terminal_summary(terminalreporter):
     mask tolerance: blocks whose oracle score lies within 1e-3 relative of the
     threshold are excused from bit-exactness, counted and reported here)."""
     helpers = sys.modules.get("gpu_helpers")
+    tr = terminalreporter
+    outs = getattr(helpers, "OUT_STATS", None)
+    if outs:
+        tr.section("output parity: errors against the oracle on the same kept lists")
+        for label, mx, mn in outs:
+            tr.write_line(f"{label.split('::')[-1]}: max-abs {mx:.2e} mean-abs {mn:.2e}")
     stats = getattr(helpers, "MASK_STATS", None)
     if not stats:
         return
-    tr = terminalreporter
     tr.section("mask parity: near-threshold blocks")
     tot = {"near": 0, "excused": 0, "outside": 0, "compared": 0}
     for label, r in stats:

@@ -141,6 +141,15 @@ def check_mask_counts(res):
         f"({res['near']} near, {res['compared']} compared)")
 
 
+# output errors of every parity check in this session, printed by conftest.py's
+# terminal summary: (test, max-abs, mean-abs)
+OUT_STATS = []
+
+
+def record_output_errors(label, mx, mn):
+    OUT_STATS.append((label, mx, mn))
+
+
 def out_errors(gpu_o, ref_o, rows=None):
     a, b = gpu_o, ref_o
     if rows is not None:

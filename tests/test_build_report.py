@@ -3,8 +3,8 @@
 The attention kernel's warp roles trade registers with setmaxnreg, which only
 redistributes what the CTA was launched with; the kernel must therefore be
 built with exactly kLaunchRegs per thread (the host refuses to launch it with
-fewer).  Its few spills are known and bounded; the other kernels must not
-spill at all."""
+fewer).  With the 216 / 72 split it does not spill today; the bound below
+leaves a little room.  The other kernels must not spill at all."""
 import os
 import re
 
@@ -24,7 +24,7 @@ def test_kernel_registers_and_spills():
     assert len(att) == 4, names                      # bf16 and e4m3, without and with the variance term
     for k in att:
         assert k["regs"] == _launch_regs(), k
-        assert k["spill_stores"] <= 64 and k["spill_loads"] <= 256, k
+        assert k["spill_stores"] <= 16 and k["spill_loads"] <= 64, k
     for short in ("pool_kernel", "score_kernel", "meanlp_kernel", "setup_kernel"):
         ks = [k for k in rep if short in k["name"]]
         assert ks, short

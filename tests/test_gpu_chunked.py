@@ -14,8 +14,8 @@ import numpy as np
 import pytest
 
 from gpu_helpers import (BF16_MAX_ABS, BF16_MEAN_ABS, E4M3_MAX_ABS, check_mask_counts, chunk_block_index,
-                         chunk_rows_of_blocks, compare_masks, oracle, out_errors, run_gpu, run_gpu_chunked,
-                         sample_blocks)
+                         chunk_rows_of_blocks, compare_masks, oracle, out_errors, record_output_errors, run_gpu,
+                         run_gpu_chunked, sample_blocks)
 from workloads import make_chunked_workload, make_workload
 
 pytestmark = pytest.mark.gpu
@@ -38,6 +38,7 @@ def _check(wl, g, sel=None, e4m3=False):
     ref = orc.run(wl, kept={"kept_cnt": g["kept_cnt"], "kept_idx": g["kept_idx"]}, sel=sel)
     rows = None if sel is None else chunk_rows_of_blocks(wl, sel)
     mx, mn = out_errors(g["o"], ref["o"], rows)
+    record_output_errors(_label(), mx, mn)
     lm, _ = out_errors(g["lse"], ref["lse"], rows)
     if e4m3:
         assert mx <= E4M3_MAX_ABS and lm < E4M3_MAX_ABS, f"max-abs {mx:.3e} lse {lm:.3e}"
