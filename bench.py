@@ -365,23 +365,26 @@ def approximation_error(st, wl, n_rows=256, seed=7):
                     q_scale=base.q_scale, k_scale=base.k_scale, v_scale=base.v_scale)
     out0 = torch.empty_like(st["out"])
     out2 = torch.empty_like(st["out"])
+    # the variance term needs the block key variances: the same estimate with k_var
+    meta2 = fp2.BlockMeta.empty(p2, wl.batch, T, wl.max_seqlen, st["q"].device)
+    fp2.estimate(p2, st["q"], st["k"], st["v"], st["cu"], wl.max_seqlen, meta2, st["ws"])
     fp2.sparse_prefill(p0, st["q"], st["k"], st["v"], st["cu"], wl.max_seqlen, st["meta"], out0, st["ws"])
-    fp2.sparse_prefill(p2, st["q"], st["k"], st["v"], st["cu"], wl.max_seqlen, st["meta"], out2, st["ws"])
+    fp2.sparse_prefill(p2, st["q"], st["k"], st["v"], st["cu"], wl.max_seqlen, meta2, out2, st["ws"])
     torch.cuda.synchronize()
 
-    def attention_ms(params, out, reps=5):
+    def attention_ms(params, meta, out, reps=5):
         for _ in range(2):
-            fp2.sparse_prefill(params, st["q"], st["k"], st["v"], st["cu"], wl.max_seqlen, st["meta"], out, st["ws"])
+            fp2.sparse_prefill(params, st["q"], st["k"], st["v"], st["cu"], wl.max_seqlen, meta, out, st["ws"])
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
         for _ in range(reps):
-            fp2.sparse_prefill(params, st["q"], st["k"], st["v"], st["cu"], wl.max_seqlen, st["meta"], out, st["ws"])
+            fp2.sparse_prefill(params, st["q"], st["k"], st["v"], st["cu"], wl.max_seqlen, meta, out, st["ws"])
         e1.record()
         torch.cuda.synchronize()
         return e0.elapsed_time(e1) / reps
 
-    ms_mean = attention_ms(base, torch.empty_like(st["out"]))
-    ms_var = attention_ms(p2, out2)
+    ms_mean = attention_ms(base, st["meta"], torch.empty_like(st["out"]))
+    ms_var = attention_ms(p2, meta2, out2)
     q = st["q"][rows_t].double()
     keys = torch.arange(T, device=q.device)
     causal = keys[None, :] > rows_t[:, None]
@@ -404,7 +407,7 @@ def approximation_error(st, wl, n_rows=256, seed=7):
         e = torch.stack(err[key])
         res[key + "_correction"] = {"max_abs": float(e.abs().max()), "mean_abs": float(e.abs().mean()),
                                     "rel_l2": math.sqrt(float((e ** 2).sum()) / ref_norm)}
-    del out0, out2
+    del out0, out2, meta2
     return res
 
 
@@ -546,7 +549,7 @@ def mask_parity(wl, est, gpu_cnt, gpu_idx, near_threshold):
                     "the threshold m + ln(alpha) for some head of the group"}
 
 
-def cpu_baseline(wl, n_sample=48, shift=0, gpu_kept=None):
+def cpu_baseline(wl, n_sample=64, shift=0, gpu_kept=None):
     """The oracle on a bounded sample of the layer, timed on the host cores: its float
     build (the same code as the double parity build, compiled with -DORC_FP32; OpenMP
     over the host cores) runs the full estimator, then attention on `n_sample` q-blocks
@@ -847,6 +850,60 @@ def paged_batch(args):
                       "tflops_layer_with_correction": (f + c) / (ms * 1e-3) / 1e12}), flush=True)
 
 
+def chunked(args):
+    """Chunked prefill alone (1 GPU): the last 16384 query rows of the 128K layer (its keys all
+    cached), bf16, through fp2_estimate_chunked + fp2_prefill_chunked; one JSON line."""
+    import torch
+    import block_sparse_prefill_b200 as fp2
+    from workloads import make_chunked_workload
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    S, Lq = args.seqlen or 131072, 16384
+    wl = make_chunked_workload([S], [Lq], 32, 8, alpha=0.05, seed=1002, n_retrieval=16)
+    params = fp2.Params(num_q_heads=32, num_kv_heads=8, alpha=wl.alpha)
+    Tk, Tq = wl.total_tokens, wl.total_queries
+    q, k, v = wl.q.to(dev), wl.k.to(dev), wl.v.to(dev)
+    cu_q = torch.from_numpy(wl.cu_seqlens_q).to(dev)
+    cu_k = torch.from_numpy(wl.cu_seqlens).to(dev)
+    meta = fp2.BlockMeta.empty(params, 1, Tk, S, dev)
+    ws = fp2.Workspace(params, 1, Tk, S, dev)
+    out = torch.empty((Tq, 32, 128), dtype=torch.bfloat16, device=dev)
+
+    def layer():
+        fp2.estimate_chunked(params, q, k, v, cu_q, cu_k, Tk, S, meta, ws)
+        fp2.prefill_chunked(params, q, k, v, cu_q, cu_k, Tk, S, meta, out, ws)
+
+    for _ in range(args.warmup):
+        layer()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        layer()
+    e1.record()
+    torch.cuda.synchronize()
+    err = fp2.get_error(ws)
+    if err != 0:
+        raise RuntimeError(f"device error: {fp2.status_string(err)}")
+    ms = e0.elapsed_time(e1) / args.steps
+    # kept-pair work of the chunk: rows of q-block i see the kept blocks j < i fully and the
+    # diagonal causally (the chunk starts on a block boundary here)
+    nq = Lq // 128
+    cnt = meta.kept_cnt[:nq].cpu().numpy()
+    idx = meta.kept_idx[:nq].cpu().numpy()
+    i0 = (S - Lq) // 128
+    pairs = 0
+    for t in range(nq):
+        i = i0 + t
+        for g in range(8):
+            js = idx[t, g, :cnt[t, g]]
+            pairs += 4 * (128 * 128 * int((js < i).sum()) + 128 * 129 // 2)
+    flops = 4.0 * 128 * pairs
+    print(json.dumps({"workload": f"chunked prefill: the last {Lq} of {S} tokens (keys cached), Hq=32, Hkv=8, "
+                                  "d=128, bf16, alpha=0.05",
+                      "ms_per_layer": ms, "tflops_kept_pairs": flops / (ms * 1e-3) / 1e12}), flush=True)
+
+
 def reference(args):
     """The CPU oracle as the reference arm, on bounded samples of the layer."""
     rank = int(os.environ.get("RANK", "0"))
@@ -897,6 +954,8 @@ def main():
     ap.add_argument("--paged-batch", action="store_true",
                     help="time the paged ragged batch (8 requests, 4K-75K tokens, one page pool) instead of "
                          "the 128K layer")
+    ap.add_argument("--chunked", action="store_true",
+                    help="time chunked prefill (the last 16K rows of the 128K layer) instead of the 128K layer")
     ap.add_argument("--e4m3-only", action="store_true",
                     help="profiling aid: time only the e4m3 layer (config 3) and print its line, so that "
                          "a profiler sees no bf16 launch")
@@ -909,6 +968,8 @@ def main():
         e4m3_only(args)
     elif args.paged_batch:
         paged_batch(args)
+    elif args.chunked:
+        chunked(args)
     else:
         ours(args)
 

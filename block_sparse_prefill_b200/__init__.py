@@ -207,7 +207,13 @@ class BlockMeta:
 
     @staticmethod
     def empty(params: Params, batch: int, total_tokens: int, max_seqlen: int, device="cuda",
-              scores: bool = False, nb_max: Optional[int] = None) -> "BlockMeta":
+              scores: bool = False, nb_max: Optional[int] = None,
+              variance: Optional[bool] = None) -> "BlockMeta":
+        """Device arrays for ``total_tokens`` keys.  ``variance`` (default: when
+        ``params.correction == 2``) also allocates ``k_var``, which the estimator
+        then fills (a little extra work in its pooling pass)."""
+        if variance is None:
+            variance = int(params.correction) == 2
         mb = max(1, max_blocks(batch, total_tokens))
         nbm = nb_max or max(1, (max_seqlen + BLOCK - 1) // BLOCK)
         hkv = params.num_kv_heads
@@ -219,7 +225,7 @@ class BlockMeta:
             score_dbg=(torch.full((mb, params.num_q_heads, nbm), float("nan"), dtype=torch.float32,
                                   device=device) if scores else None),
             nb_max=nbm, max_blocks=mb,
-            k_var=torch.zeros((mb, hkv), dtype=torch.float32, device=device))
+            k_var=torch.zeros((mb, hkv), dtype=torch.float32, device=device) if variance else None)
 
     def c(self) -> _lib.fp2_blockmeta:
         return _lib.fp2_blockmeta(_ptr(self.kept_cnt), _ptr(self.kept_idx), _ptr(self.k_mean),

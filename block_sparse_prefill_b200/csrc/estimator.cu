@@ -71,31 +71,29 @@ __global__ void setup_kernel(SetupArgs a) {
         if (!good) set_error(a.hdr, FP2_ERR_BAD_INDEX, bad);
         ok = good;
     }
-    for (int32_t e = threadIdx.x; e <= nbins; e += blockDim.x) hist[e] = 0;
+    if (cost)
+        for (int32_t e = threadIdx.x; e <= nbins; e += blockDim.x) hist[e] = 0;
     __syncthreads();
     if (!ok) return;
-    // request of every key block and q-block; histogram of the sort key: the
-    // q-block's absolute index in its request, or the cost of each (q-block,
-    // KV head) work item
+    // request of every key block and q-block; for the attention call, the
+    // histogram of the work items' costs
     for (int32_t b = 0; b < a.batch; ++b) {
         for (int32_t t = a.cu_blocks[b] + threadIdx.x; t < a.cu_blocks[b + 1]; t += blockDim.x)
             a.blk_req[t] = b;
         const int32_t i0 = req_span(a.cu_q, a.cu_k, b).i0, cq = a.cu_qblocks[b];
         for (int32_t t = cq + threadIdx.x; t < a.cu_qblocks[b + 1]; t += blockDim.x) {
             a.blk_req_q[t] = b;
-            const int32_t i = i0 + t - cq;
-            if (!cost)
-                atomicAdd(&hist[i], 1);
-            else
-                for (int32_t g = 0; g < a.hkv; ++g) atomicAdd(&hist[item_cost(a, t, i, g)], 1);
+            if (cost)
+                for (int32_t g = 0; g < a.hkv; ++g) atomicAdd(&hist[item_cost(a, t, i0 + t - cq, g)], 1);
         }
     }
+    // the estimator call needs no work order
+    if (!cost) return;
     __syncthreads();
-    // order: largest key first (the causal kept lists grow with the block index,
-    // so either key puts the longest work items first for the persistent
-    // attention kernel).  Exclusive scan of the histogram in descending key
-    // order: each thread scans a contiguous run of bins, the runs' totals are
-    // scanned across the block.
+    // order: largest cost first, so the persistent attention kernel takes the
+    // longest work items first.  Exclusive scan of the histogram in descending
+    // cost order: each thread scans a contiguous run of bins, the runs' totals
+    // are scanned across the block.
     {
         __shared__ int32_t wsum[32];
         const int32_t tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -132,14 +130,9 @@ __global__ void setup_kernel(SetupArgs a) {
     __syncthreads();
     for (int32_t b = 0; b < a.batch; ++b) {
         const int32_t i0 = req_span(a.cu_q, a.cu_k, b).i0, cq = a.cu_qblocks[b];
-        for (int32_t t = cq + threadIdx.x; t < a.cu_qblocks[b + 1]; t += blockDim.x) {
-            const int32_t i = i0 + t - cq;
-            if (!cost)
-                a.order[atomicAdd(&hist[i], 1)] = t;
-            else
-                for (int32_t g = 0; g < a.hkv; ++g)
-                    a.order[atomicAdd(&hist[item_cost(a, t, i, g)], 1)] = t * a.hkv + g;
-        }
+        for (int32_t t = cq + threadIdx.x; t < a.cu_qblocks[b + 1]; t += blockDim.x)
+            for (int32_t g = 0; g < a.hkv; ++g)
+                a.order[atomicAdd(&hist[item_cost(a, t, i0 + t - cq, g)], 1)] = t * a.hkv + g;
     }
 }
 

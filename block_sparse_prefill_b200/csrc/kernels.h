@@ -24,7 +24,8 @@ struct SetupArgs {
     int64_t max_blocks;
     int32_t nb_cap;  // >= blocks of the longest request (histogram bins)
     // attention call: order the (q-block, KV head) work items by their cost
-    // (kept tiles + correction tiles), heaviest first; NULL: blocks by index
+    // (kept tiles + correction tiles), heaviest first; NULL (the estimator
+    // call): no work order
     const int32_t* kept_cnt;   // [max_blocks, hkv]
     int32_t hkv;
     int32_t correction;
@@ -34,13 +35,13 @@ struct SetupArgs {
     int32_t* cu_tiles;    // estimator tiles of q-blocks
     int32_t* blk_req;     // request of every key block
     int32_t* blk_req_q;   // request of every q-block
-    int32_t* order;  // kept_cnt == NULL: global q-blocks; else codes t * hkv + g (t a q-block)
+    int32_t* order;  // codes t * hkv + g (t a q-block), heaviest first (attention call)
 };
 
-// Histogram bins of the setup kernel: block index (< nb_cap) or item cost
-// (kept tiles <= nb_cap, correction tiles <= ceil(nb_cap / 128), fill 2).
+// Histogram bins of the setup kernel's cost order (kept tiles <= nb_cap,
+// correction tiles <= ceil(nb_cap / 128), fill 2); the estimator call has none.
 __host__ __device__ inline int32_t setup_bins(int32_t nb_cap, bool cost) {
-    return cost ? nb_cap + (nb_cap + 127) / 128 + 3 : nb_cap;
+    return cost ? nb_cap + (nb_cap + 127) / 128 + 3 : 0;
 }
 
 struct PoolArgs {

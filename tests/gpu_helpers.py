@@ -12,6 +12,10 @@ from oracle.oracle import Oracle, chunk_starts, near_threshold
 
 BF16_MAX_ABS, BF16_MEAN_ABS = 2e-2, 2e-3
 E4M3_MAX_ABS = 6e-2
+# e4m3 mean-abs: not fixed by the stated tolerances; taken with the bf16 bounds' ratio
+# (mean-abs = max-abs / 10), which catches a systematic bias of the e4m3 correction
+# operands (block means rounded to e4m3) that the max-abs bound alone would let through
+E4M3_MEAN_ABS = 6e-3
 
 _ORC = None
 
@@ -74,7 +78,7 @@ def run_gpu(wl, alpha=None, correction=True, paged=False, scores=False, lse=True
         "kept_idx": meta.kept_idx[:nblk].cpu().numpy(),
         "k_mean": meta.k_mean[:nblk].cpu().numpy(),
         "v_mean": meta.v_mean[:nblk].cpu().numpy(),
-        "k_var": meta.k_var[:nblk].cpu().numpy(),
+        "k_var": meta.k_var[:nblk].cpu().numpy() if meta.k_var is not None else None,
         "o": out.float().cpu().numpy(),
         "lse": lse_t.cpu().numpy() if lse else None,
         "score_dbg": meta.score_dbg[:nblk].cpu().numpy() if scores else None,

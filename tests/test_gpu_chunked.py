@@ -13,7 +13,8 @@ import os
 import numpy as np
 import pytest
 
-from gpu_helpers import (BF16_MAX_ABS, BF16_MEAN_ABS, E4M3_MAX_ABS, check_mask_counts, chunk_block_index,
+from gpu_helpers import (BF16_MAX_ABS, BF16_MEAN_ABS, E4M3_MAX_ABS, E4M3_MEAN_ABS, check_mask_counts,
+                         chunk_block_index,
                          chunk_rows_of_blocks, compare_masks, oracle, out_errors, record_output_errors, run_gpu,
                          run_gpu_chunked, sample_blocks)
 from workloads import make_chunked_workload, make_workload
@@ -41,7 +42,8 @@ def _check(wl, g, sel=None, e4m3=False):
     record_output_errors(_label(), mx, mn)
     lm, _ = out_errors(g["lse"], ref["lse"], rows)
     if e4m3:
-        assert mx <= E4M3_MAX_ABS and lm < E4M3_MAX_ABS, f"max-abs {mx:.3e} lse {lm:.3e}"
+        assert mx <= E4M3_MAX_ABS and mn <= E4M3_MEAN_ABS and lm < E4M3_MAX_ABS, \
+            f"max-abs {mx:.3e} mean-abs {mn:.3e} lse {lm:.3e}"
     else:
         assert mx <= BF16_MAX_ABS and mn <= BF16_MEAN_ABS and lm < 2e-2, \
             f"max-abs {mx:.3e} mean-abs {mn:.3e} lse {lm:.3e}"
