@@ -307,10 +307,10 @@ def sparse_prefill_noalloc(params: Params, q, k, v, cu_seqlens, max_seqlen: int,
            "fp2_sparse_prefill_noalloc")
 
 
-def _chunk_args(params: Params, where: str, q, k, v, cu_q, cu_k, out=None, lse=None, block_table=None,
-                num_pages: int = 0):
+def _chunk_args(params: Params, where: str, q, k, v, cu_q, cu_k, total_k: int, out=None, lse=None,
+                block_table=None, num_pages: int = 0):
     """Layouts of a chunked call: q / out / lse [total_q, ...], k / v [total_k, Hkv, d] (or page
-    pools), cu_seqlens_q and cu_seqlens_k [batch + 1] int32."""
+    pools), cu_seqlens_q and cu_seqlens_k [batch + 1] int32; then the device."""
     for name, t in (("cu_seqlens_q", cu_q), ("cu_seqlens_k", cu_k)):
         if t is None:
             raise TypeError(f"{where}: {name} is required")
@@ -331,6 +331,8 @@ def _chunk_args(params: Params, where: str, q, k, v, cu_q, cu_k, out=None, lse=N
     Tq = int(q.shape[0])
     _arg(out, "out", (torch.bfloat16,), (Tq, hq, d), where)
     _arg(lse, "lse", (torch.float32,), (Tq, hq), where)
+    if block_table is None and int(total_k) != int(k.shape[0]):
+        raise ValueError(f"{where}: total_k = {total_k} but k has {k.shape[0]} rows")
     _same_cuda(where, q=q, k=k, v=v, cu_seqlens_q=cu_q, cu_seqlens_k=cu_k, out=out, lse=lse,
                block_table=block_table, q_scale=params.q_scale, k_scale=params.k_scale, v_scale=params.v_scale)
 
@@ -342,9 +344,8 @@ def estimate_chunked(params: Params, q, k, v, cu_seqlens_q, cu_seqlens_k, total_
     means of all keys) into ``meta``.  ``total_k`` = cu_seqlens_k[-1] (the keys of the
     batch; with contiguous K/V, k.shape[0])."""
     where = "fp2_estimate_chunked"
-    _chunk_args(params, where, q, k, v, cu_seqlens_q, cu_seqlens_k, block_table=block_table, num_pages=num_pages)
-    if block_table is None and int(total_k) != int(k.shape[0]):
-        raise ValueError(f"{where}: total_k = {total_k} but k has {k.shape[0]} rows")
+    _chunk_args(params, where, q, k, v, cu_seqlens_q, cu_seqlens_k, total_k, block_table=block_table,
+                num_pages=num_pages)
     p, m = params.c(), meta.c()
     bt, mbps, npg = _bt_args(block_table, num_pages)
     _check(_lib.load().fp2_estimate_chunked(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens_q),
@@ -360,9 +361,7 @@ def prefill_chunked(params: Params, q, k, v, cu_seqlens_q, cu_seqlens_k, total_k
     """``fp2_prefill_chunked``: attention of the chunk rows over the kept blocks of all
     keys (+ mean correction), contiguous K/V or page pools through ``block_table``."""
     where = "fp2_prefill_chunked"
-    _chunk_args(params, where, q, k, v, cu_seqlens_q, cu_seqlens_k, out, lse, block_table, num_pages)
-    if block_table is None and int(total_k) != int(k.shape[0]):
-        raise ValueError(f"{where}: total_k = {total_k} but k has {k.shape[0]} rows")
+    _chunk_args(params, where, q, k, v, cu_seqlens_q, cu_seqlens_k, total_k, out, lse, block_table, num_pages)
     p, m = params.c(), meta.c()
     bt, mbps, npg = _bt_args(block_table, num_pages)
     _check(_lib.load().fp2_prefill_chunked(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens_q),

@@ -168,3 +168,42 @@ def test_e4m3_scales_are_required_and_checked(e4m3):
     p.v_scale = p.v_scale.double()
     with pytest.raises(TypeError, match="v_scale has dtype"):
         fp2.sparse_prefill(p, e4m3.q, e4m3.k, e4m3.v, cu, e4m3.max_seqlen, None, out, None)
+
+
+@pytest.fixture(scope="module")
+def chunk():
+    from workloads.synthetic import make_chunked_workload
+    return make_chunked_workload([300, 200], [100, 200], 8, 2, alpha=0.1, seed=3, paged=True)
+
+
+def test_well_formed_chunk_arguments_reach_the_device_check(chunk):
+    p = _params(chunk)
+    cu_q, cu_k = torch.from_numpy(chunk.cu_seqlens_q), torch.from_numpy(chunk.cu_seqlens)
+    Tq, Tk = chunk.total_queries, chunk.total_tokens
+    out = torch.zeros((Tq, 8, 128), dtype=torch.bfloat16)
+    lse = torch.zeros((Tq, 8), dtype=torch.float32)
+    bt = torch.from_numpy(chunk.block_table)
+    with pytest.raises(ValueError, match=CPU_MSG):
+        fp2.estimate_chunked(p, chunk.q, chunk.k, chunk.v, cu_q, cu_k, Tk, chunk.max_seqlen, None, None)
+    with pytest.raises(ValueError, match=CPU_MSG):
+        fp2.prefill_chunked(p, chunk.q, chunk.k, chunk.v, cu_q, cu_k, Tk, chunk.max_seqlen, None, out, None,
+                            lse=lse)
+    with pytest.raises(ValueError, match=CPU_MSG):
+        fp2.prefill_chunked(p, chunk.q, chunk.k_pool, chunk.v_pool, cu_q, cu_k, Tk, chunk.max_seqlen, None, out,
+                            None, lse=lse, block_table=bt, num_pages=chunk.num_pages)
+
+
+def test_malformed_chunk_arguments_are_named(chunk):
+    p = _params(chunk)
+    cu_q, cu_k = torch.from_numpy(chunk.cu_seqlens_q), torch.from_numpy(chunk.cu_seqlens)
+    Tq, Tk = chunk.total_queries, chunk.total_tokens
+    out = torch.zeros((Tq, 8, 128), dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="same batch"):
+        fp2.prefill_chunked(p, chunk.q, chunk.k, chunk.v, cu_q[:-1], cu_k, Tk, chunk.max_seqlen, None, out, None)
+    with pytest.raises(ValueError, match="total_k"):
+        fp2.estimate_chunked(p, chunk.q, chunk.k, chunk.v, cu_q, cu_k, Tk + 1, chunk.max_seqlen, None, None)
+    with pytest.raises(ValueError, match="out has shape"):
+        fp2.prefill_chunked(p, chunk.q, chunk.k, chunk.v, cu_q, cu_k, Tk, chunk.max_seqlen, None,
+                            torch.zeros((Tk, 8, 128), dtype=torch.bfloat16), None)
+    with pytest.raises(TypeError, match="cu_seqlens_k has dtype"):
+        fp2.estimate_chunked(p, chunk.q, chunk.k, chunk.v, cu_q, cu_k.long(), Tk, chunk.max_seqlen, None, None)
