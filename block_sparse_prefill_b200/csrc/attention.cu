@@ -10,10 +10,15 @@
 //   o_r = [sum_{kept c <= r} e^{l_c} v_c + sum_{pruned j<i} 128 e^{lbar_j} vbar_j]
 //       / [sum_{kept c <= r} e^{l_c}     + sum_{pruned j<i} 128 e^{lbar_j}]
 // with l_c = tau q_r . k_c and lbar_j = tau q_r . kbar_j (pruned blocks are full).
+// With correction 2 each pruned block's lbar_j also gets (tau^2 / 2) |q_r|^2 kvar_j,
+// kvar_j its key variance averaged over the dimensions.  Chunked prefill: the
+// q-blocks keep the request's absolute grid, so only the Q tile's row offset and
+// the rows the epilogue stores change.
 //
 // Structure: persistent, one CTA per SM.  A work item is one q-block x two query
 // heads of one KV head, so every K/V tile fetched into shared memory serves both
-// heads; the CTA takes items from a counter in the workspace, longest first.
+// heads; the CTA takes items from a counter in the workspace, in the order the
+// setup kernel wrote: most tiles first.
 //   warpgroup 0 (warps 0-3)  softmax of Q tile 0 (one thread per row = TMEM lane)
 //   warpgroup 1 (warps 4-7)  softmax of Q tile 1
 //   warpgroup 2: warp 8      TMA producer: Q tiles, then K/V (or mean-K/mean-V)

@@ -96,3 +96,26 @@ def test_16k_chunk_of_a_128k_request_sampled():
     nq = g["kept_cnt"].shape[0]
     sel = sample_blocks(nq, 16, seed=5, include=(0, nq - 1))
     _check(wl, g, sel=sel)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "e4m3"])
+def test_chunks_with_the_variance_term(dtype):
+    """correction = 2 on chunks (paged): the oracle's isotropic variance mode with the key
+    variances of all keys, the cached prefix's pruned blocks included."""
+    wl = make_chunked_workload(SEQLENS, QUERY_LENS, 8, 2, alpha=0.1, seed=55, dtype=dtype, paged=True)
+    g = run_gpu_chunked(wl, paged=True, correction=2)
+    orc = oracle()
+    q, k, v = wl.float_inputs()
+    cu_q, cu_k = wl.cu_seqlens_q, wl.cu_seqlens
+    kbar = orc.block_means(k, cu_k, 128, wl.k_scale)
+    vbar = orc.block_means(v, cu_k, 128, wl.v_scale)
+    kvar = orc.block_vars(k, cu_k, 128, kbar, wl.k_scale)
+    ref = orc.attend(q, k, v, cu_q, 128, 1.0 / np.sqrt(128.0), g["kept_cnt"], g["kept_idx"], correction=4,
+                     kbar=kbar, vbar=vbar, kvar=kvar, q_scale=wl.q_scale, k_scale=wl.k_scale,
+                     v_scale=wl.v_scale, cu_seqlens_k=cu_k)
+    mx, mn = out_errors(g["o"], ref["o"])
+    record_output_errors(_label(), mx, mn)
+    if dtype == "bf16":
+        assert mx <= BF16_MAX_ABS and mn <= BF16_MEAN_ABS, f"max-abs {mx:.3e} mean-abs {mn:.3e}"
+    else:
+        assert mx <= E4M3_MAX_ABS and mn <= E4M3_MEAN_ABS, f"max-abs {mx:.3e} mean-abs {mn:.3e}"
