@@ -108,7 +108,7 @@ def test_llama_shape_32k_sweep(alpha):
     g = run_gpu(wl)
     _check_masks(wl, g)
     nblk = g["kept_cnt"].shape[0]
-    sel = sample_blocks(nblk, 24, seed=int(alpha * 1000), include=(0, nblk - 1))
+    sel = sample_blocks(nblk, 32, seed=int(alpha * 1000), include=(0, nblk - 1))
     _check_outputs(wl, g, True, sel=sel)
 
 
@@ -117,7 +117,7 @@ def test_128k_bf16_sampled():
     g = run_gpu(wl)
     _check_masks(wl, g)
     nblk = g["kept_cnt"].shape[0]
-    sel = sample_blocks(nblk, 48, seed=2, include=(0, nblk - 1))
+    sel = sample_blocks(nblk, 64, seed=2, include=(0, nblk - 1))
     _check_outputs(wl, g, True, sel=sel)
 
 
@@ -133,7 +133,7 @@ def test_128k_e4m3_sampled():
     g = run_gpu(wl)
     _check_masks(wl, g)
     nblk = g["kept_cnt"].shape[0]
-    sel = sample_blocks(nblk, 48, seed=3, include=(0, nblk - 1))
+    sel = sample_blocks(nblk, 64, seed=3, include=(0, nblk - 1))
     _check_outputs(wl, g, True, sel=sel, max_abs=E4M3_MAX_ABS, mean_abs=E4M3_MEAN_ABS, lse_abs=E4M3_MAX_ABS)
 
 
