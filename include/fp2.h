@@ -44,7 +44,8 @@
  * Ownership: every pointer passed to a compute call is a DEVICE pointer owned
  * by the caller, except the fp2_params / fp2_blockmeta structs themselves,
  * which are read on the host during the call.  The library allocates no memory
- * and keeps no global state; scratch memory is the caller's workspace.
+ * and keeps no global state; scratch memory is the caller's workspace (the one
+ * exception, fp2_sparse_prefill_noalloc, uses a static device array instead).
  * Alignment: q, k, v (or the pools), out, k_mean and v_mean start on 16-byte
  * boundaries (TMA operands and 16-byte accesses), lse on 4 bytes, the workspace
  * on 256 bytes; otherwise the call returns FP2_ERR_INVALID_ARG (FP2_ERR_WORKSPACE
