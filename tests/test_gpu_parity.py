@@ -264,3 +264,23 @@ def test_variance_correction_32k_sampled():
     nblk = g["kept_cnt"].shape[0]
     sel = sample_blocks(nblk, 12, seed=21, include=(0, nblk - 1))
     _check_variance(wl, g, sel=sel)
+
+
+def test_many_short_requests():
+    """200 requests of 1-300 tokens (seeded) in one batch: many requests per score tile
+    and per setup pass, tiny diagonal-only items, the cost order over all of them."""
+    rng = np.random.default_rng(71)
+    lens = [int(x) for x in rng.integers(1, 301, size=200)]
+    wl = make_workload(lens, 8, 2, alpha=0.1, seed=71, n_retrieval=1)
+    g = run_gpu(wl)
+    _check_masks(wl, g)
+    _check_outputs(wl, g, True)
+
+
+def test_eight_query_heads_per_kv_head():
+    """G = 8 (Hq = 16, Hkv = 2): four work items per (q-block, KV head), a score tile of 16
+    q-blocks whose 8 rows per q-block meet in warp shuffles."""
+    wl = make_workload([1500, 700, 1], 16, 2, alpha=0.1, seed=72, n_retrieval=1)
+    g = run_gpu(wl)
+    _check_masks(wl, g)
+    _check_outputs(wl, g, True)
