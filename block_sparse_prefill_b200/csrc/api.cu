@@ -405,6 +405,7 @@ fp2_status run_attention(const fp2_params* p, const void* q, const void* k, cons
     a.k_scale = p->k_scale;
     a.v_scale = p->v_scale;
     a.out = out;
+    a.out_align32 = aligned(out, 32) ? 1 : 0;
     a.lse = lse;
     a.hdr = hdr;
     return launched(launch_attention(e4m3, a, tq, tk, tv, tkb, tvb, pr.max_qblocks, s));

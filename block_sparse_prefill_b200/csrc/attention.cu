@@ -829,10 +829,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                         for (int c = 0; c < 16; ++c)
                             pk[c] = pack_bf16(__uint_as_float(ov[2 * c]) * inv,
                                               __uint_as_float(ov[2 * c + 1]) * inv);
-                        uint4* dst = reinterpret_cast<uint4*>(orow + c0);
+                        // each thread writes its own row: with 32-byte stores a warp's
+                        // store covers whole sectors of 32 rows, half as many requests
+                        // as with 16-byte ones (the epilogue is bound by those requests)
+                        if (a.out_align32) {
+                            st_global_v8(orow + c0, pk);
+                            st_global_v8(orow + c0 + 16, pk + 8);
+                        } else {
+                            uint4* dst = reinterpret_cast<uint4*>(orow + c0);
 #pragma unroll
-                        for (int c = 0; c < 4; ++c)
-                            dst[c] = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+                            for (int c = 0; c < 4; ++c)
+                                dst[c] = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+                        }
                     }
                 }
                 if (a.lse && store) {

@@ -126,6 +126,8 @@ struct AttnArgs {
     const float* k_scale;
     const float* v_scale;
     void* out;                   // bf16 [T, Hq, d]
+    int32_t out_align32;         // 1: out is 32-byte aligned (each output row is then
+                                 // written with 256-bit stores, else 128-bit ones)
     float* lse;                  // [T, Hq] or NULL
     WsHeader* hdr;
 };

@@ -38,18 +38,23 @@ def params_for(wl, alpha=None, correction=True, dev="cuda"):
     return p
 
 
-def run_gpu(wl, alpha=None, correction=True, paged=False, scores=False, lse=True, dev="cuda", kept=None):
+def run_gpu(wl, alpha=None, correction=True, paged=False, scores=False, lse=True, dev="cuda", kept=None,
+            out_shift=0):
     """Estimator + attention on the GPU.  Returns numpy arrays.  With ``kept``
     (dict of kept_cnt / kept_idx numpy arrays, e.g. the oracle's) the attention
     runs on those lists instead of the estimator's (the block means still come
-    from the estimator)."""
+    from the estimator).  ``out_shift`` places the output ``out_shift`` bf16
+    elements past the start of its allocation (8: 16-byte but not 32-byte aligned)."""
     params = params_for(wl, alpha, correction, dev)
     T, B = wl.total_tokens, wl.batch
     cu = torch.from_numpy(wl.cu_seqlens).to(dev)
     q = wl.q.to(dev)
     meta = fp2.BlockMeta.empty(params, B, T, wl.max_seqlen, dev, scores=scores)
     ws = fp2.Workspace(params, B, T, wl.max_seqlen, dev)
-    out = torch.full((T, wl.num_q_heads, 128), float("nan"), dtype=torch.bfloat16, device=dev)
+    n_out = T * wl.num_q_heads * 128
+    out_buf = torch.full((n_out + 16,), float("nan"), dtype=torch.bfloat16, device=dev)
+    out = out_buf[out_shift:out_shift + n_out].view(T, wl.num_q_heads, 128)
+    assert out_shift != 8 or out.data_ptr() % 32 == 16
     lse_t = torch.full((T, wl.num_q_heads), float("nan"), dtype=torch.float32, device=dev) if lse else None
     def given_mask():
         if kept is not None:

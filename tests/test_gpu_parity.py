@@ -146,6 +146,21 @@ def test_paged_equals_contiguous_small():
     _check_outputs(wl, gp, True)
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "e4m3"])
+def test_output_16_byte_aligned(dtype):
+    """An output that is 16- but not 32-byte aligned (the ABI's minimum) takes the
+    epilogue's 128-bit stores; it holds the same bytes as a 32-byte aligned one."""
+    wl = make_workload([900, 130, 2000, 1], 8, 2, alpha=0.1, seed=43, dtype=dtype)
+    g16 = run_gpu(wl, out_shift=8)
+    g32 = run_gpu(wl, out_shift=0)
+    assert np.array_equal(g16["o"], g32["o"], equal_nan=True), "output depends on its alignment"
+    assert np.array_equal(g16["lse"], g32["lse"], equal_nan=True)
+    if dtype == "bf16":
+        _check_outputs(wl, g16, True)
+    else:
+        _check_outputs(wl, g16, True, max_abs=E4M3_MAX_ABS, mean_abs=E4M3_MEAN_ABS, lse_abs=E4M3_MAX_ABS)
+
+
 def test_e4m3_paged_equals_contiguous():
     """e4m3 page pools (the pooling kernel's byte-wide TMA boxes over pages) give the masks
     and the output of the contiguous e4m3 path, which matches the oracle."""
