@@ -694,9 +694,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int wi = 0; wi < 4; ++wi) {
                         const uint32_t bits = (w0 + wi < nwords) ? pruned[w0 + wi] : 0u;
+                        // (the same word for the whole warp: most words of a correction
+                        // tile are all pruned, and those need no per-column test)
+                        if (bits != 0xffffffffu) {
 #pragma unroll
-                        for (int c = 0; c < 32; ++c)
-                            if (!((bits >> c) & 1u)) sv[wi * 32 + c] = __float_as_uint(-INFINITY);
+                            for (int c = 0; c < 32; ++c)
+                                if (!((bits >> c) & 1u)) sv[wi * 32 + c] = __float_as_uint(-INFINITY);
+                        }
                     }
                 }
                 // a correction column stands for the 128 keys of a pruned block: its
