@@ -37,9 +37,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 E4M3_OVER_BF16 = 2.0  # nominal dense ratio (4.5 / 2.25 PFLOP/s)
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch of the 128K bf16 layer's
 # kernels, from one single-pass ncu capture each of the kernels as they stand (attention:
-# 6.40 GB read + 1.06 GB written; pooling: 1.61 GB + 0.03 GB).  Reported only for that
+# 6.29 GB read + 1.07 GB written; pooling: 1.61 GB + 0.03 GB).  Reported only for that
 # workload; to be captured again whenever these kernels change.
-TRAFFIC_128K = {"attention": 7.47e9, "pool": 1.64e9}
+TRAFFIC_128K = {"attention": 7.36e9, "pool": 1.64e9}
 
 
 def load_peaks():

@@ -683,7 +683,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                 //   diagonal block (n == 0): keys c <= r
                 //   kept block: every key
                 //   correction tile: pruned block means only, weighted by 128
-                if (n == 0) {
+                if (n == 0 && kE4M3) {
+                    // warp w % 4 holds rows [32 (w % 4), 32 (w % 4) + 32): only that
+                    // column block needs a per-element test; the blocks right of it are
+                    // masked whole, those left of it not at all (uniform branches).
+                    // Measured at 128K: e4m3 1.8% faster than the per-element form
+                    // below, bf16 1% slower, so bf16 keeps that one.
+                    const int wq = warp & 3;
+#pragma unroll
+                    for (int cb = 0; cb < 4; ++cb) {
+                        if (cb == wq) {
+#pragma unroll
+                            for (int c = 0; c < 32; ++c)
+                                if (32 * cb + c > r) sv[32 * cb + c] = __float_as_uint(-INFINITY);
+                        } else if (cb > wq) {
+#pragma unroll
+                            for (int c = 0; c < 32; ++c) sv[32 * cb + c] = __float_as_uint(-INFINITY);
+                        }
+                    }
+                } else if (n == 0) {
 #pragma unroll
                     for (int c = 0; c < 128; ++c)
                         if (c > r) sv[c] = __float_as_uint(-INFINITY);
