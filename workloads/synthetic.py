@@ -190,10 +190,10 @@ def _request_tensors(rng, L, hq, hkv, d, bs, n_retrieval, lam, u):
 def quantize_e4m3(x: torch.Tensor):
     """Per-head absmax scaling to e4m3.  x: [T, H, d] float. Returns (codes, scale[H])."""
     xf = x.float()
-    amax = xf.abs().amax(dim=(0, 2)) if xf.shape[0] > 0 else torch.zeros(xf.shape[1])
+    amax = xf.abs().amax(dim=(0, 2)) if xf.shape[0] > 0 else torch.zeros(xf.shape[1], device=xf.device)
     scale = torch.where(amax > 0, amax / E4M3_MAX, torch.ones_like(amax))
     codes = (xf / scale[None, :, None]).clamp(-E4M3_MAX, E4M3_MAX).to(torch.float8_e4m3fn)
-    return codes, scale.numpy().astype(np.float32)
+    return codes, scale.cpu().numpy().astype(np.float32)
 
 
 def page_kv(k: torch.Tensor, v: torch.Tensor, seqlens, bs: int, rng):
