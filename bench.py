@@ -579,6 +579,11 @@ def cpu_baseline(wl, n_sample=64, shift=0, gpu_kept=None):
     nblk = est["kept_cnt"].shape[0]
     pts = np.linspace(0, nblk - 1, n_sample + 2)[1:-1]
     sel = np.unique((np.round(pts).astype(np.int64) + shift) % nblk)
+    # untimed warm-up on one q-block: the first call pays the page faults of the
+    # full-size output array (seconds for GBs), a per-process cost that the
+    # extrapolation by work share would otherwise multiply
+    orc.attend(q, k, v, cu, 128, tau, est["kept_cnt"], est["kept_idx"], correction=True,
+               kbar=kb, vbar=vb, q_scale=wl.q_scale, k_scale=wl.k_scale, v_scale=wl.v_scale, sel=sel[:1])
     t1 = time.perf_counter()
     orc.attend(q, k, v, cu, 128, tau, est["kept_cnt"], est["kept_idx"], correction=True,
                kbar=kb, vbar=vb, q_scale=wl.q_scale, k_scale=wl.k_scale, v_scale=wl.v_scale, sel=sel)
