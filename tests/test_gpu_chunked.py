@@ -88,14 +88,17 @@ def test_chunk_paged_on_the_oracle_mask():
     assert mx <= BF16_MAX_ABS and mn <= BF16_MEAN_ABS
 
 
-def test_16k_chunk_of_a_128k_request_sampled():
+@pytest.mark.parametrize("dtype,paged", [("bf16", False), ("e4m3", True)])
+def test_16k_chunk_of_a_128k_request_sampled(dtype, paged):
     """The last 16384 rows of the 128K Llama-3-8B-shaped layer (Hq=32, Hkv=8, alpha=0.05,
-    the 128K layer's planted structure): every kept list, outputs on 16 q-blocks."""
-    wl = make_chunked_workload([131072], [16384], 32, 8, alpha=0.05, seed=1002, n_retrieval=16)
-    g = run_gpu_chunked(wl)
+    the 128K layer's planted structure): every kept list, outputs on 16 q-blocks; in bf16
+    on contiguous K/V, in e4m3 on a page pool of the 128K keys."""
+    wl = make_chunked_workload([131072], [16384], 32, 8, alpha=0.05, seed=1002, n_retrieval=16, dtype=dtype,
+                               paged=paged)
+    g = run_gpu_chunked(wl, paged=paged)
     nq = g["kept_cnt"].shape[0]
     sel = sample_blocks(nq, 16, seed=5, include=(0, nq - 1))
-    _check(wl, g, sel=sel)
+    _check(wl, g, sel=sel, e4m3=dtype == "e4m3")
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "e4m3"])
